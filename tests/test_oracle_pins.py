@@ -1,0 +1,411 @@
+"""Pins of the fp64 oracle against facts that do not come from the oracle.
+
+Each test ties one part of the oracle to something fixed independently: a
+value a source page prints (fixtures under tests/golden/), a closed form, a
+special case that reduces to a library routine, the joint softmax written out
+the long way, or an invariant. They are chosen so that a plausible slip in the
+oracle (an off-by-one window bound, a dropped sink or window term, a wrong
+causal rule, a transposed operand, a sign error in the gradient) fails one.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+from scipy.special import logsumexp
+
+import oracle
+import synth
+from tests.longway import FLT_MIN, target_long_way
+
+GOLD = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _gold(name):
+    with open(os.path.join(GOLD, name)) as f:
+        return json.load(f)
+
+
+def _f64(bits):
+    return synth.bf16_to_f32(bits).astype(np.float64)
+
+
+def _rand_problem(seed, B=1, S=32, H=3, D=16, K=6, cr=4, W=5, docs=False, sink=True, scatter=True):
+    rng = np.random.default_rng(seed)
+    Q = synth.bf16_bits(rng.standard_normal((B, S, H, D), dtype=np.float32))
+    Kw = synth.bf16_bits(rng.standard_normal((B, S, D), dtype=np.float32))
+    P = S // cr
+    pool = synth.bf16_bits(rng.standard_normal((B, P, D), dtype=np.float32))
+    snk = rng.standard_normal(H).astype(np.float32) if sink else None
+    ds = None
+    if docs:
+        ds = np.zeros((B, S), dtype=np.int32)
+        for b in range(B):
+            s0 = int(rng.integers(1, S))
+            ds[b, s0:] = s0
+    # indices over the whole pool (some non-causal, so masked) plus -1 scattered
+    idx = rng.integers(0, P, size=(B, S, K)).astype(np.int32)
+    if scatter:
+        idx[rng.random((B, S, K)) < 0.25] = -1
+    for b in range(B):
+        for t in range(S):
+            # keep the selected rows distinct
+            seen = set()
+            for k in range(K):
+                if idx[b, t, k] in seen:
+                    idx[b, t, k] = -1
+                elif idx[b, t, k] >= 0:
+                    seen.add(int(idx[b, t, k]))
+    return Q, Kw, pool, idx, snk, ds
+
+
+# ---------------------------------------------------------------- window_lse
+
+def test_window_single_key_is_the_logit():
+    """W = 1: the window is the token itself, so the log-mass is its one logit."""
+    Q, Kw, *_ = _rand_problem(1, B=2, S=16, H=3, D=16)
+    scale = 0.25
+    wl = oracle.window_lse(Q, Kw, None, 1, scale)
+    q, k = _f64(Q), _f64(Kw)
+    expect = scale * np.einsum("bthd,btd->bth", q, k).reshape(-1, 3)
+    np.testing.assert_allclose(wl, expect, rtol=0, atol=1e-13)
+
+
+@pytest.mark.parametrize("W", [1, 3, 7, 40])
+def test_window_zero_queries_counts_keys(W):
+    """q = 0: every logit is 0, so the log-mass is log(number of window keys),
+    min(W, t - d0 + 1) with the document start d0."""
+    S, H, D = 24, 2, 8
+    Q = np.zeros((2, S, H, D), dtype=np.uint16)
+    Kw = synth.bf16_bits(np.random.default_rng(2).standard_normal((2, S, D), dtype=np.float32))
+    ds = np.zeros((2, S), dtype=np.int32)
+    ds[1, 9:] = 9
+    wl = oracle.window_lse(Q, Kw, ds, W, 0.5).reshape(2, S, H)
+    for b in range(2):
+        for t in range(S):
+            d0 = ds[b, t]
+            n = min(W, t - d0 + 1)
+            assert wl[b, t, 0] == pytest.approx(math.log(n), abs=1e-14)
+            assert wl[b, t, 1] == pytest.approx(math.log(n), abs=1e-14)
+
+
+def test_window_covering_sequence_is_causal_lse():
+    """W >= S: the window is the whole causal prefix; compare with scipy's
+    logsumexp over the masked matmul logits."""
+    Q, Kw, *_ = _rand_problem(3, B=1, S=20, H=2, D=8)
+    scale = 0.3
+    wl = oracle.window_lse(Q, Kw, None, 64, scale).reshape(20, 2)
+    q, k = _f64(Q)[0], _f64(Kw)[0]
+    z = scale * np.einsum("thd,sd->ths", q, k)
+    for t in range(20):
+        np.testing.assert_allclose(wl[t], logsumexp(z[t, :, :t + 1], axis=1), rtol=0, atol=1e-12)
+
+
+def test_window_batches_are_independent():
+    """Two identical batch rows give identical results (batch offset b*S)."""
+    Q, Kw, *_ = _rand_problem(4, B=1, S=12, H=2, D=8)
+    Q2, K2 = np.concatenate([Q, Q]), np.concatenate([Kw, Kw])
+    wl = oracle.window_lse(Q2, K2, None, 4, 0.5).reshape(2, 12, 2)
+    np.testing.assert_array_equal(wl[0], wl[1])
+
+
+def test_window_token_sample_matches_full():
+    Q, Kw, *_ = _rand_problem(5, B=2, S=16, H=2, D=8)
+    full = oracle.window_lse(Q, Kw, None, 5, 0.5)
+    tok = np.array([0, 3, 17, 31])
+    np.testing.assert_array_equal(oracle.window_lse(Q, Kw, None, 5, 0.5, tok), full[tok])
+
+
+# ------------------------------------------------------------ distill_target
+
+def test_causal_block_rule_golden():
+    """MaxText page: with t=4 and compress rate 4, block 0 is allowed and
+    block 1 masked. With q = 0 the target is uniform over allowed slots."""
+    g = _gold("causal_block_t4_cr4.json")
+    t, cr = g["t"], g["cr"]
+    S, H, D, K = 8, 1, 8, 2
+    Q = np.zeros((1, S, H, D), dtype=np.uint16)
+    Kw = np.zeros((1, S, D), dtype=np.uint16)
+    pool = np.zeros((1, S // cr, D), dtype=np.uint16)
+    idx = np.tile(np.array([0, 1], dtype=np.int32), (1, S, 1))
+    wl = oracle.window_lse(Q, Kw, None, 4, 1.0)
+    p, bad = oracle.distill_target(Q, pool, idx, wl, None, None, cr, 1.0)
+    p = p.reshape(S, K)
+    assert bad == 0
+    assert (p[t, 0] > 0) == g["allowed"]["0"]
+    assert (p[t, 1] > 0) == g["allowed"]["1"]
+    assert p[t, 0] == 1.0 and p[t, 1] == 0.0
+
+
+def test_zero_queries_give_uniform_target():
+    """q = 0: all logits tie, so p = 1/n_sel on the allowed slots and 0 on
+    masked ones, where n_sel counts slots with 0<=idx<P, (idx+1)*cr-1<=t and
+    idx*cr >= document start."""
+    Q, Kw, pool, idx, snk, ds = _rand_problem(6, B=2, S=32, H=3, D=8, K=7, docs=True)
+    Q[:] = 0
+    wl = oracle.window_lse(Q, Kw, ds, 5, 0.5)
+    p, bad = oracle.distill_target(Q, pool, idx, wl, snk, ds, 4, 0.5)
+    p = p.reshape(2, 32, 7)
+    for b in range(2):
+        for t in range(32):
+            d0 = ds[b, t]
+            j = idx[b, t].astype(int)
+            ok = (j >= 0) & (j < 8) & ((j + 1) * 4 - 1 <= t) & (j * 4 >= d0)
+            n = ok.sum()
+            if n == 0:
+                assert np.all(p[b, t] == 0)
+            else:
+                np.testing.assert_allclose(p[b, t][ok], 1.0 / n, rtol=1e-15)
+                assert np.all(p[b, t][~ok] == 0)
+
+
+@pytest.mark.parametrize("seed,docs,sink,W", [(10, False, True, 5), (11, True, True, 3),
+                                              (12, False, False, 9), (13, True, False, 1)])
+def test_target_matches_joint_softmax_long_way(seed, docs, sink, W):
+    Q, Kw, pool, idx, snk, ds = _rand_problem(seed, B=2, S=32, H=3, D=16, K=6, W=W, docs=docs, sink=sink)
+    scale = 1 / 4
+    wl = oracle.window_lse(Q, Kw, ds, W, scale)
+    p, bad = oracle.distill_target(Q, pool, idx, wl, snk, ds, 4, scale)
+    ref = target_long_way(Q, Kw, pool, idx, snk, ds, W, 4, scale)
+    np.testing.assert_allclose(p, ref, rtol=0, atol=1e-12)
+
+
+def test_target_long_way_on_tiny_workload():
+    w = synth.make("tiny")
+    wl = oracle.window_lse(w.Q, w.Kw, w.doc_start, w.W, w.scale)
+    p, bad = oracle.distill_target(w.Q, w.pool, w.idx, wl, w.sink, w.doc_start, w.cr, w.scale)
+    ref = target_long_way(w.Q, w.Kw, w.pool, w.idx, w.sink, w.doc_start, w.W, w.cr, w.scale)
+    assert bad == 0
+    np.testing.assert_allclose(p, ref, rtol=0, atol=1e-12)
+
+
+def test_target_long_way_on_small_workload_sample():
+    """The local-branch-dominates workload (sink +8, q aligned to the key)."""
+    w = synth.make("small")
+    tok = synth.sample_tokens(w.B, w.S, 48)
+    wl = oracle.window_lse(w.Q, w.Kw, w.doc_start, w.W, w.scale, tok)
+    p, bad = oracle.distill_target(w.Q, w.pool, w.idx, wl, w.sink, w.doc_start, w.cr, w.scale, tok)
+    ref = target_long_way(w.Q, w.Kw, w.pool, w.idx, w.sink, w.doc_start, w.W, w.cr, w.scale, tok)
+    np.testing.assert_allclose(p, ref, rtol=0, atol=1e-12)
+
+
+def test_target_per_branch_limit_is_maxtext_formula():
+    """With no sink and a window whose logits are pushed to -200, the joint
+    target reduces to the MaxText page's per-branch formula
+    L1_Normalize(Sum_h Softmax_k(z)), computed here with scipy's softmax."""
+    from scipy.special import softmax
+    Q, Kw, pool, idx, _, _ = _rand_problem(20, B=1, S=32, H=3, D=16, K=6, scatter=False)
+    # window keys = -c * q of head 0 direction makes every window logit very
+    # negative only for a single-key window whose key opposes every head: use
+    # one shared direction for all heads and keys.
+    rng = np.random.default_rng(21)
+    v = rng.standard_normal(16).astype(np.float32)
+    v /= np.linalg.norm(v)
+    qf = np.abs(rng.standard_normal((1, 32, 3, 1))).astype(np.float32) + 1.0
+    Qx = synth.bf16_bits(qf * v[None, None, None, :] * 8)
+    Kx = synth.bf16_bits(np.tile(-v * 200.0, (1, 32, 1)))
+    scale = 1.0
+    wl = oracle.window_lse(Qx, Kx, None, 1, scale)
+    assert wl.max() < -100
+    p, _ = oracle.distill_target(Qx, pool, idx, wl, None, None, 4, scale)
+    q, pl = _f64(Qx)[0], _f64(pool)[0]
+    for t in range(32):
+        j = idx[0, t].astype(int)
+        ok = (j >= 0) & ((j + 1) * 4 - 1 <= t)
+        if not ok.any():
+            continue
+        z = scale * q[t] @ pl[j[ok]].T                 # [H, n]
+        ref = softmax(z, axis=1).sum(axis=0)
+        ref = ref / ref.sum()
+        np.testing.assert_allclose(p.reshape(32, 6)[t][ok], ref, rtol=1e-9, atol=1e-12)
+
+
+def test_target_invariants():
+    Q, Kw, pool, idx, snk, ds = _rand_problem(30, B=2, S=32, H=4, D=16, K=8, docs=True)
+    scale = 0.25
+    wl = oracle.window_lse(Q, Kw, ds, 6, scale)
+    p, _ = oracle.distill_target(Q, pool, idx, wl, snk, ds, 4, scale)
+    p = p.reshape(2, 32, 8)
+    assert np.all(np.isfinite(p)) and np.all(p >= 0) and np.all(p <= 1)
+    sums = p.sum(-1)
+    nonempty = sums > 0
+    np.testing.assert_allclose(sums[nonempty], 1.0, rtol=0, atol=1e-13)
+    # slot permutation permutes p
+    perm = np.random.default_rng(31).permutation(8)
+    p2, _ = oracle.distill_target(Q, pool, idx[..., perm], wl, snk, ds, 4, scale)
+    np.testing.assert_allclose(p2.reshape(2, 32, 8), p[..., perm], rtol=0, atol=1e-15)
+    # head permutation (queries, sink and window log-mass together) leaves p
+    hp = np.array([2, 0, 3, 1])
+    wl2 = oracle.window_lse(Q[:, :, hp], Kw, ds, 6, scale)
+    np.testing.assert_array_equal(wl2, wl[:, hp])
+    p3, _ = oracle.distill_target(Q[:, :, hp], pool, idx, wl2, snk[hp], ds, 4, scale)
+    np.testing.assert_allclose(p3.reshape(2, 32, 8), p, rtol=0, atol=1e-14)
+
+
+def test_target_empty_row_and_bad_indices():
+    Q, Kw, pool, idx, snk, ds = _rand_problem(40, B=1, S=16, H=2, D=8, K=4)
+    idx[0, 5] = -1                 # empty row
+    idx[0, 9, 0] = 4               # == P: out of range
+    idx[0, 9, 1] = -7              # below -1: out of range
+    wl = oracle.window_lse(Q, Kw, ds, 4, 0.5)
+    p, bad = oracle.distill_target(Q, pool, idx, wl, snk, ds, 4, 0.5)
+    p = p.reshape(16, 4)
+    assert bad == 2
+    assert np.all(p[5] == 0)
+    assert p[9, 0] == 0 and p[9, 1] == 0
+    assert np.all(np.isfinite(p))
+
+
+@pytest.mark.parametrize("sink_val", [8.0, 40.0, 200.0])
+def test_target_local_branch_dominates(sink_val):
+    """A head whose sink and window carry almost all its attention leaves a
+    compressed mass far below 1 (about e^-40 for sink=+40, below float32 tiny
+    for sink=+200). The target stays finite, non-negative and sums to at most
+    1. At sink=+40 the mass lies between float32 tiny and the old 1e-10 floor,
+    so the row must still sum to 1: the Primus page moved the floor because
+    1e-10 would clip exactly such an almost entirely local query."""
+    Q, Kw, pool, idx, snk, ds = _rand_problem(50, B=1, S=32, H=2, D=16, K=6, scatter=False)
+    kf = _f64(Kw)
+    Qa = synth.bf16_bits((kf[:, :, None, :] + 0.1 * np.random.default_rng(51).standard_normal((1, 32, 2, 16))).astype(np.float32))
+    snk = np.full(2, sink_val, dtype=np.float32)
+    scale = 0.25
+    wl = oracle.window_lse(Qa, Kw, None, 4, scale)
+    p, _ = oracle.distill_target(Qa, pool, idx, wl, snk, None, 4, scale)
+    ref = target_long_way(Qa, Kw, pool, idx, snk, None, 4, 4, scale)
+    assert np.all(np.isfinite(p)) and np.all(p >= 0)
+    assert np.all(p.sum(-1) <= 1 + 1e-12)
+    np.testing.assert_allclose(p, ref, rtol=0, atol=1e-12)
+    if sink_val == 200.0:
+        assert p.sum(-1).max() < 1e-6
+    if sink_val == 40.0:
+        rows = p.sum(-1) > 0
+        np.testing.assert_allclose(p.sum(-1)[rows], 1.0, rtol=0, atol=1e-12)
+
+
+def test_floor_value_golden():
+    g = _gold("float32_tiny.json")
+    assert FLT_MIN == g["float32_tiny"]
+    assert float(np.finfo(np.float32).tiny) == g["float32_tiny"]
+
+
+# ----------------------------------------------------------------- distill_kl
+
+def test_kl_two_slot_closed_form():
+    """p = (1/2, 1/2), scores (0, log 3): q = (1/4, 3/4),
+    KL = 1/2 log 2 + 1/2 log(2/3) = 1/2 log(4/3); dscores = coeff (q - p)."""
+    p = np.array([[0.5, 0.5]])
+    s = np.array([[0.0, math.log(3.0)]], dtype=np.float32)
+    v = np.ones((1, 2), dtype=np.uint8)
+    loss, ds, klr = oracle.distill_kl(p, s, v, 0.01)
+    q1 = 1.0 / (1.0 + math.exp(float(s[0, 1])))
+    assert klr[0] == pytest.approx(0.5 * math.log(0.5 / q1) + 0.5 * math.log(0.5 / (1 - q1)), rel=1e-14)
+    assert klr[0] == pytest.approx(0.5 * math.log(4.0 / 3.0), rel=1e-7)
+    assert loss == pytest.approx(0.01 * klr[0], rel=1e-15)
+    np.testing.assert_allclose(ds[0], 0.01 * np.array([q1 - 0.5, (1 - q1) - 0.5]), rtol=1e-13)
+
+
+def test_kl_zero_when_scores_match_target():
+    rng = np.random.default_rng(60)
+    p = rng.random((5, 9)) + 0.05
+    p /= p.sum(1, keepdims=True)
+    s = (np.log(p) + rng.standard_normal((5, 1)))  # any per-row shift
+    v = np.ones((5, 9), dtype=np.uint8)
+    # fp32 scores carry rounding; evaluate the oracle on exactly those scores
+    s32 = s.astype(np.float32)
+    pe = np.exp(s32.astype(np.float64))
+    pe /= pe.sum(1, keepdims=True)
+    loss, ds, _ = oracle.distill_kl(pe, s32, v, 0.01)
+    assert abs(loss) < 1e-15
+    assert np.abs(ds).max() < 1e-15
+
+
+def test_kl_gradient_matches_finite_differences():
+    rng = np.random.default_rng(70)
+    R, K = 4, 7
+    p = rng.random((R, K))
+    p[0, 2] = 0.0
+    p /= p.sum(1, keepdims=True)
+    s = rng.standard_normal((R, K)) * 1.4
+    v = (rng.random((R, K)) > 0.2).astype(np.uint8)
+    v[3] = 0                                     # a row with no valid slot
+    coeff = 0.01
+
+    def loss_at(sv):
+        # fp64 scores through the float32 interface would lose the step, so
+        # the step is applied to values exactly representable in float32
+        l, _, _ = oracle.distill_kl(p, sv.astype(np.float32), v, coeff)
+        return l
+
+    s = s.astype(np.float32).astype(np.float64)
+    _, ds, _ = oracle.distill_kl(p, s.astype(np.float32), v, coeff)
+    h = 2.0 ** -12
+    for r in range(R):
+        for k in range(K):
+            sp, sm = s.copy(), s.copy()
+            sp[r, k] += h
+            sm[r, k] -= h
+            fd = (loss_at(sp) - loss_at(sm)) / (2 * h)
+            assert fd == pytest.approx(ds[r, k], rel=1e-6, abs=1e-12)
+    assert np.all(ds[3] == 0)
+    assert np.all(ds[v == 0] == 0)
+
+
+def test_kl_masked_rows_do_not_count():
+    rng = np.random.default_rng(80)
+    p = rng.random((3, 4)); p /= p.sum(1, keepdims=True)
+    s = rng.standard_normal((3, 4)).astype(np.float32)
+    v = np.ones((3, 4), dtype=np.uint8)
+    v[1] = 0
+    loss3, ds3, klr = oracle.distill_kl(p, s, v, 1.0)
+    keep = [0, 2]
+    loss2, ds2, _ = oracle.distill_kl(p[keep], s[keep], v[keep], 1.0)
+    assert klr[1] == 0.0
+    assert loss3 == pytest.approx(loss2, rel=1e-15)
+    np.testing.assert_allclose(ds3[keep], ds2, rtol=1e-15)
+
+
+def test_kl_single_slot_is_zero():
+    p = np.array([[1.0], [0.0]])
+    s = np.array([[3.0], [-2.0]], dtype=np.float32)
+    v = np.ones((2, 1), dtype=np.uint8)
+    loss, ds, _ = oracle.distill_kl(p, s, v, 0.01)
+    assert loss == 0.0
+    assert ds[0, 0] == 0.0
+
+
+def test_kl_gradient_sums_to_zero_when_target_normalised():
+    rng = np.random.default_rng(90)
+    p = rng.random((6, 10)); p /= p.sum(1, keepdims=True)
+    s = rng.standard_normal((6, 10)).astype(np.float32)
+    v = np.ones((6, 10), dtype=np.uint8)
+    _, ds, _ = oracle.distill_kl(p, s, v, 0.01)
+    np.testing.assert_allclose(ds.sum(1), 0.0, atol=1e-17)
+
+
+# ------------------------------------------------------------- the workloads
+
+def test_workload_shapes_and_indices():
+    g = _gold("v4_flash_gather.json")
+    sp = synth.CONFIGS["flash"]
+    gathered = sp.B * sp.S * sp.K * sp.D * g["dtype_bytes"]
+    assert round(gathered / 1e9, 1) == g["gathered_bytes_GB"]
+    for name in ("tiny", "small"):
+        w = synth.make(name)
+        P = w.S // w.cr
+        for b in range(w.B):
+            for t in range(w.S):
+                row = w.idx[b, t]
+                sel = row[row >= 0]
+                assert len(set(sel.tolist())) == len(sel)
+                assert np.all((sel + 1) * w.cr - 1 <= t)
+                assert len(sel) == min(w.K, (t + 1) // w.cr)
+                assert np.all(row[len(sel):] == -1)
+
+
+def test_end_to_end_oracle_finite_on_tiny():
+    w = synth.make("tiny")
+    wl, p, loss, ds, bad = oracle.run_all(w)
+    assert bad == 0
+    assert np.isfinite(loss) and loss > 0
+    assert np.all(np.isfinite(ds))
