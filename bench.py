@@ -1,0 +1,402 @@
+"""Benchmark: CSA indexer distillation loss, forward + backward, on B200.
+
+One step = sai_window_lse -> sai_distill_target -> sai_distill_kl (with
+dscores) over one batch of the V4-Flash-width workload (B=1, S=4096, H=64,
+D=512, cr=4, K=512, W=128; seeded synthetic inputs). The metric is tokens/s
+(B*S per step). Inputs are resident in HBM for `value`; `e2e` repeats the step
+through the same C-ABI calls from pinned host buffers, with the host->device
+copies of every input and the device->host copy of the loss and dscores inside
+the timed region.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Under torchrun (N > 1) every rank runs its own batch (independent problems,
+weak scaling, no collective on the data path); the time is the max over ranks.
+`--impl reference` times the fp64 CPU oracle on the host cores instead.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+WORKLOAD = "flash"
+METRIC = "distill-loss tokens/s (fwd+bwd), S=4096 H=64 K=512 D=512; % bf16 TC peak"
+UNIT = "tokens/s"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="sai", choices=["sai", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    return ap.parse_args()
+
+
+def workload_config(w, n):
+    return {
+        "workload": f"{WORKLOAD}: B={w.B} S={w.S} H={w.H} D={w.D} cr={w.cr} K={w.K} W={w.W}, "
+                    f"top-K of a random causal score, sorted ascending; bf16 Q/Kw/pool N(0,1), "
+                    f"fp32 sink N(0,1), scores N(0,2); seed 1003",
+        "global_batch": w.B * n,
+        "seq_len": w.S,
+        "parallelism": f"dp{n}" if n > 1 else "single",
+        "l2": "flushed between timed steps (256 MiB write, untimed)",
+    }
+
+
+def algorithmic_counts(w):
+    """Valid selected slots and window keys: the units behind the flop and byte
+    counts (2*H*D flops per slot or key)."""
+    t = np.arange(w.S)
+    sel = int((w.valid != 0).sum())
+    win = 0
+    for b in range(w.B):
+        d0 = np.zeros(w.S, dtype=np.int64) if w.doc_start is None else w.doc_start[b].astype(np.int64)
+        lo = np.maximum(d0, t - w.W + 1)
+        win += int((t - lo + 1).sum())
+    return sel, win
+
+
+def to_dev(w, dev):
+    import torch
+    t = {}
+    for k in ("Q", "Kw", "pool"):
+        t[k] = torch.from_numpy(getattr(w, k).view(np.int16)).to(dev).view(torch.bfloat16)
+    for k in ("idx", "sink", "doc_start", "scores", "valid"):
+        a = getattr(w, k)
+        t[k] = None if a is None else torch.from_numpy(a).to(dev)
+    return t
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d.get("bf16_tflops", 1590.0), d.get("hbm_gbs", 6650.0), "measured"
+    return 1590.0, 6650.0, "fallback"
+
+
+def traffic_record(kernel_src: str):
+    """dram bytes per launch from a committed ncu summary, if it was taken on
+    the current source of the kernel (else null)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f)
+    src = os.path.join(ROOT, "sparse_attention_indexer_window_b200", "csrc", kernel_src)
+    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    r = rec.get(kernel_src)
+    if not r or r.get("src_sha256_16") != h:
+        return None
+    return r.get("dram_bytes_per_launch")
+
+
+class Clocks:
+    """nvidia-smi sampling of SM clocks and throttle reasons while running."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_bench_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        sm, mx, reasons, n = [], None, set(), 0
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            n += 1
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": n}
+
+
+def cpu_baseline(w, seconds: float):
+    """The fp64 oracle on a bounded sample of the workload's tokens."""
+    import oracle
+    rng = np.random.default_rng(11)
+    probe = np.sort(rng.choice(w.B * w.S, size=16, replace=False))
+    t0 = time.perf_counter()
+    oracle.run_all(w, probe)
+    dt = max(time.perf_counter() - t0, 1e-3)
+    n = int(min(w.B * w.S, max(16, seconds / dt * 16)))
+    tok = np.sort(rng.choice(w.B * w.S, size=n, replace=False))
+    t0 = time.perf_counter()
+    oracle.run_all(w, tok)
+    dt = time.perf_counter() - t0
+    return {"value": n / dt, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{n} of {w.B * w.S} tokens drawn uniformly (seed 11), whole path "
+                      f"(window_lse, target, KL rows), fp64, {dt:.1f} s"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import oracle
+    import synth
+    w = synth.make(WORKLOAD)
+    per_tok = 0.0
+    probe = np.arange(w.S - 8, w.S)
+    t0 = time.perf_counter()
+    oracle.run_all(w, probe)
+    per_tok = (time.perf_counter() - t0) / len(probe)
+    budget = 150.0
+    n_per_step = int(max(1, min(w.B * w.S, budget / max(args.steps + args.warmup, 1) / max(per_tok, 1e-6))))
+    rng = np.random.default_rng(12)
+    for _ in range(args.warmup):
+        oracle.run_all(w, np.sort(rng.choice(w.B * w.S, n_per_step, replace=False)))
+    done, el = 0, 0.0
+    for _ in range(args.steps):
+        tok = np.sort(rng.choice(w.B * w.S, n_per_step, replace=False))
+        t0 = time.perf_counter()
+        oracle.run_all(w, tok)
+        el += time.perf_counter() - t0
+        done += n_per_step
+    v = done / el
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * el / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": workload_config(w, 1),
+            "cpu_baseline": {"value": v, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+                             "sample": f"{n_per_step} uniformly drawn tokens of {w.B * w.S} per step"},
+            "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+    dev = torch.device("cuda", local)
+
+    import sparse_attention_indexer_window_b200 as sai
+    import synth
+
+    w = synth.make(WORKLOAD, seed=synth.CONFIGS[WORKLOAD].seed + rank)
+    t = to_dev(w, dev)
+    B, S, H, D, K = w.B, w.S, w.H, w.D, w.K
+    wl = torch.empty((B, S, H), device=dev)
+    p = torch.empty((B, S, K), device=dev)
+    ds = torch.empty((B, S, K), device=dev)
+    loss = torch.empty(1, device=dev)
+    ws = torch.empty(sai.kl_workspace_bytes(B, S, K), dtype=torch.uint8, device=dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        sai.window_lse(t["Q"], t["Kw"], w.W, w.scale, t["doc_start"], out=wl)
+        sai.distill_target(t["Q"], t["pool"], t["idx"], wl, w.cr, w.scale, sink=t["sink"],
+                           doc_start=t["doc_start"], err=err, out=p)
+        sai.distill_kl(p, t["scores"], t["valid"], w.coeff, workspace=ws, loss=loss, dscores=ds)
+
+    for _ in range(max(args.warmup, 3)):
+        flush.fill_(1)
+        step()
+    torch.cuda.synchronize(dev)
+
+    nsteps = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(nsteps)]
+    clocks = Clocks(local)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    for i in range(nsteps):
+        flush.fill_(i & 0xFF)
+        e = ev[i]
+        e[0].record(stream)
+        sai.window_lse(t["Q"], t["Kw"], w.W, w.scale, t["doc_start"], out=wl)
+        e[1].record(stream)
+        sai.distill_target(t["Q"], t["pool"], t["idx"], wl, w.cr, w.scale, sink=t["sink"],
+                           doc_start=t["doc_start"], err=err, out=p)
+        e[2].record(stream)
+        sai.distill_kl(p, t["scores"], t["valid"], w.coeff, workspace=ws, loss=loss, dscores=ds)
+        e[3].record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    k_win = [e[0].elapsed_time(e[1]) for e in ev]
+    k_tgt = [e[1].elapsed_time(e[2]) for e in ev]
+    k_kl = [e[2].elapsed_time(e[3]) for e in ev]
+    total_ms = float(sum(e[0].elapsed_time(e[3]) for e in ev))
+    if world > 1:
+        tt = torch.tensor([total_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        total_ms = float(tt.item())
+    assert int(err.item()) == 0
+    ms_step = total_ms / nsteps
+    tokens_total = B * S * world * nsteps
+    value = tokens_total / (total_ms / 1e3)
+
+    # ---------------------------------------------------------------- e2e
+    host = {}
+    for k in ("Q", "Kw", "pool", "idx", "sink", "scores", "valid"):
+        if t[k] is not None:
+            host[k] = t[k].cpu().pin_memory()
+    out_loss = torch.empty(1).pin_memory()
+    out_ds = torch.empty((B, S, K)).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = out_loss.numel() * 4 + out_ds.numel() * 4
+    dq = {k: torch.empty_like(v, device=dev) for k, v in host.items()}
+
+    def e2e_step():
+        for k, v in host.items():
+            dq[k].copy_(v, non_blocking=True)
+        sai.window_lse(dq["Q"], dq["Kw"], w.W, w.scale, None, out=wl)
+        sai.distill_target(dq["Q"], dq["pool"], dq["idx"], wl, w.cr, w.scale, sink=dq.get("sink"),
+                           err=err, out=p)
+        sai.distill_kl(p, dq["scores"], dq["valid"], w.coeff, workspace=ws, loss=loss, dscores=ds)
+        out_loss.copy_(loss, non_blocking=True)
+        out_ds.copy_(ds, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        tt = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e_ms = float(tt.item())
+    e2e_value = B * S * world * args.e2e_steps / (e2e_ms / 1e3)
+
+    # mean loss over ranks, for the record (not part of the timed path)
+    lv = torch.tensor([float(loss.item())], device=dev, dtype=torch.float64)
+    if world > 1:
+        dist.all_reduce(lv)
+        lv /= world
+
+    if rank == 0:
+        peak_tf, hbm_gbs, peak_src = load_peaks()
+        sel, win = algorithmic_counts(w)
+        fl_tgt = 2.0 * H * D * sel
+        fl_win = 2.0 * H * D * win
+        fl_step = fl_tgt + fl_win
+        tgt_ms = statistics.mean(k_tgt)
+        win_ms = statistics.mean(k_win)
+        kl_ms = statistics.mean(k_kl)
+        achieved = fl_tgt / (tgt_ms / 1e3) / 1e12
+        # algorithmic bytes of the two HBM-bound kernels
+        win_bytes = B * S * H * D * 2 + B * S * D * 2 + B * S * H * 4
+        kl_bytes = B * S * K * (4 + 4 + 1 + 4)
+        line = {
+            "metric": METRIC,
+            "value": value,
+            "unit": UNIT,
+            "n_gpus": world,
+            "steps": nsteps,
+            "warmup": args.warmup,
+            "ms_per_step": ms_step,
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "bf16",
+            "data": "synthetic",
+            "config": workload_config(w, world),
+            "tc_peak_frac_step": fl_step / (ms_step / 1e3) / 1e12 / peak_tf,
+            "roofline": {
+                "kernel": "distill_target (target_tc_kernel<64>)",
+                "bound": "tensor",
+                "achieved": achieved,
+                "peak": peak_tf,
+                "unit": "TFLOP/s",
+                "frac": achieved / peak_tf,
+                "peak_source": f"{peak_src} bf16 dense (burst)",
+                "algorithmic": f"2*H*D flops per selected slot x {sel} selected slots = {fl_tgt:.4g} flops/launch",
+                "traffic": traffic_record("target_tc.cu"),
+            },
+            "kernels_ms": {"window_lse": win_ms, "distill_target": tgt_ms, "distill_kl": kl_ms},
+            "kernels_roofline": {
+                "window_lse": {"bound": "hbm", "achieved_gbs": win_bytes / (win_ms / 1e3) / 1e9,
+                               "peak_gbs": hbm_gbs, "frac": win_bytes / (win_ms / 1e3) / 1e9 / hbm_gbs,
+                               "tflops": fl_win / (win_ms / 1e3) / 1e12},
+                "distill_kl": {"bound": "hbm", "achieved_gbs": kl_bytes / (kl_ms / 1e3) / 1e9,
+                               "peak_gbs": hbm_gbs, "frac": kl_bytes / (kl_ms / 1e3) / 1e9 / hbm_gbs},
+            },
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "steps": args.e2e_steps},
+            "gpu_launches": 4 * nsteps,
+            "clocks": clk,
+            "loss": float(lv.item()),
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

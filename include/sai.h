@@ -1,0 +1,162 @@
+/*
+ * libsai: DeepSeek-V4 CSA lightning-indexer distillation loss on NVIDIA B200
+ * (sm_100a). C ABI.
+ *
+ * The loss is split in three calls, as on the Primus page "perf(deepseek-v4):
+ * fuse and enable the indexer distillation loss" (file table:
+ * indexer_distill_window_lse, indexer_distill_target, indexer_distill_kl):
+ *
+ *   sai_window_lse      Q, Kw            -> window_lse [B,S,H]
+ *   sai_distill_target  Q, pool, idx, window_lse, sink -> p [B,S,K]
+ *   sai_distill_kl      p, scores, valid -> loss (device scalar), dscores [B,S,K]
+ *
+ * Conventions for every call
+ *   - Tensor arguments are DEVICE pointers to dense row-major (C-contiguous)
+ *     arrays, owned by the caller. The library never allocates device memory
+ *     and never synchronises the stream.
+ *   - bf16 tensors are passed as uint16_t bit patterns.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream). All work
+ *     is enqueued on it; results are ready when the stream reaches that point.
+ *   - Host-detectable errors (NULL pointers, bad sizes, unsupported shapes,
+ *     misaligned pointers, a short workspace) return an error status before
+ *     anything is enqueued. A failed launch returns SAI_ERR_CUDA.
+ *   - Outputs are fully overwritten; masked slots are written as exact 0.
+ *   - There is no fallback to another implementation: a shape the kernels do
+ *     not cover returns SAI_ERR_UNSUPPORTED.
+ *   - Calls on the same stream are ordered; calls on different streams that
+ *     share output buffers race.
+ */
+#ifndef SAI_H
+#define SAI_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum sai_status {
+    SAI_OK = 0,
+    SAI_ERR_NULL = 1,        /* a required pointer is NULL                          */
+    SAI_ERR_SHAPE = 2,       /* a size is non-positive or sizes are inconsistent     */
+    SAI_ERR_UNSUPPORTED = 3, /* the shape is outside what the kernels cover          */
+    SAI_ERR_CUDA = 4,        /* a CUDA runtime/driver call or a launch failed        */
+    SAI_ERR_INDEX = 5,       /* device error word: an idx entry outside {-1}U[0,P)   */
+    SAI_ERR_WORKSPACE = 6,   /* workspace NULL, too small or not 16-byte aligned     */
+    SAI_ERR_ALIGN = 7,       /* a tensor pointer is not 16-byte aligned              */
+    SAI_ERR_TIMEOUT = 8      /* device error word: a kernel gave up a bounded wait   */
+} sai_status;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *sai_status_string(int status);
+
+/* Library version, major*10000 + minor*100 + patch. */
+int sai_version(void);
+
+/*
+ * sai_window_lse -- sliding-window log-mass per (token, head).
+ *
+ * Source: Primus page, second commit message ("the cost is computing the mass,
+ * a [S, window] score matrix per head ... indexer_distill_window_lse keeps the
+ * scores in registers and loads only the key band a query block spans").
+ *
+ *   window_lse[b,t,h] = log sum_{s=lo}^{t} exp(scale * <Q[b,t,h,:], Kw[b,s,:]>)
+ *   lo = max(d0, t - W + 1),  d0 = clamp(doc_start[b,t], 0, t) or 0 if NULL.
+ *
+ * The window holds W single-latent keys (one Kw row per token, shared by all
+ * heads) ending at the token itself and clipped at its document start. The
+ * per-head sink is not included (sai_distill_target adds it).
+ *
+ *   Q          [B,S,H,D] bf16, 16-byte aligned
+ *   Kw         [B,S,D]   bf16, 16-byte aligned
+ *   doc_start  [B,S] int32 or NULL (one document per row)
+ *   scale      logit scale, e.g. 1/sqrt(D)
+ *   window_lse [B,S,H] fp32, written
+ *
+ * Sizes: B,S,H,D,W >= 1 and D % 8 == 0. Errors: SAI_ERR_NULL, SAI_ERR_SHAPE,
+ * SAI_ERR_ALIGN, SAI_ERR_UNSUPPORTED, SAI_ERR_CUDA.
+ */
+sai_status sai_window_lse(const uint16_t *Q, const uint16_t *Kw, const int32_t *doc_start,
+                          int B, int S, int H, int D, int W, float scale,
+                          float *window_lse, void *stream);
+
+/*
+ * sai_distill_target -- the indexer's teacher target p[b,t,:].
+ *
+ * Source: Primus page, first commit message ("indexer_distill_target indexes
+ * the pool inside the kernel, so the gather never exists and the softmax and
+ * head sum happen in registers") and second commit message / "Why the target
+ * was wrong" (one softmax over window keys, selected compressed entries and
+ * the per-head sink; each head's share exp(compressed_lse - full_lse); floor
+ * float32 tiny). Causal block rule: MaxText page "Add Indexer Loss
+ * [Deepseek v4]", commit messages (block j is visible to token t iff
+ * (j+1)*cr - 1 <= t; cross-document blocks masked).
+ *
+ *   slot k selected iff 0 <= idx[b,t,k] < P (P = S/cr), (idx+1)*cr - 1 <= t
+ *                       and idx*cr >= d0 (d0 as in sai_window_lse)
+ *   z[h,k]      = scale * <Q[b,t,h,:], pool[b,idx[b,t,k],:]>
+ *   clse[h]     = log sum_{selected k} exp z[h,k]
+ *   lse_full[h] = logsumexp(window_lse[b,t,h], clse[h], sink[h])
+ *   u[k]        = sum_h exp(z[h,k] - lse_full[h]);   m = sum_k u[k]
+ *   p[b,t,k]    = u[k] / max(m, FLT_MIN) on selected slots, 0 elsewhere
+ *
+ *   Q          [B,S,H,D] bf16, 16-byte aligned
+ *   pool       [B,P,D]   bf16 compressed entries, 16-byte aligned
+ *   idx        [B,S,K]   int32 top-k rows, -1 = empty slot
+ *   window_lse [B,S,H]   fp32 (from sai_window_lse)
+ *   sink       [H] fp32 per-head sink logits, or NULL for no sink
+ *   doc_start  [B,S] int32 or NULL
+ *   p          [B,S,K] fp32, written
+ *   d_err      device int32 or NULL. Data errors found on the device (an idx
+ *              entry outside {-1} U [0,P)) mask the slot and store
+ *              SAI_ERR_INDEX here; the caller zeroes it and reads it back.
+ *
+ * Sizes: S % cr == 0, 1 <= K <= S/cr (the MaxText page's topk <= length/4
+ * check), D % 8 == 0. Errors: SAI_ERR_NULL, SAI_ERR_SHAPE, SAI_ERR_ALIGN,
+ * SAI_ERR_UNSUPPORTED, SAI_ERR_CUDA.
+ */
+sai_status sai_distill_target(const uint16_t *Q, const uint16_t *pool, const int32_t *idx,
+                              const float *window_lse, const float *sink, const int32_t *doc_start,
+                              int B, int S, int H, int D, int K, int cr, float scale,
+                              float *p, int32_t *d_err, void *stream);
+
+/* Bytes of device workspace sai_distill_kl needs for these sizes. */
+size_t sai_distill_kl_workspace_bytes(int B, int S, int K);
+
+/*
+ * sai_distill_kl -- KL(attention || indexer) and its gradient in one pass.
+ *
+ * Source: Primus page, first commit message ("indexer_distill_kl fuses the
+ * KL tail with an analytic backward, so nothing beyond the inputs is saved
+ * for it"); MaxText page review (log-softmax gives the exact gradient Q - P;
+ * the valid mask includes the indexer mask).
+ *
+ * Per token row over its valid slots (valid[b,t,k] != 0):
+ *   log q[k]  = scores[k] - log sum_{valid k'} exp scores[k']
+ *   KL_t      = sum_{valid k, p[k] > 0} p[k] (log p[k] - log q[k])
+ *   N         = number of rows with at least one valid slot
+ *   *loss     = coeff * sum_t KL_t / max(N, 1)
+ *   dscores[k]= coeff / max(N,1) * (q[k] * sum_{valid} p - p[k]) on valid
+ *               slots of valid rows, 0 elsewhere
+ *
+ *   p, scores  [B,S,K] fp32; valid [B,S,K] uint8
+ *   loss       device fp32 scalar, written
+ *   dscores    [B,S,K] fp32, written; NULL = forward only
+ *   workspace  device scratch of ws_bytes >= sai_distill_kl_workspace_bytes(),
+ *              16-byte aligned; no initialisation needed; must not be shared
+ *              by calls that overlap on the device.
+ *
+ * The loss is reduced in a fixed order (deterministic). Errors: SAI_ERR_NULL,
+ * SAI_ERR_SHAPE, SAI_ERR_ALIGN, SAI_ERR_WORKSPACE, SAI_ERR_CUDA.
+ */
+sai_status sai_distill_kl(const float *p, const float *scores, const uint8_t *valid,
+                          int B, int S, int K, float coeff,
+                          float *loss, float *dscores, void *workspace, size_t ws_bytes,
+                          void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SAI_H */

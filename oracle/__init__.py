@@ -46,8 +46,15 @@ def _load():
         lib.orc_count_valid_rows.restype = I
         lib.orc_distill_kl.argtypes = [P, P, P, I, I, Dd, I, P, P, P]
         lib.orc_distill_kl.restype = None
+        lib.orc_num_threads.argtypes = []
+        lib.orc_num_threads.restype = ctypes.c_int
         _lib = lib
     return _lib
+
+
+def num_threads() -> int:
+    """Threads the oracle's OpenMP loops use."""
+    return int(_load().orc_num_threads())
 
 
 def _ptr(a: Optional[np.ndarray]):

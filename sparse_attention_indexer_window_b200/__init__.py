@@ -1,0 +1,179 @@
+"""Thin Python binding of libsai (CSA indexer distillation loss, sm_100a).
+
+Every function marshals torch CUDA tensors into the C ABI of ``include/sai.h``
+and raises ``SaiError`` on a non-zero status. There is no computation and no
+fallback here: if ``libsai.so`` is missing the import fails.
+
+    window_lse(Q, Kw, W, scale, doc_start=None)                -> [B,S,H] fp32
+    distill_target(Q, pool, idx, wl, cr, scale, sink=None, doc_start=None, err=None) -> [B,S,K] fp32
+    distill_kl(p, scores, valid, coeff, want_grad=True, workspace=None) -> (loss[1], dscores)
+
+bf16 tensors may be passed as torch.bfloat16 or as int16/uint16 bit patterns.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libsai.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"libsai.so is not built ({LIB_PATH}); run "
+                      "`python -m sparse_attention_indexer_window_b200.build`")
+
+_lib = ctypes.CDLL(LIB_PATH)
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_F = ctypes.c_float
+_lib.sai_window_lse.argtypes = [_P, _P, _P, _I, _I, _I, _I, _I, _F, _P, _P]
+_lib.sai_window_lse.restype = _I
+_lib.sai_distill_target.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P]
+_lib.sai_distill_target.restype = _I
+_lib.sai_distill_kl_workspace_bytes.argtypes = [_I, _I, _I]
+_lib.sai_distill_kl_workspace_bytes.restype = ctypes.c_size_t
+_lib.sai_distill_kl.argtypes = [_P, _P, _P, _I, _I, _I, _F, _P, _P, _P, ctypes.c_size_t, _P]
+_lib.sai_distill_kl.restype = _I
+_lib.sai_status_string.argtypes = [_I]
+_lib.sai_status_string.restype = ctypes.c_char_p
+_lib.sai_version.argtypes = []
+_lib.sai_version.restype = _I
+
+SAI_ERR_INDEX = 5
+SAI_ERR_TIMEOUT = 8
+
+
+class SaiError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {_lib.sai_status_string(status).decode()}")
+
+
+def lib() -> ctypes.CDLL:
+    return _lib
+
+
+def version() -> int:
+    return int(_lib.sai_version())
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(dev: torch.device):
+    return ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
+
+
+def _check(st: int, where: str):
+    if st != 0:
+        raise SaiError(st, where)
+
+
+def _bf16_bits(t: torch.Tensor, name: str) -> torch.Tensor:
+    if t.dtype in (torch.bfloat16, torch.int16, torch.uint16):
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+        return t
+    raise TypeError(f"{name} must be bfloat16 (or its int16/uint16 bit pattern), got {t.dtype}")
+
+
+def _want(t: Optional[torch.Tensor], name: str, dtype, shape=None):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    return t
+
+
+def window_lse(Q: torch.Tensor, Kw: torch.Tensor, W: int, scale: float,
+               doc_start: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    B, S, H, D = Q.shape
+    Q = _bf16_bits(Q, "Q")
+    Kw = _bf16_bits(Kw, "Kw")
+    if tuple(Kw.shape) != (B, S, D):
+        raise ValueError("Kw must be [B,S,D]")
+    _want(doc_start, "doc_start", torch.int32, (B, S))
+    if out is None:
+        out = torch.empty((B, S, H), dtype=torch.float32, device=Q.device)
+    _want(out, "out", torch.float32, (B, S, H))
+    st = _lib.sai_window_lse(_ptr(Q), _ptr(Kw), _ptr(doc_start), B, S, H, D, int(W), float(scale),
+                             _ptr(out), _stream(Q.device))
+    _check(st, "sai_window_lse")
+    return out
+
+
+def distill_target(Q: torch.Tensor, pool: torch.Tensor, idx: torch.Tensor, wl: torch.Tensor, cr: int,
+                   scale: float, sink: Optional[torch.Tensor] = None, doc_start: Optional[torch.Tensor] = None,
+                   err: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    B, S, H, D = Q.shape
+    K = idx.shape[-1]
+    Q = _bf16_bits(Q, "Q")
+    pool = _bf16_bits(pool, "pool")
+    if tuple(pool.shape) != (B, S // cr, D):
+        raise ValueError("pool must be [B,S/cr,D]")
+    _want(idx, "idx", torch.int32, (B, S, K))
+    _want(wl, "window_lse", torch.float32, (B, S, H))
+    if sink is not None:
+        # The Primus page: a sink must hold one value per head (else ValueError).
+        if sink.numel() != H:
+            raise ValueError(f"sink must hold {H} head values, got {sink.numel()}")
+        _want(sink, "sink", torch.float32)
+    _want(doc_start, "doc_start", torch.int32, (B, S))
+    _want(err, "err", torch.int32)
+    if out is None:
+        out = torch.empty((B, S, K), dtype=torch.float32, device=Q.device)
+    _want(out, "out", torch.float32, (B, S, K))
+    st = _lib.sai_distill_target(_ptr(Q), _ptr(pool), _ptr(idx), _ptr(wl), _ptr(sink), _ptr(doc_start),
+                                 B, S, H, D, K, int(cr), float(scale), _ptr(out), _ptr(err), _stream(Q.device))
+    _check(st, "sai_distill_target")
+    return out
+
+
+def kl_workspace_bytes(B: int, S: int, K: int) -> int:
+    return int(_lib.sai_distill_kl_workspace_bytes(B, S, K))
+
+
+def distill_kl(p: torch.Tensor, scores: torch.Tensor, valid: torch.Tensor, coeff: float,
+               want_grad: bool = True, workspace: Optional[torch.Tensor] = None,
+               loss: Optional[torch.Tensor] = None, dscores: Optional[torch.Tensor] = None
+               ) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    B, S, K = scores.shape
+    _want(p, "p", torch.float32, (B, S, K))
+    _want(scores, "scores", torch.float32, (B, S, K))
+    if valid.dtype == torch.bool:
+        valid = valid.view(torch.uint8)
+    _want(valid, "valid", torch.uint8, (B, S, K))
+    need = kl_workspace_bytes(B, S, K)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=scores.device)
+    if loss is None:
+        loss = torch.empty(1, dtype=torch.float32, device=scores.device)
+    if want_grad and dscores is None:
+        dscores = torch.empty((B, S, K), dtype=torch.float32, device=scores.device)
+    if not want_grad:
+        dscores = None
+    st = _lib.sai_distill_kl(_ptr(p), _ptr(scores), _ptr(valid), B, S, K, float(coeff), _ptr(loss),
+                             _ptr(dscores), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                             _stream(scores.device))
+    _check(st, "sai_distill_kl")
+    return loss, dscores
+
+
+def distill_loss(Q, Kw, pool, idx, scores, valid, *, W: int, cr: int, scale: float, coeff: float,
+                 sink=None, doc_start=None, err=None, workspace=None):
+    """The whole path, three calls on the current stream:
+    window_lse -> distill_target -> distill_kl. Returns (loss, dscores, p, wl)."""
+    wl = window_lse(Q, Kw, W, scale, doc_start)
+    p = distill_target(Q, pool, idx, wl, cr, scale, sink=sink, doc_start=doc_start, err=err)
+    loss, ds = distill_kl(p, scores, valid, coeff, workspace=workspace)
+    return loss, ds, p, wl

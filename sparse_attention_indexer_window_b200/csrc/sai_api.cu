@@ -1,0 +1,223 @@
+// C-ABI entry points of libsai (declared in include/sai.h): argument
+// validation, kernel selection by shape, TMA descriptor encoding and launch.
+// Nothing here allocates device memory or synchronises the stream.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include "sai.h"
+#include "sai_kernels.h"
+
+namespace {
+
+using sai::KlPlan;
+
+int sm_count()
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess)
+        return 0;
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return 0;
+    return n;
+}
+
+int max_smem_optin()
+{
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess)
+        return 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+        return 0;
+    return n;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
+
+// bf16 matrix [rows, cols] (row-major), box = box_rows x 64 columns, 128-byte
+// swizzle (the layout the tcgen05 descriptors expect).
+bool make_map_bf16(CUtensorMap *m, const void *ptr, uint64_t rows, uint64_t cols, uint32_t box_rows)
+{
+    PFN_cuTensorMapEncodeTiled_v12000 enc = encode_fn();
+    if (!enc)
+        return false;
+    cuuint64_t gdim[2] = {cols, rows};
+    cuuint64_t gstride[1] = {cols * 2};
+    cuuint32_t box[2] = {64, box_rows};
+    cuuint32_t estride[2] = {1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr), gdim, gstride, box, estride,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+bool al16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool al4(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+bool tc_heads(int H) { return H == 16 || H == 32 || H == 64 || H == 128; }
+
+sai_status cuda_status(cudaError_t e) { return e == cudaSuccess ? SAI_OK : SAI_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+const char *sai_status_string(int status)
+{
+    switch (status) {
+    case SAI_OK: return "SAI_OK";
+    case SAI_ERR_NULL: return "SAI_ERR_NULL: a required pointer is NULL";
+    case SAI_ERR_SHAPE: return "SAI_ERR_SHAPE: a size is out of range or sizes are inconsistent";
+    case SAI_ERR_UNSUPPORTED: return "SAI_ERR_UNSUPPORTED: shape outside what the kernels cover";
+    case SAI_ERR_CUDA: return "SAI_ERR_CUDA: a CUDA call or kernel launch failed";
+    case SAI_ERR_INDEX: return "SAI_ERR_INDEX: an idx entry lies outside {-1} U [0, S/cr)";
+    case SAI_ERR_WORKSPACE: return "SAI_ERR_WORKSPACE: workspace missing, too small or misaligned";
+    case SAI_ERR_ALIGN: return "SAI_ERR_ALIGN: a tensor pointer is not suitably aligned";
+    case SAI_ERR_TIMEOUT: return "SAI_ERR_TIMEOUT: a kernel gave up a bounded wait";
+    default: return "unknown sai_status";
+    }
+}
+
+int sai_version(void) { return 100; }
+
+sai_status sai_window_lse(const uint16_t *Q, const uint16_t *Kw, const int32_t *doc_start, int B, int S, int H,
+                          int D, int W, float scale, float *window_lse, void *stream)
+{
+    if (!Q || !Kw || !window_lse)
+        return SAI_ERR_NULL;
+    if (B < 1 || S < 1 || H < 1 || D < 1 || W < 1 || (D % 8) != 0 || !isfinite(scale))
+        return SAI_ERR_SHAPE;
+    if ((int64_t)B * S * H * D > INT32_MAX || (int64_t)B * S * H > INT32_MAX)
+        return SAI_ERR_SHAPE;
+    if (!al16(Q) || !al16(Kw) || !al4(window_lse) || (doc_start && !al4(doc_start)))
+        return SAI_ERR_ALIGN;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const int smem_cap = max_smem_optin();
+
+    if (tc_heads(H) && (D % 64) == 0 && S % (128 / H) == 0 && W + 128 / H - 1 <= 256) {
+        sai::WinTcArgs a;
+        a.B = B;
+        a.S = S;
+        a.H = H;
+        a.D = D;
+        a.W = W;
+        a.TQ = 128 / H;
+        a.NB = ((W + a.TQ - 1) + 15) / 16 * 16;
+        a.n_tiles = B * S / a.TQ;
+        a.b_stage_bytes = (uint32_t)(((size_t)a.NB * 128 + 1023) & ~size_t(1023));
+        a.scale = scale;
+        a.doc_start = doc_start;
+        a.out = window_lse;
+        if ((int)sai::window_tc_smem_bytes(a.NB) > smem_cap)
+            return SAI_ERR_UNSUPPORTED;
+        CUtensorMap mq, mk;
+        if (!make_map_bf16(&mq, Q, (uint64_t)B * S * H, D, 128) ||
+            !make_map_bf16(&mk, Kw, (uint64_t)B * S, D, (uint32_t)a.NB))
+            return SAI_ERR_CUDA;
+        int grid = sm_count();
+        if (grid <= 0)
+            return SAI_ERR_CUDA;
+        if (grid > a.n_tiles)
+            grid = a.n_tiles;
+        return cuda_status(sai::launch_window_lse_tc(mq, mk, a, grid, st));
+    }
+    if ((int)sai::window_simt_smem_bytes(H, D, W) <= smem_cap)
+        return cuda_status(sai::launch_window_lse_simt(Q, Kw, doc_start, B, S, H, D, W, scale, window_lse, st));
+    return SAI_ERR_UNSUPPORTED;
+}
+
+sai_status sai_distill_target(const uint16_t *Q, const uint16_t *pool, const int32_t *idx, const float *window_lse,
+                              const float *sink, const int32_t *doc_start, int B, int S, int H, int D, int K,
+                              int cr, float scale, float *p, int32_t *d_err, void *stream)
+{
+    if (!Q || !pool || !idx || !window_lse || !p)
+        return SAI_ERR_NULL;
+    if (B < 1 || S < 1 || H < 1 || D < 1 || K < 1 || cr < 1 || (D % 8) != 0 || (S % cr) != 0 ||
+        !isfinite(scale))
+        return SAI_ERR_SHAPE;
+    const int P = S / cr;
+    if (K > P)
+        return SAI_ERR_SHAPE;
+    if ((int64_t)B * S * H * D > INT32_MAX || (int64_t)B * S * K > INT32_MAX)
+        return SAI_ERR_SHAPE;
+    if (!al16(Q) || !al16(pool) || !al4(idx) || !al4(window_lse) || !al4(p) || (sink && !al4(sink)) ||
+        (doc_start && !al4(doc_start)) || (d_err && !al4(d_err)))
+        return SAI_ERR_ALIGN;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const int smem_cap = max_smem_optin();
+
+    if (tc_heads(H) && (D % 64) == 0 && (int)sai::target_tc_smem_bytes(H, K) <= smem_cap) {
+        sai::TgtTcArgs a;
+        a.B = B;
+        a.S = S;
+        a.H = H;
+        a.D = D;
+        a.K = K;
+        a.cr = cr;
+        a.P = P;
+        a.n_tok = B * S;
+        a.tiles_per_group = 256 / H;
+        a.scale = scale;
+        a.idx = idx;
+        a.wl = window_lse;
+        a.sink = sink;
+        a.doc_start = doc_start;
+        a.p = p;
+        a.err = d_err;
+        CUtensorMap mq, mp;
+        if (!make_map_bf16(&mq, Q, (uint64_t)B * S * H, D, (uint32_t)H) ||
+            !make_map_bf16(&mp, pool, (uint64_t)B * P, D, 1))
+            return SAI_ERR_CUDA;
+        int grid = sm_count();
+        if (grid <= 0)
+            return SAI_ERR_CUDA;
+        if (grid > a.n_tok)
+            grid = a.n_tok;
+        return cuda_status(sai::launch_target_tc(mq, mp, a, grid, st));
+    }
+    if ((int)sai::target_simt_smem_bytes(H, D, K) <= smem_cap)
+        return cuda_status(sai::launch_target_simt(Q, pool, idx, window_lse, sink, doc_start, B, S, H, D, K, cr,
+                                                   scale, p, d_err, st));
+    return SAI_ERR_UNSUPPORTED;
+}
+
+size_t sai_distill_kl_workspace_bytes(int B, int S, int K)
+{
+    if (B < 1 || S < 1 || K < 1)
+        return 0;
+    return sai::kl_plan(B, S, K).ws_bytes;
+}
+
+sai_status sai_distill_kl(const float *p, const float *scores, const uint8_t *valid, int B, int S, int K,
+                          float coeff, float *loss, float *dscores, void *workspace, size_t ws_bytes,
+                          void *stream)
+{
+    if (!p || !scores || !valid || !loss)
+        return SAI_ERR_NULL;
+    if (B < 1 || S < 1 || K < 1 || !isfinite(coeff) || (int64_t)B * S * K > INT32_MAX)
+        return SAI_ERR_SHAPE;
+    if (!al16(p) || !al16(scores) || !al16(valid) || !al4(loss) || (dscores && !al16(dscores)))
+        return SAI_ERR_ALIGN;
+    const KlPlan pl = sai::kl_plan(B, S, K);
+    if (!workspace || !al16(workspace) || ws_bytes < pl.ws_bytes)
+        return SAI_ERR_WORKSPACE;
+    return cuda_status(sai::launch_distill_kl(pl, p, scores, valid, coeff, loss, dscores, workspace,
+                                              reinterpret_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

@@ -1,0 +1,65 @@
+// Internal launch interface between the C-ABI entry points (sai_api.cu) and
+// the kernels. Not installed; not part of the public ABI.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace sai {
+
+// ---------------------------------------------------------------- window_lse
+struct WinTcArgs {
+    int B, S, H, D, W;
+    int TQ;               // tokens per 128-row tile (128 / H)
+    int NB;               // band rows = roundup16(W + TQ - 1), <= 256
+    int n_tiles;          // B*S / TQ
+    uint32_t b_stage_bytes;
+    float scale;
+    const int32_t *doc_start;
+    float *out;
+};
+size_t window_tc_smem_bytes(int NB);
+cudaError_t launch_window_lse_tc(const CUtensorMap &mapQ, const CUtensorMap &mapK, const WinTcArgs &a,
+                                 int grid, cudaStream_t stream);
+
+// ------------------------------------------------------------ distill_target
+struct TgtTcArgs {
+    int B, S, H, D, K, cr, P;
+    int n_tok;            // B*S
+    int tiles_per_group;  // 128-slot tiles per TMEM accumulator (256 / H)
+    float scale;
+    const int32_t *idx;
+    const float *wl;
+    const float *sink;
+    const int32_t *doc_start;
+    float *p;
+    int32_t *err;
+};
+size_t target_tc_smem_bytes(int H, int K);
+cudaError_t launch_target_tc(const CUtensorMap &mapQ, const CUtensorMap &mapPool, const TgtTcArgs &a, int grid,
+                             cudaStream_t stream);
+
+// ------------------------------------------- generic CUDA-core kernels
+// For shapes the tensor-core kernels do not take (small H or D).
+size_t window_simt_smem_bytes(int H, int D, int W);
+cudaError_t launch_window_lse_simt(const uint16_t *Q, const uint16_t *Kw, const int32_t *doc_start, int B, int S,
+                                   int H, int D, int W, float scale, float *out, cudaStream_t stream);
+size_t target_simt_smem_bytes(int H, int D, int K);
+cudaError_t launch_target_simt(const uint16_t *Q, const uint16_t *pool, const int32_t *idx, const float *wl,
+                               const float *sink, const int32_t *doc_start, int B, int S, int H, int D, int K,
+                               int cr, float scale, float *p, int32_t *err, cudaStream_t stream);
+
+// ---------------------------------------------------------------- distill_kl
+struct KlPlan {
+    int rows, K;
+    int count_blocks;   // blocks of the valid-row count kernel
+    int row_blocks;     // blocks of the row kernel
+    size_t ws_bytes;
+};
+KlPlan kl_plan(int B, int S, int K);
+cudaError_t launch_distill_kl(const KlPlan &pl, const float *p, const float *scores, const uint8_t *valid,
+                              float coeff, float *loss, float *dscores, void *ws, cudaStream_t stream);
+
+}  // namespace sai

@@ -189,12 +189,17 @@ def _idx_topk_sorted(rng, S, cr, K, doc_start, b) -> np.ndarray:
 
 
 def make(name: str, *, seed: Optional[int] = None, with_sink: bool = True,
-         S: Optional[int] = None, B: Optional[int] = None) -> Workload:
-    """Draw the named workload. ``S``/``B`` override the sizes (same recipe)."""
+         S: Optional[int] = None, B: Optional[int] = None, K: Optional[int] = None,
+         W: Optional[int] = None) -> Workload:
+    """Draw the named workload. ``S``/``B``/``K``/``W`` override the sizes
+    (same recipe and value distributions)."""
     sp = CONFIGS[name]
     B_ = B if B is not None else sp.B
     S_ = S if S is not None else sp.S
-    H, D, cr, K, W = sp.H, sp.D, sp.cr, sp.K, sp.W
+    H, D, cr = sp.H, sp.D, sp.cr
+    K = sp.K if K is None else K
+    W = sp.W if W is None else W
+    assert K <= S_ // cr
     assert S_ % cr == 0
     P = S_ // cr
     rng = np.random.Generator(np.random.PCG64(sp.seed if seed is None else seed))

@@ -1,0 +1,100 @@
+"""The C-ABI library: it builds for sm_100a, loads, exports every symbol that
+include/sai.h declares, and rejects bad arguments on the host before touching
+the GPU (so these run without a GPU)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "sai.h")
+
+
+@pytest.fixture(scope="module")
+def sai():
+    from sparse_attention_indexer_window_b200 import build
+    build.build()
+    import sparse_attention_indexer_window_b200 as m
+    return m
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"\b(sai_[a-z0-9_]+)\s*\(", src)
+    return sorted(set(names))
+
+
+def test_header_declares_the_three_calls():
+    names = declared_functions()
+    for n in ("sai_window_lse", "sai_distill_target", "sai_distill_kl", "sai_distill_kl_workspace_bytes",
+              "sai_status_string", "sai_version"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(sai):
+    lib = ctypes.CDLL(sai.LIB_PATH)
+    for n in declared_functions():
+        assert hasattr(lib, n), n
+
+
+def test_status_strings(sai):
+    lib = sai.lib()
+    for code in range(0, 9):
+        s = lib.sai_status_string(code).decode()
+        assert s.startswith("SAI_")
+    assert b"unknown" in lib.sai_status_string(99)
+
+
+def test_workspace_size(sai):
+    lib = sai.lib()
+    assert lib.sai_distill_kl_workspace_bytes(0, 1, 1) == 0
+    n = lib.sai_distill_kl_workspace_bytes(1, 4096, 512)
+    assert 16 < n < 1 << 20 and n % 16 == 0
+
+
+FAKE = 1 << 20          # a 16-byte aligned non-NULL address; never dereferenced
+FAKE_MIS = FAKE + 4     # misaligned for 16-byte tensors
+
+
+def test_window_lse_host_errors(sai):
+    lib = sai.lib()
+    ok = dict(B=1, S=64, H=4, D=32, W=16)
+    f = lib.sai_window_lse
+    assert f(None, FAKE, None, 1, 64, 4, 32, 16, 0.1, FAKE, None) == 1          # NULL Q
+    assert f(FAKE, FAKE, None, 0, 64, 4, 32, 16, 0.1, FAKE, None) == 2          # B = 0
+    assert f(FAKE, FAKE, None, 1, 64, 4, 30, 16, 0.1, FAKE, None) == 2          # D % 8
+    assert f(FAKE, FAKE, None, 1, 64, 4, 32, 0, 0.1, FAKE, None) == 2           # W = 0
+    assert f(FAKE, FAKE, None, 1, 64, 4, 32, 16, float("nan"), FAKE, None) == 2
+    assert f(FAKE_MIS, FAKE, None, 1, 64, 4, 32, 16, 0.1, FAKE, None) == 7      # misaligned Q
+
+
+def test_distill_target_host_errors(sai):
+    f = sai.lib().sai_distill_target
+    a = [FAKE] * 4
+    assert f(None, FAKE, FAKE, FAKE, None, None, 1, 64, 4, 32, 8, 4, 0.1, FAKE, None, None) == 1
+    assert f(*a, None, None, 1, 64, 4, 32, 8, 3, 0.1, FAKE, None, None) == 2     # S % cr
+    assert f(*a, None, None, 1, 64, 4, 32, 17, 4, 0.1, FAKE, None, None) == 2    # K > S/cr
+    assert f(*a, None, None, 1, 64, 4, 32, 0, 4, 0.1, FAKE, None, None) == 2     # K = 0
+    assert f(FAKE, FAKE_MIS, FAKE, FAKE, None, None, 1, 64, 4, 32, 8, 4, 0.1, FAKE, None, None) == 7
+
+
+def test_distill_kl_host_errors(sai):
+    f = sai.lib().sai_distill_kl
+    need = sai.lib().sai_distill_kl_workspace_bytes(1, 64, 8)
+    assert f(None, FAKE, FAKE, 1, 64, 8, 0.01, FAKE, FAKE, FAKE, need, None) == 1
+    assert f(FAKE, FAKE, FAKE, 1, 0, 8, 0.01, FAKE, FAKE, FAKE, need, None) == 2
+    assert f(FAKE, FAKE, FAKE, 1, 64, 8, 0.01, FAKE, FAKE, FAKE, need - 1, None) == 6   # short workspace
+    assert f(FAKE, FAKE, FAKE, 1, 64, 8, 0.01, FAKE, FAKE, None, need, None) == 6       # no workspace
+    assert f(FAKE, FAKE, FAKE, 1, 64, 8, 0.01, FAKE, FAKE, FAKE_MIS, need, None) == 6   # misaligned
+    assert f(FAKE_MIS, FAKE, FAKE, 1, 64, 8, 0.01, FAKE, FAKE, FAKE, need, None) == 7
+
+
+def test_python_sink_length_check(sai):
+    """The Primus page's rule: a sink must hold one value per head."""
+    import torch
+    Q = torch.zeros((1, 8, 4, 8), dtype=torch.bfloat16)
+    with pytest.raises((ValueError, TypeError)):
+        sai.distill_target(Q, torch.zeros((1, 2, 8), dtype=torch.bfloat16), torch.zeros((1, 8, 2), dtype=torch.int32),
+                           torch.zeros((1, 8, 4)), 4, 0.1, sink=torch.zeros(3))
