@@ -71,7 +71,7 @@ int sai_version(void);
  *   Q          [B,S,H,D] bf16, 16-byte aligned
  *   Kw         [B,S,D]   bf16, 16-byte aligned
  *   doc_start  [B,S] int32 or NULL (one document per row)
- *   scale      logit scale, e.g. 1/sqrt(D)
+ *   scale      logit scale > 0, e.g. 1/sqrt(D)
  *   window_lse [B,S,H] fp32, written
  *
  * Sizes: B,S,H,D,W >= 1 and D % 8 == 0. Errors: SAI_ERR_NULL, SAI_ERR_SHAPE,
@@ -113,7 +113,7 @@ sai_status sai_window_lse(const uint16_t *Q, const uint16_t *Kw, const int32_t *
  *              SAI_ERR_INDEX here; the caller zeroes it and reads it back.
  *
  * Sizes: S % cr == 0, 1 <= K <= S/cr (the MaxText page's topk <= length/4
- * check), D % 8 == 0. Errors: SAI_ERR_NULL, SAI_ERR_SHAPE, SAI_ERR_ALIGN,
+ * check), D % 8 == 0, scale > 0. Errors: SAI_ERR_NULL, SAI_ERR_SHAPE, SAI_ERR_ALIGN,
  * SAI_ERR_UNSUPPORTED, SAI_ERR_CUDA.
  */
 sai_status sai_distill_target(const uint16_t *Q, const uint16_t *pool, const int32_t *idx,

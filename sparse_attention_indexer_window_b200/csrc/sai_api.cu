@@ -100,7 +100,7 @@ sai_status sai_window_lse(const uint16_t *Q, const uint16_t *Kw, const int32_t *
 {
     if (!Q || !Kw || !window_lse)
         return SAI_ERR_NULL;
-    if (B < 1 || S < 1 || H < 1 || D < 1 || W < 1 || (D % 8) != 0 || !isfinite(scale))
+    if (B < 1 || S < 1 || H < 1 || D < 1 || W < 1 || (D % 8) != 0 || !isfinite(scale) || scale <= 0.f)
         return SAI_ERR_SHAPE;
     if ((int64_t)B * S * H * D > INT32_MAX || (int64_t)B * S * H > INT32_MAX)
         return SAI_ERR_SHAPE;
@@ -148,7 +148,7 @@ sai_status sai_distill_target(const uint16_t *Q, const uint16_t *pool, const int
     if (!Q || !pool || !idx || !window_lse || !p)
         return SAI_ERR_NULL;
     if (B < 1 || S < 1 || H < 1 || D < 1 || K < 1 || cr < 1 || (D % 8) != 0 || (S % cr) != 0 ||
-        !isfinite(scale))
+        !isfinite(scale) || scale <= 0.f)
         return SAI_ERR_SHAPE;
     const int P = S / cr;
     if (K > P)
@@ -172,23 +172,24 @@ sai_status sai_distill_target(const uint16_t *Q, const uint16_t *pool, const int
         a.P = P;
         a.n_tok = B * S;
         a.tiles_per_group = 256 / H;
+        a.idx_bulk = ((K % 4) == 0 && al16(idx)) ? 1 : 0;
         a.scale = scale;
+        a.pool = pool;
         a.idx = idx;
         a.wl = window_lse;
         a.sink = sink;
         a.doc_start = doc_start;
         a.p = p;
         a.err = d_err;
-        CUtensorMap mq, mp;
-        if (!make_map_bf16(&mq, Q, (uint64_t)B * S * H, D, (uint32_t)H) ||
-            !make_map_bf16(&mp, pool, (uint64_t)B * P, D, 1))
+        CUtensorMap mq;
+        if (!make_map_bf16(&mq, Q, (uint64_t)B * S * H, D, (uint32_t)H))
             return SAI_ERR_CUDA;
         int grid = sm_count();
         if (grid <= 0)
             return SAI_ERR_CUDA;
         if (grid > a.n_tok)
             grid = a.n_tok;
-        return cuda_status(sai::launch_target_tc(mq, mp, a, grid, st));
+        return cuda_status(sai::launch_target_tc(mq, a, grid, st));
     }
     if ((int)sai::target_simt_smem_bytes(H, D, K) <= smem_cap)
         return cuda_status(sai::launch_target_simt(Q, pool, idx, window_lse, sink, doc_start, B, S, H, D, K, cr,

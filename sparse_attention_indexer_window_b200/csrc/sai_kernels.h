@@ -29,7 +29,9 @@ struct TgtTcArgs {
     int B, S, H, D, K, cr, P;
     int n_tok;            // B*S
     int tiles_per_group;  // 128-slot tiles per TMEM accumulator (256 / H)
+    int idx_bulk;         // idx rows are 16-byte aligned (K % 4 == 0): stage them by bulk copy
     float scale;
+    const uint16_t *pool;
     const int32_t *idx;
     const float *wl;
     const float *sink;
@@ -38,8 +40,7 @@ struct TgtTcArgs {
     int32_t *err;
 };
 size_t target_tc_smem_bytes(int H, int K);
-cudaError_t launch_target_tc(const CUtensorMap &mapQ, const CUtensorMap &mapPool, const TgtTcArgs &a, int grid,
-                             cudaStream_t stream);
+cudaError_t launch_target_tc(const CUtensorMap &mapQ, const TgtTcArgs &a, int grid, cudaStream_t stream);
 
 // ------------------------------------------- generic CUDA-core kernels
 // For shapes the tensor-core kernels do not take (small H or D).

@@ -1,5 +1,5 @@
-// Distillation target on tcgen05 tensor cores with an in-kernel TMA gather of
-// the selected pool rows (sm_100a).
+// Distillation target on tcgen05 tensor cores with an in-kernel gather of the
+// selected pool rows (sm_100a).
 //
 // For every token (b,t) (Primus page "perf(deepseek-v4): fuse and enable the
 // indexer distillation loss": first commit message -- the pool is indexed
@@ -15,57 +15,72 @@
 // Layout of the contraction. The problem is transposed so the MMA keeps M=128
 // although a token has only H heads: A = 128 gathered pool rows (one TMEM lane
 // per selected slot), B = Q[t] (N = H columns, one per head), K-dim = D in
-// 64-element (128-byte, swizzled) chunks. The producer compacts the token's
-// idx row (selected slots first, masked slots last) and gathers the selected
-// rows four at a time with TMA tile::gather4 straight into the swizzled smem
-// operand layout; masked slots are never loaded.
+// 64-element (128-byte, swizzled) chunks.
+//
+// Gather. A dedicated warp compacts each token's idx row (selected slots
+// first, masked slots last), up to two tokens ahead; the idx rows arrive by a
+// 1-D bulk copy. Eight gather warps then copy the selected rows into the
+// swizzled K-major operand layout with 16-byte cp.async (eight lanes per row,
+// four rows per instruction, every 128-byte row segment one coalesced
+// request); each thread's cp.async.mbarrier arrival publishes a stage. On
+// B200 a random-row gather from L2 saturates near 45 bytes/clock per SM this
+// way with eight or more warps (TMA tile::gather4 near 20), so the gather, not
+// the tensor core, bounds this kernel. Q[t] chunks (contiguous) arrive by TMA
+// tile loads. Masked slots are never loaded.
 //
 // The epilogue needs the per-head log-sum-exp over ALL selected slots before
 // it can form u, so a token's scores stay in TMEM until it is done: up to
-// 256/H tiles (512 slots at H=64) per accumulator, two accumulators so the
-// epilogue of one token overlaps the MMA of the next. Tokens with more
-// selected slots run in groups: a first pass over the groups merges per-head
-// (max, sum-exp) statistics, a second pass recomputes each group's scores and
-// forms u.
+// 256/H tiles (512 slots at H=64) per accumulator. Two epilogue warpgroups
+// take alternate tokens, each with its own 256-column accumulator, so one
+// token's epilogue overlaps the next token's MMA. Tokens with more selected
+// slots run in groups: a first pass over the groups merges per-head (max,
+// sum-exp) statistics, a second pass recomputes each group and forms u.
 //
 // Epilogue arithmetic (one exponential per score):
 //   M[h] = max_k z[k,h]  (column max: transposing warp butterfly + smem)
 //   e[k,h] = exp(z[k,h] - M[h]) written back to TMEM, S[h] = sum_k e[k,h]
 //   a[h] = M[h] - lse_full[h],  A = max_h a[h],  w[h] = exp(a[h] - A) in (0,1]
-//   u'[k] = sum_h e[k,h] w[h]   (per thread, one TMEM lane = one slot)
-//   m' = sum_k u'[k] >= 1, and u = u' e^A, m = m' e^A, so
-//   p[k] = u'[k]/m'              if log m' + A >= log FLT_MIN
+//   u'[k] = sum_h e[k,h] w[h]   (per thread: one TMEM lane = one slot)
+//   m' = sum_k u'[k] >= 1; with u = u' e^A and m = m' e^A:
+//   p[k] = u'[k]/m'                     if log m' + A >= log FLT_MIN
 //        = u'[k] exp(A - log FLT_MIN)   otherwise (the float32-tiny floor),
-// which never forms a subnormal intermediate however small the compressed
-// share of every head is.
+// so no intermediate is subnormal however small each head's compressed share.
 //
-// Warp roles (192 threads): warp 0 producer (idx compaction by the whole
-// warp, TMA by lane 0; TMEM owner), warp 1 MMA issuer, warps 2..5 epilogue.
-// Persistent CTAs walk tokens from the last (heaviest) to the first. All
-// waits are bounded; a timeout is reported through err and the CTA unwinds.
+// Warp roles (576 threads): warp 0 idx staging and compaction, warps 1..8
+// row gathers (warp 1 also loads Q), warp 9 MMA issuer and TMEM owner, warps
+// 10..13 and 14..17 the two epilogue groups. Persistent CTAs walk tokens from the last
+// (heaviest) to the first. All mbarrier waits are bounded; a timeout is
+// reported through err and the CTA unwinds. Named barriers are only used
+// where every participating thread is guaranteed to arrive.
 #include "sai_device.cuh"
 #include "sai_kernels.h"
 
 namespace sai {
 namespace {
 
-constexpr int kTgtThreads = 192;
-constexpr int kAStages = 6;
+// Warpgroups 0..2 (warps 0..11): warp 0 compaction, warp 8 MMA, the other
+// ten warps row gathers; warpgroups 3 and 4 (warps 12..19): epilogue.
+constexpr int kMetaWarp = 0;
+constexpr int kMmaWarp = 8;
+constexpr int kGatherWarps = 10;
+constexpr int kEpiWarp0 = 12;
+constexpr int kTgtThreads = 20 * 32;                // 640
+// Register split (setmaxnreg): launched at kLaunchRegs a thread; warpgroups
+// 0..2 give theirs down to kLowRegs, the two epilogue warpgroups take
+// kHighRegs. 384*56 + 256*152 = 60416 <= 640*96 = 61440 (the launch total).
+constexpr int kLaunchRegs = 96;
+constexpr int kLowRegs = 56;
+constexpr int kHighRegs = 152;
+static_assert(384 * kLowRegs + 256 * kHighRegs <= kTgtThreads * kLaunchRegs, "register split");
+constexpr int kMaxAStages = 8;
 constexpr int kQStages = 3;
-constexpr uint32_t kATile = 128 * 128;  // 128 rows x 128 bytes
+constexpr int kMeta = 3;                            // compaction runs up to two tokens ahead
+constexpr uint32_t kATile = 128 * 128;              // 128 rows x 128 bytes
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLnFltMin = -87.33654475055310898657f;  // log(2^-126)
 
 template <int HH>
-struct TgtSmem {
-    uint64_t a_full[kAStages], a_empty[kAStages];
-    uint64_t q_full[kQStages], q_empty[kQStages];
-    uint64_t acc_full[2], acc_empty[2];
-    uint64_t meta_full[2], meta_empty[2];
-    uint64_t drain;
-    uint32_t tmem_base;
-    int abort_flag;
-    int nsel[2];
+struct EpiState {                 // one per epilogue warpgroup
     float red_max[4][HH];
     float red_sum[4][HH];
     float colM[HH];
@@ -73,12 +88,24 @@ struct TgtSmem {
     float head_a[HH];
     float wprime[HH];
     float red_m[4];
+    int flag;
 };
 
-struct Job {
-    int pass;    // 0 = statistics only, 1 = final (u)
-    int grp;
+template <int HH>
+struct TgtSmem {
+    uint64_t a_full[kMaxAStages], a_empty[kMaxAStages];
+    uint64_t q_full[kQStages], q_empty[kQStages];
+    uint64_t acc_full[2], acc_empty[2];
+    uint64_t meta_full[kMeta], meta_empty[kMeta];
+    uint64_t idx_full[2];
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort_flag;
+    int nsel[kMeta];
+    EpiState<HH> epi[2];
 };
+
+__host__ __device__ inline int a_stages_for(int K) { return K <= 1024 ? kMaxAStages : 6; }
 
 __device__ __forceinline__ int n_groups(int nsel, int TB)
 {
@@ -86,34 +113,42 @@ __device__ __forceinline__ int n_groups(int nsel, int TB)
     return (nt + TB - 1) / TB;
 }
 
+// Selection rule for one idx entry j of token t (document start d0).
+__device__ __forceinline__ bool selected(int j, int t, int d0, int P, int cr)
+{
+    return j >= 0 && j < P && (j + 1) * cr - 1 <= t && j * cr >= d0;
+}
+
 template <int HH>
 __global__ void __launch_bounds__(kTgtThreads, 1)
-    target_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapPool,
-                     const TgtTcArgs a)
+    target_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const TgtTcArgs a)
 {
     constexpr int TB = 256 / HH;                 // tiles per accumulator
-    constexpr int IB = TB < 4 ? TB : 4;          // tiles per TMEM load batch
+    constexpr int IB = TB < 2 ? TB : 2;          // tiles per TMEM load batch
     constexpr uint32_t kQTile = HH * 128;        // H rows x 128 bytes
     constexpr int NC16 = HH / 16;
 
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t *a_buf = base;                               // kAStages x 16 KB
-    uint8_t *q_buf = a_buf + kAStages * kATile;          // kQStages x H*128
-    int32_t *rowid = reinterpret_cast<int32_t *>(q_buf + kQStages * kQTile);  // [2][K]
-    int32_t *slot = rowid + 2 * a.K;                     // [2][K]
-    float *ubuf = reinterpret_cast<float *>(slot + 2 * a.K);  // [K]
-    TgtSmem<HH> *sm = reinterpret_cast<TgtSmem<HH> *>(
-        (reinterpret_cast<uintptr_t>(ubuf + a.K) + 15) & ~uintptr_t(15));
+    const int K = a.K;
+    const int Kp = (K + 3) & ~3;
+    const int NA = a_stages_for(K);
+    uint8_t *a_buf = base;                                                   // NA x 16 KB
+    uint8_t *q_buf = a_buf + NA * kATile;                                    // kQStages x H*128
+    int32_t *rowid = reinterpret_cast<int32_t *>(q_buf + kQStages * kQTile); // [kMeta][Kp]
+    int32_t *slot = rowid + kMeta * Kp;                                      // [kMeta][Kp]
+    int32_t *idxs = slot + kMeta * Kp;                                       // [2][Kp] staged idx rows
+    float *ubuf = reinterpret_cast<float *>(idxs + 2 * Kp);                  // [2][Kp]
+    TgtSmem<HH> *sm = reinterpret_cast<TgtSmem<HH> *>(ubuf + 2 * Kp);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int K = a.K;
     const int n_chunks = a.D / 64;
+    const bool idx_bulk = a.idx_bulk != 0;       // idx rows staged by bulk copy
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kAStages; ++s) {
-            mbar_init(&sm->a_full[s], 1);
+        for (int s = 0; s < NA; ++s) {
+            mbar_init(&sm->a_full[s], kGatherWarps * 32);  // one arrival per gather thread
             mbar_init(&sm->a_empty[s], 1);
         }
         for (int s = 0; s < kQStages; ++s) {
@@ -123,6 +158,9 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
         for (int b = 0; b < 2; ++b) {
             mbar_init(&sm->acc_full[b], 1);
             mbar_init(&sm->acc_empty[b], 4);
+            mbar_init(&sm->idx_full[b], 1);
+        }
+        for (int b = 0; b < kMeta; ++b) {
             mbar_init(&sm->meta_full[b], 1);
             mbar_init(&sm->meta_empty[b], 1);
         }
@@ -130,7 +168,7 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
         sm->abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp == 0) {
+    if (warp == kMmaWarp) {
         tmem_alloc(&sm->tmem_base, 512);
         tmem_relinquish();
     }
@@ -140,155 +178,245 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
     const uint32_t tmem = sm->tmem_base;
     volatile int *abort_flag = &sm->abort_flag;
 
-    if (warp == 0) {
-        // ============================================================ producer
-        if (lane == 0) {
-            tma_prefetch_desc(&mapQ);
-            tma_prefetch_desc(&mapPool);
+    if (warp < kEpiWarp0) {
+    // warpgroups 0..2 execute this one setmaxnreg together
+    regs_dec<kLowRegs>();
+    if (warp == kMetaWarp) {
+        // ====================================================== idx compaction
+        if (lane == 0 && idx_bulk && (int)blockIdx.x < a.n_tok) {
+            const int g0 = a.n_tok - 1 - blockIdx.x;
+            mbar_arrive_expect_tx(&sm->idx_full[0], (uint32_t)K * 4u);
+            bulk_load(idxs, a.idx + (size_t)g0 * K, (uint32_t)K * 4u, &sm->idx_full[0]);
         }
-        int as = 0, qs = 0;
-        uint32_t aph = 0, qph = 0;
-        uint32_t a_issued = 0, a_last = 0, q_issued = 0, q_last = 0;
+        uint32_t i_issued = 0, i_last = 0;
         bool ok = true;
         int it = 0;
         for (int gt = blockIdx.x; gt < a.n_tok && ok; gt += gridDim.x, ++it) {
             const int g = a.n_tok - 1 - gt;
             const int b = g / a.S;
             const int t = g - b * a.S;
-            const int mb = it & 1;
-            const uint32_t mph = (it >> 1) & 1;
-            if (!mbar_wait(&sm->meta_empty[mb], mph ^ 1u, abort_flag, a.err)) {
-                ok = false;
-                break;
+            const int ib2 = it & 1;
+            const int m3 = it % kMeta;
+            int32_t *ib = idxs + ib2 * Kp;
+            if (idx_bulk) {
+                // this token's idx row has landed; start the next token's copy
+                if (lane == 0) {
+                    ok = mbar_wait(&sm->idx_full[ib2], (it >> 1) & 1, abort_flag, a.err);
+                    const int gtn = gt + gridDim.x;
+                    if (ok && gtn < a.n_tok) {
+                        const int gn = a.n_tok - 1 - gtn;
+                        const int nb = ib2 ^ 1;
+                        mbar_arrive_expect_tx(&sm->idx_full[nb], (uint32_t)K * 4u);
+                        bulk_load(idxs + nb * Kp, a.idx + (size_t)gn * K, (uint32_t)K * 4u, &sm->idx_full[nb]);
+                        i_issued |= 1u << nb;
+                        i_last = (i_last & ~(1u << nb)) | ((((it + 1) >> 1) & 1u) << nb);
+                    }
+                }
+                ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+                if (!ok)
+                    break;
             }
+            if (lane == 0)
+                ok = mbar_wait(&sm->meta_empty[m3], ((it / kMeta) & 1) ^ 1u, abort_flag, a.err);
+            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+            if (!ok)
+                break;
             int d0 = 0;
             if (a.doc_start) {
                 d0 = a.doc_start[g];
                 d0 = d0 < 0 ? 0 : (d0 > t ? t : d0);
             }
-            // Compact the idx row: selected slots in order at the front,
-            // masked slots from the back.
-            int32_t *rw = rowid + mb * K;
-            int32_t *sl = slot + mb * K;
-            const int32_t *irow = a.idx + (size_t)g * K;
+            // selected slots in order at the front, masked slots from the back;
+            // lane L takes 4 consecutive slots
+            int32_t *rw = rowid + m3 * Kp;
+            int32_t *sl = slot + m3 * Kp;
+            const int32_t *grow = a.idx + (size_t)g * K;
             int nsel = 0, nmask = 0;
-            const uint32_t lt = (1u << lane) - 1u;
-            for (int k0 = 0; k0 < K; k0 += 32) {
-                const int k = k0 + lane;
-                const bool in = k < K;
-                const int j = in ? __ldg(irow + k) : -1;
-                const bool inr = j >= 0 && j < a.P;
-                const bool sel = in && inr && (j + 1) * a.cr - 1 <= t && j * a.cr >= d0;
-                if (in && !(j == -1 || inr) && a.err)
-                    atomicExch(a.err, kErrIndex);
-                const uint32_t sm_sel = __ballot_sync(0xffffffffu, sel);
-                const uint32_t sm_msk = __ballot_sync(0xffffffffu, in && !sel);
-                if (sel) {
-                    const int pos = nsel + __popc(sm_sel & lt);
-                    rw[pos] = b * a.P + j;
-                    sl[pos] = k;
+            bool bad = false;
+            for (int k0 = 0; k0 < K; k0 += 128) {
+                const int k = k0 + 4 * lane;
+                int j[4];
+                if (idx_bulk) {
+                    int4 v = make_int4(-1, -1, -1, -1);
+                    if (k < K)
+                        v = *reinterpret_cast<const int4 *>(ib + k);
+                    j[0] = v.x;
+                    j[1] = v.y;
+                    j[2] = v.z;
+                    j[3] = v.w;
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        j[e] = (k + e < K) ? __ldg(grow + k + e) : -1;
                 }
-                if (in && !sel)
-                    sl[K - 1 - (nmask + __popc(sm_msk & lt))] = k;
-                nsel += __popc(sm_sel);
-                nmask += __popc(sm_msk);
+                int cs = 0, cm = 0;
+                bool sel[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const bool in = k + e < K;
+                    sel[e] = in && selected(j[e], t, d0, a.P, a.cr);
+                    bad |= in && !(j[e] == -1 || (j[e] >= 0 && j[e] < a.P));
+                    cs += sel[e] ? 1 : 0;
+                    cm += (in && !sel[e]) ? 1 : 0;
+                }
+                int sc = cs | (cm << 16);  // packed inclusive scan of both counts
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int y = __shfl_up_sync(0xffffffffu, sc, o);
+                    if (lane >= o)
+                        sc += y;
+                }
+                const int tot = __shfl_sync(0xffffffffu, sc, 31);
+                int ps = nsel + (sc & 0xffff) - cs;
+                int pm = nmask + (sc >> 16) - cm;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    if (sel[e]) {
+                        rw[ps] = b * a.P + j[e];
+                        sl[ps] = k + e;
+                        ++ps;
+                    } else if (k + e < K) {
+                        sl[K - 1 - pm] = k + e;
+                        ++pm;
+                    }
+                }
+                nsel += tot & 0xffff;
+                nmask += tot >> 16;
             }
+            if (__any_sync(0xffffffffu, bad) && lane == 0 && a.err)
+                atomicExch(a.err, kErrIndex);
             if (lane == 0)
-                sm->nsel[mb] = nsel;
+                sm->nsel[m3] = nsel;
             __syncwarp();
             if (lane == 0)
-                mbar_arrive(&sm->meta_full[mb]);
-
+                mbar_arrive(&sm->meta_full[m3]);
+        }
+        if (!ok && lane == 0) {
+            for (int s = 0; s < 2; ++s)
+                if (i_issued & (1u << s))
+                    mbar_drain(&sm->idx_full[s], (i_last >> s) & 1u);
+        }
+        __syncwarp();
+    } else if (warp != kMmaWarp && warp < kEpiWarp0) {
+        // ============================================================ gathers
+        const int gw = warp < kMmaWarp ? warp - 1 : warp - 2;   // 0..9
+        const bool q_loader = (gw == 0);         // also loads the Q[t] chunks by TMA
+        if (q_loader && lane == 0)
+            tma_prefetch_desc(&mapQ);
+        int as = 0, qs = 0;
+        uint32_t aph = 0, qph = 0;
+        uint32_t q_issued = 0, q_last = 0;
+        bool ok = true;
+        int it = 0;
+        const char *pool_bytes = reinterpret_cast<const char *>(a.pool);
+        const int seg = lane & 7;                // 16-byte segment of a 128-byte row chunk
+        const int r_in = lane >> 3;              // row within a 4-row group
+        for (int gt = blockIdx.x; gt < a.n_tok && ok; gt += gridDim.x, ++it) {
+            const int g = a.n_tok - 1 - gt;
+            const int m3 = it % kMeta;
+            if (lane == 0)
+                ok = mbar_wait(&sm->meta_full[m3], (it / kMeta) & 1, abort_flag, a.err);
+            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+            if (!ok)
+                break;
+            const int nsel = sm->nsel[m3];
+            const int32_t *rw = rowid + m3 * Kp;
             const int nt = (nsel + 127) / 128;
             const int G = n_groups(nsel, TB);
             const int passes = G > 1 ? 2 : 1;
-            if (lane == 0) {
-                for (int pass = 0; pass < passes && ok; ++pass) {
-                    for (int grp = 0; grp < G && ok; ++grp) {
-                        const int i0 = grp * TB;
-                        const int i1 = min(nt, i0 + TB);
-                        for (int c = 0; c < n_chunks && ok; ++c) {
-                            if (!mbar_wait(&sm->q_empty[qs], qph ^ 1u, abort_flag, a.err)) {
-                                ok = false;
-                                break;
+            for (int pass = 0; pass < passes && ok; ++pass) {
+                for (int grp = 0; grp < G && ok; ++grp) {
+                    const int i0 = grp * TB;
+                    const int ntg = min(nt, i0 + TB) - i0;
+                    for (int c = 0; c < n_chunks && ok; ++c) {
+                        if (q_loader) {
+                            if (lane == 0) {
+                                ok = mbar_wait(&sm->q_empty[qs], qph ^ 1u, abort_flag, a.err);
+                                if (ok) {
+                                    mbar_arrive_expect_tx(&sm->q_full[qs], kQTile);
+                                    tma_load_2d(q_buf + qs * kQTile, &mapQ, &sm->q_full[qs], c * 64, g * HH);
+                                    q_issued |= 1u << qs;
+                                    q_last = (q_last & ~(1u << qs)) | (qph << qs);
+                                }
                             }
-                            mbar_arrive_expect_tx(&sm->q_full[qs], kQTile);
-                            tma_load_2d(q_buf + qs * kQTile, &mapQ, &sm->q_full[qs], c * 64, g * HH);
-                            q_issued |= 1u << qs;
-                            q_last = (q_last & ~(1u << qs)) | (qph << qs);
+                            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+                            if (!ok)
+                                break;
                             if (++qs == kQStages) {
                                 qs = 0;
                                 qph ^= 1u;
                             }
-                            for (int i = i0; i < i1; ++i) {
-                                if (!mbar_wait(&sm->a_empty[as], aph ^ 1u, abort_flag, a.err)) {
-                                    ok = false;
-                                    break;
+                        }
+                        for (int i = 0; i < ntg; ++i) {
+                            if (lane == 0)
+                                ok = mbar_wait(&sm->a_empty[as], aph ^ 1u, abort_flag, a.err);
+                            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+                            if (!ok)
+                                break;
+                            const int tile_row0 = (i0 + i) * 128;
+                            const int rows = min(128, nsel - tile_row0);
+                            const uint32_t dst0 = smem_u32(a_buf + as * kATile);
+#pragma unroll
+                            for (int gi = gw; gi < 32; gi += kGatherWarps) {
+                                const int r = 4 * gi + r_in;
+                                if (r < rows) {
+                                    const int prow = rw[tile_row0 + r];
+                                    const char *src = pool_bytes + ((size_t)prow * a.D + c * 64) * 2 + seg * 16;
+                                    const uint32_t dst = dst0 + r * 128 + ((seg ^ (r & 7)) << 4);
+                                    cp_async16(dst, src);
                                 }
-                                const int rows = min(128, nsel - i * 128);
-                                const int r4 = (rows + 3) & ~3;
-                                mbar_arrive_expect_tx(&sm->a_full[as], (uint32_t)r4 * 128u);
-                                uint8_t *dst = a_buf + as * kATile;
-                                const int base_row = i * 128;
-                                const int dummy = b * a.P;
-                                for (int rr = 0; rr < r4; rr += 4) {
-                                    const int k = base_row + rr;
-                                    const int r0 = rw[k];
-                                    const int r1 = (k + 1 < nsel) ? rw[k + 1] : dummy;
-                                    const int r2 = (k + 2 < nsel) ? rw[k + 2] : dummy;
-                                    const int r3 = (k + 3 < nsel) ? rw[k + 3] : dummy;
-                                    tma_gather4(dst + rr * 128, &mapPool, &sm->a_full[as], c * 64, r0, r1, r2, r3);
-                                }
-                                a_issued |= 1u << as;
-                                a_last = (a_last & ~(1u << as)) | (aph << as);
-                                if (++as == kAStages) {
-                                    as = 0;
-                                    aph ^= 1u;
-                                }
+                            }
+                            // arrives once this thread's copies so far have landed
+                            cp_async_mbar_arrive_noinc(&sm->a_full[as]);
+                            if (++as == NA) {
+                                as = 0;
+                                aph ^= 1u;
                             }
                         }
                     }
                 }
             }
-            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
         }
-        if (!ok && lane == 0) {
-            for (int s = 0; s < kAStages; ++s)
-                if (a_issued & (1u << s))
-                    mbar_drain(&sm->a_full[s], (a_last >> s) & 1u);
+        cp_async_wait<0>();
+        if (!ok && q_loader && lane == 0) {
             for (int s = 0; s < kQStages; ++s)
                 if (q_issued & (1u << s))
                     mbar_drain(&sm->q_full[s], (q_last >> s) & 1u);
         }
         __syncwarp();
-    } else if (warp == 1) {
+    } else if (warp == kMmaWarp) {
         // ============================================================ MMA
         const uint32_t idesc = idesc_bf16_f32(128, HH);
         int as = 0, qs = 0;
         uint32_t aph = 0, qph = 0;
         bool ok = true, issued = false;
-        int it = 0, acc_it = 0;
+        int it = 0;
+        int jobs0 = 0, jobs1 = 0;
         for (int gt = blockIdx.x; gt < a.n_tok && ok; gt += gridDim.x, ++it) {
             const int mb = it & 1;
-            const uint32_t mph = (it >> 1) & 1;
-            if (!mbar_wait(&sm->meta_full[mb], mph, abort_flag, a.err)) {
+            const int m3 = it % kMeta;
+            if (!mbar_wait(&sm->meta_full[m3], (it / kMeta) & 1, abort_flag, a.err)) {
                 ok = false;
                 break;
             }
-            const int nsel = sm->nsel[mb];
+            const int nsel = sm->nsel[m3];
             const int nt = (nsel + 127) / 128;
             const int G = n_groups(nsel, TB);
             const int passes = G > 1 ? 2 : 1;
+            const uint32_t dbase = tmem + mb * 256;
             for (int pass = 0; pass < passes && ok; ++pass) {
-                for (int grp = 0; grp < G && ok; ++grp, ++acc_it) {
+                for (int grp = 0; grp < G && ok; ++grp) {
                     const int i0 = grp * TB;
-                    const int i1 = min(nt, i0 + TB);
-                    const int buf = acc_it & 1;
-                    const uint32_t bph = (acc_it >> 1) & 1;
-                    if (!mbar_wait(&sm->acc_empty[buf], bph ^ 1u, abort_flag, a.err)) {
+                    const int ntg = min(nt, i0 + TB) - i0;
+                    const int jb = mb ? jobs1 : jobs0;
+                    if (!mbar_wait(&sm->acc_empty[mb], (jb & 1) ^ 1u, abort_flag, a.err)) {
                         ok = false;
                         break;
                     }
+                    if (mb)
+                        ++jobs1;
+                    else
+                        ++jobs0;
                     tc_fence_after();
                     for (int c = 0; c < n_chunks && ok; ++c) {
                         if (!mbar_wait(&sm->q_full[qs], qph, abort_flag, a.err)) {
@@ -297,7 +425,7 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
                         }
                         tc_fence_after();
                         const uint64_t dq = sdesc_k_sw128(smem_u32(q_buf + qs * kQTile));
-                        for (int i = i0; i < i1; ++i) {
+                        for (int i = 0; i < ntg; ++i) {
                             if (!mbar_wait(&sm->a_full[as], aph, abort_flag, a.err)) {
                                 ok = false;
                                 break;
@@ -305,7 +433,7 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
                             tc_fence_after();
                             if (lane == 0) {
                                 const uint64_t da = sdesc_k_sw128(smem_u32(a_buf + as * kATile));
-                                const uint32_t d_tmem = tmem + buf * 256 + (i - i0) * HH;
+                                const uint32_t d_tmem = dbase + i * HH;
 #pragma unroll
                                 for (int kk = 0; kk < 4; ++kk)
                                     umma_bf16(d_tmem, da + 2 * kk, dq + 2 * kk, idesc, (c | kk) != 0);
@@ -313,7 +441,7 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
                                 issued = true;
                             }
                             __syncwarp();
-                            if (++as == kAStages) {
+                            if (++as == NA) {
                                 as = 0;
                                 aph ^= 1u;
                             }
@@ -331,7 +459,7 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
                     if (!ok)
                         break;
                     if (lane == 0)
-                        umma_commit(&sm->acc_full[buf]);
+                        umma_commit(&sm->acc_full[mb]);
                     __syncwarp();
                 }
             }
@@ -341,46 +469,60 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
             mbar_drain(&sm->drain, 0);
         }
         __syncwarp();
+    }
     } else {
         // ============================================================ epilogue
+        // warpgroups 3 and 4 execute this one setmaxnreg together
+        regs_inc<kHighRegs>();
+        const int wg = (warp - kEpiWarp0) >> 2;  // epilogue group: tokens with it & 1 == wg
         const int q = warp & 3;              // TMEM lane quarter
         const int r = q * 32 + lane;         // row within a 128-slot tile
-        const int et = threadIdx.x - 64;     // 0..127
-        const float scale = a.scale;
-        int it = 0, acc_it = 0;
-        bool ok = true;
-        for (int gt = blockIdx.x; gt < a.n_tok && ok; gt += gridDim.x, ++it) {
+        const int et = (warp - kEpiWarp0 - 4 * wg) * 32 + lane;  // 0..127 within the group
+        const uint32_t bar_id = 1 + wg;
+        EpiState<HH> &st = sm->epi[wg];
+        float *ub = ubuf + wg * Kp;
+        const float s2 = a.scale * kLog2e;   // scale > 0 (checked on the host)
+        const float sink_h = (a.sink && et < HH) ? a.sink[et] : -INFINITY;
+        int jobs = 0;
+        for (int it = wg; blockIdx.x + it * (int)gridDim.x < a.n_tok; it += 2) {
+            const int gt = blockIdx.x + it * gridDim.x;
             const int g = a.n_tok - 1 - gt;
-            const int mb = it & 1;
-            const uint32_t mph = (it >> 1) & 1;
-            if (!mbar_wait(&sm->meta_full[mb], mph, abort_flag, a.err)) {
-                ok = false;
+            const int m3 = it % kMeta;
+            // window log-mass of this token's heads, fetched early
+            const float wl_h = (et < HH) ? a.wl[(size_t)g * HH + et] : 0.f;
+            // leader waits; the named barrier hands the outcome to the group
+            if (et == 0)
+                st.flag = mbar_wait(&sm->meta_full[m3], (it / kMeta) & 1, abort_flag, a.err) ? 1 : 0;
+            named_bar_sync(bar_id, 128);
+            if (!st.flag)
                 break;
-            }
-            const int nsel = sm->nsel[mb];
+            const int nsel = sm->nsel[m3];
             const int nt = (nsel + 127) / 128;
             const int G = n_groups(nsel, TB);
             const int passes = G > 1 ? 2 : 1;
             float *prow = a.p + (size_t)g * K;
-            const int32_t *sl = slot + mb * K;
+            const int32_t *sl = slot + m3 * Kp;
+            const uint32_t tbase = tmem + wg * 256 + ((uint32_t)(q * 32) << 16);
             float m_part = 0.f;
-            float At = 0.f;  // max_h (M[h] - lse_full[h])
+            float At = 0.f;
+            bool ok = true;
             for (int pass = 0; pass < passes && ok; ++pass) {
-                for (int grp = 0; grp < G; ++grp, ++acc_it) {
+                for (int grp = 0; grp < G; ++grp) {
                     const int i0 = grp * TB;
-                    const int ntg = min(nt, i0 + TB) - i0;   // tiles in this group (>= 1)
-                    const int buf = acc_it & 1;
-                    const uint32_t bph = (acc_it >> 1) & 1;
-                    if (!mbar_wait(&sm->acc_full[buf], bph, abort_flag, a.err)) {
+                    const int ntg = min(nt, i0 + TB) - i0;
+                    named_bar_sync(bar_id, 128);   // st.flag is free again
+                    if (et == 0)
+                        st.flag = mbar_wait(&sm->acc_full[wg], jobs & 1, abort_flag, a.err) ? 1 : 0;
+                    named_bar_sync(bar_id, 128);
+                    if (!st.flag) {
                         ok = false;
                         break;
                     }
+                    ++jobs;
                     tc_fence_after();
-                    const uint32_t tbase = tmem + buf * 256 + ((uint32_t)(q * 32) << 16);
-                    const bool stats = (pass == 0);
                     const bool single = (G == 1);
-                    if (stats) {
-                        // ---- column max over this group's rows
+                    if (pass == 0) {
+                        // ---- column max of the raw dot products over valid rows
                         for (int cc = 0; cc < NC16; ++cc) {
                             float v16[16];
 #pragma unroll
@@ -395,30 +537,29 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
                                 tmem_ld_wait();
 #pragma unroll
                                 for (int i = 0; i < IB; ++i) {
-                                    const bool row_ok = (ib + i < ntg) && ((i0 + ib + i) * 128 + r < nsel);
+                                    if (ib + i < ntg && (i0 + ib + i) * 128 + r < nsel) {
 #pragma unroll
-                                    for (int e = 0; e < 16; ++e)
-                                        v16[e] = row_ok ? fmaxf(v16[e], __uint_as_float(v[i][e]) * scale) : v16[e];
+                                        for (int e = 0; e < 16; ++e)
+                                            v16[e] = fmaxf(v16[e], __uint_as_float(v[i][e]));
+                                    }
                                 }
                             }
                             const float red = warp_colreduce16(v16, OpMax());
                             if (lane < 16)
-                                sm->red_max[q][cc * 16 + lane] = red;
+                                st.red_max[q][cc * 16 + lane] = red;
                         }
-                        named_bar_sync(1, 128);
-                        if (et < HH) {
-                            const float gm = fmaxf(fmaxf(sm->red_max[0][et], sm->red_max[1][et]),
-                                                   fmaxf(sm->red_max[2][et], sm->red_max[3][et]));
-                            sm->head_a[et] = gm;   // group max, staged
-                        }
-                        named_bar_sync(1, 128);
-                        // ---- sum of exp(z - group max); single group: keep e in TMEM
+                        named_bar_sync(bar_id, 128);
+                        if (et < HH)
+                            st.head_a[et] = fmaxf(fmaxf(st.red_max[0][et], st.red_max[1][et]),
+                                                  fmaxf(st.red_max[2][et], st.red_max[3][et])) * s2;
+                        named_bar_sync(bar_id, 128);
+                        // ---- e = 2^(v s2 - max s2), column sums; one group: keep e in TMEM
                         for (int cc = 0; cc < NC16; ++cc) {
-                            float s16[16], gm16[16];
+                            float s16[16], m16[16];
 #pragma unroll
                             for (int e = 0; e < 16; ++e) {
                                 s16[e] = 0.f;
-                                gm16[e] = sm->head_a[cc * 16 + e] * kLog2e;
+                                m16[e] = st.head_a[cc * 16 + e];
                             }
                             for (int ib = 0; ib < ntg; ib += IB) {
                                 uint32_t v[IB][16];
@@ -429,13 +570,20 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
                                 tmem_ld_wait();
 #pragma unroll
                                 for (int i = 0; i < IB; ++i) {
-                                    const bool row_ok = (ib + i < ntg) && ((i0 + ib + i) * 128 + r < nsel);
+                                    if (ib + i < ntg) {
+                                        if ((i0 + ib + i) * 128 + r < nsel) {
 #pragma unroll
-                                    for (int e = 0; e < 16; ++e) {
-                                        const float x = ex2_approx(fmaf(__uint_as_float(v[i][e]) * scale, kLog2e, -gm16[e]));
-                                        const float ex = row_ok ? x : 0.f;
-                                        s16[e] += ex;
-                                        v[i][e] = __float_as_uint(ex);
+                                            for (int e = 0; e < 16; ++e) {
+                                                const float x =
+                                                    ex2_approx(fmaf(__uint_as_float(v[i][e]), s2, -m16[e]));
+                                                s16[e] += x;
+                                                v[i][e] = __float_as_uint(x);
+                                            }
+                                        } else {
+#pragma unroll
+                                            for (int e = 0; e < 16; ++e)
+                                                v[i][e] = 0u;
+                                        }
                                     }
                                 }
                                 if (single) {
@@ -447,54 +595,51 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
                             }
                             const float red = warp_colreduce16(s16, OpAdd());
                             if (lane < 16)
-                                sm->red_sum[q][cc * 16 + lane] = red;
+                                st.red_sum[q][cc * 16 + lane] = red;
                         }
                         if (single)
                             tmem_st_wait();
-                        named_bar_sync(1, 128);
+                        named_bar_sync(bar_id, 128);
                         if (et < HH) {
-                            const float gm = sm->head_a[et];
-                            const float gs = sm->red_sum[0][et] + sm->red_sum[1][et] + sm->red_sum[2][et] +
-                                             sm->red_sum[3][et];
+                            // group statistics in the log2 domain: max M2, sum S
+                            const float gm = st.head_a[et];
+                            const float gs = st.red_sum[0][et] + st.red_sum[1][et] + st.red_sum[2][et] +
+                                             st.red_sum[3][et];
                             if (grp == 0) {
-                                sm->colM[et] = gm;
-                                sm->colS[et] = gs;
+                                st.colM[et] = gm;
+                                st.colS[et] = gs;
                             } else {
-                                const float M0 = sm->colM[et], S0 = sm->colS[et];
+                                const float M0 = st.colM[et], S0 = st.colS[et];
                                 const float M1 = fmaxf(M0, gm);
-                                sm->colS[et] = S0 * expf(M0 - M1) + gs * expf(gm - M1);
-                                sm->colM[et] = M1;
+                                st.colS[et] = S0 * exp2f(M0 - M1) + gs * exp2f(gm - M1);
+                                st.colM[et] = M1;
                             }
                         }
-                        named_bar_sync(1, 128);
+                        named_bar_sync(bar_id, 128);
                     }
                     if (pass == passes - 1) {
                         if (grp == 0) {
                             // ---- per-head merge with the window and the sink
                             if (et < HH) {
-                                const float M = sm->colM[et];
-                                const float clse = M + logf(sm->colS[et]);
-                                const float wl = a.wl[(size_t)g * HH + et];
-                                float mm = fmaxf(wl, clse);
-                                float sk = -INFINITY;
-                                if (a.sink) {
-                                    sk = a.sink[et];
-                                    mm = fmaxf(mm, sk);
-                                }
-                                float acc = expf(wl - mm) + expf(clse - mm);
+                                const float M = st.colM[et] * 0.69314718055994531f;  // natural log units
+                                const float clse = M + logf(st.colS[et]);
+                                float mm = fmaxf(fmaxf(wl_h, clse), sink_h);
+                                float acc = expf(wl_h - mm) + expf(clse - mm);
                                 if (a.sink)
-                                    acc += expf(sk - mm);
-                                const float lse_full = mm + logf(acc);
-                                sm->head_a[et] = M - lse_full;
+                                    acc += expf(sink_h - mm);
+                                st.head_a[et] = M - (mm + logf(acc));
                             }
-                            named_bar_sync(1, 128);
-                            At = -INFINITY;
-                            for (int h = 0; h < HH; ++h)
-                                At = fmaxf(At, sm->head_a[h]);
-                            named_bar_sync(1, 128);
+                            named_bar_sync(bar_id, 128);
+                            float x = -INFINITY;
+                            for (int h = lane; h < HH; h += 32)
+                                x = fmaxf(x, st.head_a[h]);
+#pragma unroll
+                            for (int o = 16; o >= 1; o >>= 1)
+                                x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
+                            At = x;
                             if (et < HH)
-                                sm->wprime[et] = expf(sm->head_a[et] - At);
-                            named_bar_sync(1, 128);
+                                st.wprime[et] = expf(st.head_a[et] - At);
+                            named_bar_sync(bar_id, 128);
                         }
                         // ---- u'[k] = sum_h e[k,h] w[h]
                         float u[TB];
@@ -502,12 +647,10 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
                         for (int i = 0; i < TB; ++i)
                             u[i] = 0.f;
                         for (int cc = 0; cc < NC16; ++cc) {
-                            float w16[16], m16[16];
+                            float w16[16];
 #pragma unroll
-                            for (int e = 0; e < 16; ++e) {
-                                w16[e] = sm->wprime[cc * 16 + e];
-                                m16[e] = sm->colM[cc * 16 + e] * kLog2e;
-                            }
+                            for (int e = 0; e < 16; ++e)
+                                w16[e] = st.wprime[cc * 16 + e];
 #pragma unroll
                             for (int ib = 0; ib < TB; ib += IB) {
                                 if (ib >= ntg)
@@ -522,12 +665,16 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
                                 for (int i = 0; i < IB; ++i) {
                                     if (ib + i < ntg) {
                                         float acc = u[ib + i];
+                                        if (single) {
 #pragma unroll
-                                        for (int e = 0; e < 16; ++e) {
-                                            float ex = __uint_as_float(v[i][e]);
-                                            if (!single)
-                                                ex = ex2_approx(fmaf(ex * scale, kLog2e, -m16[e]));
-                                            acc = fmaf(ex, w16[e], acc);
+                                            for (int e = 0; e < 16; ++e)
+                                                acc = fmaf(__uint_as_float(v[i][e]), w16[e], acc);
+                                        } else {
+#pragma unroll
+                                            for (int e = 0; e < 16; ++e)
+                                                acc = fmaf(ex2_approx(fmaf(__uint_as_float(v[i][e]), s2,
+                                                                           -st.colM[cc * 16 + e])),
+                                                           w16[e], acc);
                                         }
                                         u[ib + i] = acc;
                                     }
@@ -538,7 +685,7 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
                         for (int i = 0; i < TB; ++i) {
                             const int j = (i0 + i) * 128 + r;
                             if (i < ntg && j < nsel) {
-                                ubuf[j] = u[i];
+                                ub[j] = u[i];
                                 m_part += u[i];
                             }
                         }
@@ -546,7 +693,7 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0)
-                        mbar_arrive(&sm->acc_empty[buf]);
+                        mbar_arrive(&sm->acc_empty[wg]);
                 }
             }
             if (!ok)
@@ -557,31 +704,27 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
             for (int o = 16; o >= 1; o >>= 1)
                 mt += __shfl_xor_sync(0xffffffffu, mt, o);
             if (lane == 0)
-                sm->red_m[q] = mt;
-            named_bar_sync(1, 128);
-            const float mtot = sm->red_m[0] + sm->red_m[1] + sm->red_m[2] + sm->red_m[3];
+                st.red_m[q] = mt;
+            named_bar_sync(bar_id, 128);
+            const float mtot = st.red_m[0] + st.red_m[1] + st.red_m[2] + st.red_m[3];
             if (nsel > 0) {
                 const bool plain = logf(mtot) + At >= kLnFltMin;
-                const float f = plain ? 0.f : expf(At - kLnFltMin);
-                for (int jj = et; jj < K; jj += 128) {
-                    float v = 0.f;
-                    if (jj < nsel)
-                        v = plain ? ubuf[jj] / mtot : ubuf[jj] * f;
-                    prow[sl[jj]] = v;
-                }
+                const float f = plain ? 1.0f / mtot : expf(At - kLnFltMin);
+                for (int jj = et; jj < K; jj += 128)
+                    prow[sl[jj]] = (jj < nsel) ? ub[jj] * f : 0.f;
             } else {
                 for (int jj = et; jj < K; jj += 128)
                     prow[jj] = 0.f;
             }
-            named_bar_sync(1, 128);
+            named_bar_sync(bar_id, 128);
             if (et == 0)
-                mbar_arrive(&sm->meta_empty[mb]);
+                mbar_arrive(&sm->meta_empty[m3]);
         }
     }
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 0) {
+    if (warp == kMmaWarp) {
         tc_fence_after();
         tmem_dealloc(tmem, 512);
     }
@@ -590,20 +733,27 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
 template <int HH>
 size_t smem_bytes_for(int K)
 {
-    return 1024 + kAStages * kATile + kQStages * (HH * 128) + (size_t)K * (4 + 4) * 2 + (size_t)K * 4 + 16 +
+    const size_t Kp = (size_t)((K + 3) & ~3);
+    return 1024 + (size_t)a_stages_for(K) * kATile + kQStages * (HH * 128) + Kp * 4 * (2 * kMeta + 4) +
            sizeof(TgtSmem<HH>) + 64;
 }
 
 template <int HH>
-cudaError_t launch_h(const CUtensorMap &mapQ, const CUtensorMap &mapPool, const TgtTcArgs &a, int grid,
-                     cudaStream_t stream)
+cudaError_t launch_h(const CUtensorMap &mapQ, const TgtTcArgs &a, int grid, cudaStream_t stream)
 {
-    const size_t smem = smem_bytes_for<HH>(a.K);
-    cudaError_t e =
-        cudaFuncSetAttribute(target_tc_kernel<HH>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    // The register split above is only safe if every thread was launched with
+    // exactly kLaunchRegs registers; refuse to launch otherwise.
+    cudaFuncAttributes fa;
+    cudaError_t e = cudaFuncGetAttributes(&fa, target_tc_kernel<HH>);
     if (e != cudaSuccess)
         return e;
-    target_tc_kernel<HH><<<grid, kTgtThreads, smem, stream>>>(mapQ, mapPool, a);
+    if (fa.numRegs != kLaunchRegs)
+        return cudaErrorInvalidConfiguration;
+    const size_t smem = smem_bytes_for<HH>(a.K);
+    e = cudaFuncSetAttribute(target_tc_kernel<HH>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess)
+        return e;
+    target_tc_kernel<HH><<<grid, kTgtThreads, smem, stream>>>(mapQ, a);
     return cudaGetLastError();
 }
 
@@ -620,14 +770,13 @@ size_t target_tc_smem_bytes(int H, int K)
     }
 }
 
-cudaError_t launch_target_tc(const CUtensorMap &mapQ, const CUtensorMap &mapPool, const TgtTcArgs &a, int grid,
-                             cudaStream_t stream)
+cudaError_t launch_target_tc(const CUtensorMap &mapQ, const TgtTcArgs &a, int grid, cudaStream_t stream)
 {
     switch (a.H) {
-    case 16: return launch_h<16>(mapQ, mapPool, a, grid, stream);
-    case 32: return launch_h<32>(mapQ, mapPool, a, grid, stream);
-    case 64: return launch_h<64>(mapQ, mapPool, a, grid, stream);
-    case 128: return launch_h<128>(mapQ, mapPool, a, grid, stream);
+    case 16: return launch_h<16>(mapQ, a, grid, stream);
+    case 32: return launch_h<32>(mapQ, a, grid, stream);
+    case 64: return launch_h<64>(mapQ, a, grid, stream);
+    case 128: return launch_h<128>(mapQ, a, grid, stream);
     default: return cudaErrorInvalidValue;
     }
 }

@@ -14,21 +14,21 @@
 // the sequence are zero-filled or belong to the previous sequence and are
 // masked). One MMA chain of D/64 x 4 steps (M=128, N=NB, K=16) puts the
 // 128 x NB logits in TMEM; the epilogue reads one row per thread and reduces
-// it with a masked two-pass max / sum-exp.
+// it with a masked two-pass max / sum-exp over the columns of its window.
 //
-// Warp roles (192 threads): warp 0 TMA producer (and TMEM owner), warp 1 MMA
-// issuer, warps 2..5 epilogue (TMEM lane quarters 2,3,0,1). TMEM holds two
-// 256-column accumulators so the epilogue of one tile overlaps the MMA of the
-// next. Every wait is bounded; on timeout the kernel writes NaN rows and
-// unwinds.
+// Warp roles (320 threads): warp 0 TMA producer (and TMEM owner), warp 1 MMA
+// issuer, warps 2..5 and 6..9 two epilogue groups that take alternate tiles,
+// each with its own 256-column TMEM accumulator. The kernel is bound by
+// reading Q from HBM once; six 34 KB stages keep enough bytes in flight.
+// Every wait is bounded; on timeout the kernel writes NaN rows and unwinds.
 #include "sai_device.cuh"
 #include "sai_kernels.h"
 
 namespace sai {
 namespace {
 
-constexpr int kWinStages = 4;
-constexpr int kWinThreads = 192;
+constexpr int kWinStages = 6;
+constexpr int kWinThreads = 320;
 constexpr uint32_t kATileBytes = 128 * 128;  // 128 rows x 64 bf16
 
 struct WinSmem {
@@ -46,7 +46,6 @@ __global__ void __launch_bounds__(kWinThreads, 1)
                          const WinTcArgs a)
 {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
-    // Stage buffers first (1024-aligned), bookkeeping after them.
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t b_bytes = a.b_stage_bytes;  // NB x 128, rounded to 1024
     const uint32_t stage_bytes = kATileBytes + b_bytes;
@@ -171,67 +170,85 @@ __global__ void __launch_bounds__(kWinThreads, 1)
         __syncwarp();
     } else {
         // ------------------------------------------------ epilogue
+        const int wg = (warp - 2) >> 2;    // takes tiles j with j & 1 == wg
         const int q = warp & 3;            // TMEM lane quarter of this warp
         const int r = q * 32 + lane;       // tile row
-        const float scale = a.scale;
+        const float s2 = a.scale * 1.4426950408889634f;  // scale > 0 (checked on the host)
         const int ncol16 = a.NB / 16;
-        int j = 0;
-        for (int tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++j) {
-            const int buf = j & 1;
-            const uint32_t aphase = (j >> 1) & 1;
+        const int rt = r / a.H;            // token of this row within the tile
+        const int h = r - rt * a.H;
+        int j = wg;
+        int uses = 0;
+        for (int tile = blockIdx.x + wg * gridDim.x; tile < n_tiles; tile += 2 * gridDim.x, j += 2, ++uses) {
             const int g0 = tile * a.TQ;
-            const int g = g0 + r / a.H;
-            const int h = r - (r / a.H) * a.H;
+            const int g = g0 + rt;
             const int b = g0 / a.S;
             const int t = g - b * a.S;
             const int t0 = g0 - b * a.S;
-            if (!mbar_wait(&sm->acc_full[buf], aphase, abort_flag, nullptr)) {
-                a.out[(size_t)g * a.H + h] = __int_as_float(0x7fc00000);
-                break;
-            }
-            tc_fence_after();
             int d0 = 0;
             if (a.doc_start) {
                 d0 = a.doc_start[g];
                 d0 = d0 < 0 ? 0 : (d0 > t ? t : d0);
             }
+            if (!mbar_wait(&sm->acc_full[wg], uses & 1, abort_flag, nullptr)) {
+                a.out[(size_t)g * a.H + h] = __int_as_float(0x7fc00000);
+                break;
+            }
+            tc_fence_after();
             const int lo = max(d0, t - a.W + 1);
             const int band0 = t0 - a.W + 1;      // key of band column 0
             const int clo = lo - band0, chi = t - band0;
-            const uint32_t taddr = tmem + buf * 256 + ((uint32_t)(q * 32) << 16);
+            // chunks any row of this warp needs
+            int wlo = clo, whi = chi;
+#pragma unroll
+            for (int o = 16; o >= 1; o >>= 1) {
+                wlo = min(wlo, __shfl_xor_sync(0xffffffffu, wlo, o));
+                whi = max(whi, __shfl_xor_sync(0xffffffffu, whi, o));
+            }
+            const int c_begin = wlo >> 4, c_end = min(ncol16 - 1, whi >> 4);
+            const uint32_t taddr = tmem + wg * 256 + ((uint32_t)(q * 32) << 16);
             float mx = -INFINITY;
-            for (int cc = 0; cc < ncol16; ++cc) {
+            for (int cc = c_begin; cc <= c_end; ++cc) {
                 uint32_t v[16];
                 tmem_ld16(taddr + cc * 16, v);
                 tmem_ld_wait();
+                const int c0 = cc * 16;
+                if (c0 >= clo && c0 + 15 <= chi) {
 #pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    const int col = cc * 16 + e;
-                    const float z = __uint_as_float(v[e]) * scale;
-                    if (col >= clo && col <= chi)
-                        mx = fmaxf(mx, z);
+                    for (int e = 0; e < 16; ++e)
+                        mx = fmaxf(mx, __uint_as_float(v[e]));
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 16; ++e)
+                        if (c0 + e >= clo && c0 + e <= chi)
+                            mx = fmaxf(mx, __uint_as_float(v[e]));
                 }
             }
-            const float l2e = 1.4426950408889634f;
+            const float m2 = mx * s2;
             float sum = 0.f;
-            for (int cc = 0; cc < ncol16; ++cc) {
+            for (int cc = c_begin; cc <= c_end; ++cc) {
                 uint32_t v[16];
                 tmem_ld16(taddr + cc * 16, v);
                 tmem_ld_wait();
+                const int c0 = cc * 16;
+                if (c0 >= clo && c0 + 15 <= chi) {
 #pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    const int col = cc * 16 + e;
-                    const float z = __uint_as_float(v[e]) * scale;
-                    const float x = ex2_approx((z - mx) * l2e);
-                    sum += (col >= clo && col <= chi) ? x : 0.f;
+                    for (int e = 0; e < 16; ++e)
+                        sum += ex2_approx(fmaf(__uint_as_float(v[e]), s2, -m2));
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 16; ++e)
+                        if (c0 + e >= clo && c0 + e <= chi)
+                            sum += ex2_approx(fmaf(__uint_as_float(v[e]), s2, -m2));
                 }
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0)
-                mbar_arrive(&sm->acc_empty[buf]);
-            a.out[(size_t)g * a.H + h] = mx + logf(sum);
+                mbar_arrive(&sm->acc_empty[wg]);
+            a.out[(size_t)g * a.H + h] = mx * a.scale + logf(sum);
         }
+        (void)j;
     }
 
     tc_fence_before();

@@ -52,7 +52,8 @@ def check_full(sai, w, *, err_expect=0):
     # bit-exact masks: p is exactly 0 wherever the oracle's is
     assert np.all(pg[op == 0] == 0)
     lg = float(loss.item())
-    assert abs(lg - oloss) <= TOL_LOSS_REL * abs(oloss), (lg, oloss)
+    # a float32 result cannot resolve below its spacing at zero (2^-149)
+    assert abs(lg - oloss) <= TOL_LOSS_REL * abs(oloss) + 2.0 ** -149, (lg, oloss)
     dg = ds.cpu().numpy().reshape(-1, w.K)
     assert_close("dscores", dg, ods, TOL_DS)
     assert np.abs(dg - ods).max() <= TOL_DS_REL_MAX * max(np.abs(ods).max(), 1e-30)
@@ -73,6 +74,11 @@ def test_small_full(sai):
 def test_flash_recipe_ragged_tiles(sai):
     """H=64, D=512 tensor-core path; K=200 leaves a ragged last tile."""
     check_full(sai, workload("flash_s1024_k200", name="flash", S=1024, K=200))
+
+
+def test_flash_recipe_odd_k(sai):
+    """K not a multiple of 4: idx rows are read directly, not staged."""
+    check_full(sai, synth.make("flash", S=512, K=101, seed=4242))
 
 
 def test_packed_recipe_documents(sai):
