@@ -13,6 +13,7 @@ bf16 tensors may be passed as torch.bfloat16 or as int16/uint16 bit patterns.
 from __future__ import annotations
 
 import ctypes
+import importlib.util
 import os
 from typing import Optional, Tuple
 
@@ -21,9 +22,20 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libsai.so")
 
-if not os.path.exists(LIB_PATH):
-    raise ImportError(f"libsai.so is not built ({LIB_PATH}); run "
-                      "`python -m sparse_attention_indexer_window_b200.build`")
+
+def _builder():
+    spec = importlib.util.spec_from_file_location("_sai_build", os.path.join(_HERE, "build.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
+
+
+# Rebuild when a source is newer than the library (a no-op otherwise).
+try:
+    _builder().build()
+except Exception as exc:  # no nvcc here: only an existing, current library will do
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"libsai.so is not built ({LIB_PATH}) and cannot be built: {exc}") from exc
 
 _lib = ctypes.CDLL(LIB_PATH)
 _P = ctypes.c_void_p

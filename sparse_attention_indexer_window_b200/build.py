@@ -1,6 +1,9 @@
 """Build libsai.so in-tree with nvcc for sm_100a.
 
-    python -m sparse_attention_indexer_window_b200.build
+    python sparse_attention_indexer_window_b200/build.py [--force] [--ptxas-v]
+
+Runs as a plain script (it does not import the package, which loads the
+library it builds).
 """
 from __future__ import annotations
 

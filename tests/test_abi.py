@@ -13,8 +13,6 @@ HEADER = os.path.join(ROOT, "include", "sai.h")
 
 @pytest.fixture(scope="module")
 def sai():
-    from sparse_attention_indexer_window_b200 import build
-    build.build()
     import sparse_attention_indexer_window_b200 as m
     return m
 

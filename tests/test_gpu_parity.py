@@ -24,8 +24,6 @@ torch = pytest.importorskip("torch")
 
 @pytest.fixture(scope="module")
 def sai():
-    from sparse_attention_indexer_window_b200 import build
-    build.build()
     import sparse_attention_indexer_window_b200 as m
     return m
 
