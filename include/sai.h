@@ -155,6 +155,31 @@ sai_status sai_distill_kl(const float *p, const float *scores, const uint8_t *va
                           float *loss, float *dscores, void *workspace, size_t ws_bytes,
                           void *stream);
 
+/*
+ * sai_distill_kl_noalloc -- sai_distill_kl for callers that cannot allocate.
+ *
+ * The source pages have no counterpart to this call; it is a library
+ * convenience. Same inputs, outputs, arithmetic and errors as sai_distill_kl,
+ * but there is no workspace argument: the scratch words live in a fixed device
+ * array inside the library (sai_distill_kl_noalloc_max_scratch_bytes() bytes,
+ * held by every GPU that loads the library until the process exits). It calls
+ * no cudaMalloc/cudaFree and no allocating library routine, so it suits a
+ * caller whose framework owns all device memory, or one that must avoid the
+ * device-wide synchronisation an allocation can bring.
+ *
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture begins.
+ *   - Every call on a device shares the one array: calls that overlap on the
+ *     GPU (other streams, other host threads) race and can corrupt each
+ *     other's loss. Nothing needs clearing between calls.
+ *   - Sizes whose scratch would exceed the array return SAI_ERR_WORKSPACE.
+ */
+size_t sai_distill_kl_noalloc_max_scratch_bytes(void);
+sai_status sai_distill_kl_noalloc(const float *p, const float *scores, const uint8_t *valid,
+                                  int B, int S, int K, float coeff,
+                                  float *loss, float *dscores, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -49,6 +49,10 @@ _lib.sai_distill_kl_workspace_bytes.argtypes = [_I, _I, _I]
 _lib.sai_distill_kl_workspace_bytes.restype = ctypes.c_size_t
 _lib.sai_distill_kl.argtypes = [_P, _P, _P, _I, _I, _I, _F, _P, _P, _P, ctypes.c_size_t, _P]
 _lib.sai_distill_kl.restype = _I
+_lib.sai_distill_kl_noalloc.argtypes = [_P, _P, _P, _I, _I, _I, _F, _P, _P, _P]
+_lib.sai_distill_kl_noalloc.restype = _I
+_lib.sai_distill_kl_noalloc_max_scratch_bytes.argtypes = []
+_lib.sai_distill_kl_noalloc_max_scratch_bytes.restype = ctypes.c_size_t
 _lib.sai_status_string.argtypes = [_I]
 _lib.sai_status_string.restype = ctypes.c_char_p
 _lib.sai_version.argtypes = []
@@ -179,6 +183,26 @@ def distill_kl(p: torch.Tensor, scores: torch.Tensor, valid: torch.Tensor, coeff
                              _stream(scores.device))
     _check(st, "sai_distill_kl")
     return loss, dscores
+
+
+def distill_kl_noalloc(p: torch.Tensor, scores: torch.Tensor, valid: torch.Tensor, coeff: float,
+                       loss: torch.Tensor, dscores: Optional[torch.Tensor] = None) -> None:
+    """sai_distill_kl_noalloc: the KL call for callers that cannot allocate.
+
+    Writes into the caller's ``loss`` (and ``dscores``, if given) without any
+    workspace: the library keeps its scratch in a fixed device array. Calls
+    running at the same time on one GPU share that array and race."""
+    B, S, K = scores.shape
+    _want(p, "p", torch.float32, (B, S, K))
+    _want(scores, "scores", torch.float32, (B, S, K))
+    if valid.dtype == torch.bool:
+        valid = valid.view(torch.uint8)
+    _want(valid, "valid", torch.uint8, (B, S, K))
+    _want(loss, "loss", torch.float32)
+    _want(dscores, "dscores", torch.float32, (B, S, K))
+    st = _lib.sai_distill_kl_noalloc(_ptr(p), _ptr(scores), _ptr(valid), B, S, K, float(coeff), _ptr(loss),
+                                     _ptr(dscores), _stream(scores.device))
+    _check(st, "sai_distill_kl_noalloc")
 
 
 def distill_loss(Q, Kw, pool, idx, scores, valid, *, W: int, cr: int, scale: float, coeff: float,
