@@ -151,13 +151,13 @@ __device__ __forceinline__ float kl_row_vec(const float *__restrict__ pr, const 
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
             const bool v = (vv[j] >> (8 * e)) & 0xffu;
-            se += v ? expf(s4[e] - mx) : 0.f;
+            se += v ? __expf(s4[e] - mx) : 0.f;
             ps += v ? p4[e] : 0.f;
         }
     }
     se = warp_sum(se);
     ps = warp_sum(ps);
-    const float lse = mx + logf(se);
+    const float lse = mx + __logf(se);
     float kl = 0.f;
 #pragma unroll
     for (int j = 0; j < NV; ++j) {
@@ -168,8 +168,8 @@ __device__ __forceinline__ float kl_row_vec(const float *__restrict__ pr, const 
         for (int e = 0; e < 4; ++e) {
             const bool v = (vv[j] >> (8 * e)) & 0xffu;
             const float logq = s4[e] - lse;
-            kl += (v && p4[e] > 0.f) ? p4[e] * (logf(p4[e]) - logq) : 0.f;
-            d4[e] = v ? c * fmaf(expf(logq), ps, -p4[e]) : 0.f;
+            kl += (v && p4[e] > 0.f) ? p4[e] * (__logf(p4[e]) - logq) : 0.f;
+            d4[e] = v ? c * fmaf(__expf(logq), ps, -p4[e]) : 0.f;
         }
         const int k = 4 * lane + 128 * j;
         if (dr && k < K)
@@ -190,10 +190,10 @@ __device__ __forceinline__ float kl_row_any(const float *__restrict__ pr, const 
             const float s = sr[k];
             any = true;
             if (s > mx) {
-                se = se * expf(mx - s) + 1.f;
+                se = se * __expf(mx - s) + 1.f;
                 mx = s;
             } else {
-                se += expf(s - mx);
+                se += __expf(s - mx);
             }
             ps += pr[k];
         }
@@ -205,24 +205,24 @@ __device__ __forceinline__ float kl_row_any(const float *__restrict__ pr, const 
         return 0.f;
     }
     const float gmx = warp_max(mx);
-    se = (mx == -INFINITY) ? 0.f : se * expf(mx - gmx);
+    se = (mx == -INFINITY) ? 0.f : se * __expf(mx - gmx);
     se = warp_sum(se);
     ps = warp_sum(ps);
-    const float lse = gmx + logf(se);
+    const float lse = gmx + __logf(se);
     float kl = 0.f;
     for (int k = lane; k < K; k += 32) {
         const bool v = vr[k] != 0;
         const float p = pr[k];
         const float logq = sr[k] - lse;
-        kl += (v && p > 0.f) ? p * (logf(p) - logq) : 0.f;
+        kl += (v && p > 0.f) ? p * (__logf(p) - logq) : 0.f;
         if (dr)
-            dr[k] = v ? c * fmaf(expf(logq), ps, -p) : 0.f;
+            dr[k] = v ? c * fmaf(__expf(logq), ps, -p) : 0.f;
     }
     return warp_sum(kl);
 }
 
 template <int NV>
-__global__ void __launch_bounds__(kKlThreads)
+__global__ void __launch_bounds__(kKlThreads, 4)
     kl_rows_kernel(const float *__restrict__ p, const float *__restrict__ scores, const uint8_t *__restrict__ valid,
                    int rows, int K, float coeff, float *loss, float *dscores, void *ws, int count_blocks)
 {
@@ -271,13 +271,24 @@ __global__ void __launch_bounds__(kKlThreads)
         last = (prev == gridDim.x - 1);
     }
     __syncthreads();
-    if (last && threadIdx.x == 0) {
+    if (last) {
+        // fixed-order parallel sum of the per-block partials
         __threadfence();
         const volatile double *kp = w.kl_part;
         double s = 0.0;
-        for (int i = 0; i < (int)gridDim.x; ++i)
+        for (int i = threadIdx.x; i < (int)gridDim.x; i += blockDim.x)
             s += kp[i];
-        *loss = (float)((double)coeff * s / (double)(N > 1 ? N : 1));
+        for (int o = 16; o >= 1; o >>= 1)
+            s += __shfl_xor_sync(0xffffffffu, s, o);
+        if (lane == 0)
+            wkl[warp] = s;
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            double t = 0.0;
+            for (int i = 0; i < kKlWarps; ++i)
+                t += wkl[i];
+            *loss = (float)((double)coeff * t / (double)(N > 1 ? N : 1));
+        }
     }
 }
 

@@ -161,7 +161,10 @@ sai_status sai_distill_target(const uint16_t *Q, const uint16_t *pool, const int
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const int smem_cap = max_smem_optin();
 
-    if (tc_heads(H) && (D % 64) == 0 && (int)sai::target_tc_smem_bytes(H, K) <= smem_cap) {
+    // the tensor-core kernel addresses pool rows with 32-bit byte offsets
+    const bool pool_fits = (uint64_t)B * P * D * 2 < 0xffffffffull;
+    const int n_astages = tc_heads(H) && (D % 64) == 0 && pool_fits ? sai::target_tc_stages(H, K, smem_cap) : 0;
+    if (n_astages > 0) {
         sai::TgtTcArgs a;
         a.B = B;
         a.S = S;
@@ -173,6 +176,7 @@ sai_status sai_distill_target(const uint16_t *Q, const uint16_t *pool, const int
         a.n_tok = B * S;
         a.tiles_per_group = 256 / H;
         a.idx_bulk = ((K % 4) == 0 && al16(idx)) ? 1 : 0;
+        a.n_astages = n_astages;
         a.scale = scale;
         a.pool = pool;
         a.idx = idx;

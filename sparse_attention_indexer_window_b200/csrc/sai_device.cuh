@@ -270,12 +270,14 @@ __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads)
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
-// 2^x with the hardware approximation (relative error about 2^-22),
-// subnormal results kept (no flush to zero).
+// 2^x with the hardware approximation (relative error about 2^-22); results
+// below 2^-126 flush to zero. Callers only exponentiate differences to a
+// maximum (x <= 0) and use the results in sums that contain a 1, so a flushed
+// term changes the result by less than 2^-126 relative.
 __device__ __forceinline__ float ex2_approx(float x)
 {
     float y;
-    asm("ex2.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
 }
 

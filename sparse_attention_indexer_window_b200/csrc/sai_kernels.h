@@ -30,6 +30,7 @@ struct TgtTcArgs {
     int n_tok;            // B*S
     int tiles_per_group;  // 128-slot tiles per TMEM accumulator (256 / H)
     int idx_bulk;         // idx rows are 16-byte aligned (K % 4 == 0): stage them by bulk copy
+    int n_astages;        // depth of the gathered-row stage ring
     float scale;
     const uint16_t *pool;
     const int32_t *idx;
@@ -39,7 +40,8 @@ struct TgtTcArgs {
     float *p;
     int32_t *err;
 };
-size_t target_tc_smem_bytes(int H, int K);
+// Deepest gathered-row stage ring that fits `smem_limit` bytes (0: none).
+int target_tc_stages(int H, int K, int smem_limit);
 cudaError_t launch_target_tc(const CUtensorMap &mapQ, const TgtTcArgs &a, int grid, cudaStream_t stream);
 
 // ------------------------------------------- generic CUDA-core kernels

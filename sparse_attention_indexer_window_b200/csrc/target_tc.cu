@@ -72,7 +72,7 @@ constexpr int kLaunchRegs = 96;
 constexpr int kLowRegs = 56;
 constexpr int kHighRegs = 152;
 static_assert(384 * kLowRegs + 256 * kHighRegs <= kTgtThreads * kLaunchRegs, "register split");
-constexpr int kMaxAStages = 8;
+constexpr int kMaxAStages = 12;
 constexpr int kQStages = 3;
 constexpr int kMeta = 3;                            // compaction runs up to two tokens ahead
 constexpr uint32_t kATile = 128 * 128;              // 128 rows x 128 bytes
@@ -105,7 +105,9 @@ struct TgtSmem {
     EpiState<HH> epi[2];
 };
 
-__host__ __device__ inline int a_stages_for(int K) { return K <= 1024 ? kMaxAStages : 6; }
+// Bytes of dynamic smem other than the A-stage ring.
+template <int HH>
+__host__ __device__ inline size_t fixed_smem_bytes(int K);
 
 __device__ __forceinline__ int n_groups(int nsel, int TB)
 {
@@ -132,7 +134,7 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int K = a.K;
     const int Kp = (K + 3) & ~3;
-    const int NA = a_stages_for(K);
+    const int NA = a.n_astages;              // A-stage ring depth (sized on the host)
     uint8_t *a_buf = base;                                                   // NA x 16 KB
     uint8_t *q_buf = a_buf + NA * kATile;                                    // kQStages x H*128
     int32_t *rowid = reinterpret_cast<int32_t *>(q_buf + kQStages * kQTile); // [kMeta][Kp]
@@ -328,6 +330,22 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
                 for (int grp = 0; grp < G && ok; ++grp) {
                     const int i0 = grp * TB;
                     const int ntg = min(nt, i0 + TB) - i0;
+                    // byte offsets of this lane's rows in every tile of the group,
+                    // held in registers when the group has at most four tiles
+                    // (all-ones marks a row past the selected slots)
+                    constexpr int NGI = (32 + kGatherWarps - 1) / kGatherWarps;
+                    constexpr int RT = TB < 4 ? TB : 4;
+                    uint32_t roff[RT][NGI];
+#pragma unroll
+                    for (int i = 0; i < RT; ++i)
+#pragma unroll
+                        for (int u = 0; u < NGI; ++u) {
+                            const int gi = gw + u * kGatherWarps;
+                            const int r = 4 * gi + r_in;
+                            const int k = (i0 + i) * 128 + r;
+                            roff[i][u] = (gi < 32 && i < ntg && k < nsel) ? (uint32_t)rw[k] * (uint32_t)(a.D * 2)
+                                                                          : 0xffffffffu;
+                        }
                     for (int c = 0; c < n_chunks && ok; ++c) {
                         if (q_loader) {
                             if (lane == 0) {
@@ -357,11 +375,20 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
                             const int rows = min(128, nsel - tile_row0);
                             const uint32_t dst0 = smem_u32(a_buf + as * kATile);
 #pragma unroll
-                            for (int gi = gw; gi < 32; gi += kGatherWarps) {
+                            for (int u = 0; u < NGI; ++u) {
+                                const int gi = gw + u * kGatherWarps;
                                 const int r = 4 * gi + r_in;
-                                if (r < rows) {
-                                    const int prow = rw[tile_row0 + r];
-                                    const char *src = pool_bytes + ((size_t)prow * a.D + c * 64) * 2 + seg * 16;
+                                uint32_t off = 0xffffffffu;
+                                if (TB <= 4) {
+#pragma unroll
+                                    for (int ii = 0; ii < RT; ++ii)
+                                        if (ii == i)
+                                            off = roff[ii][u];
+                                } else if (gi < 32 && r < rows) {
+                                    off = (uint32_t)rw[tile_row0 + r] * (uint32_t)(a.D * 2);
+                                }
+                                if (gi < 32 && r < rows && off != 0xffffffffu) {
+                                    const char *src = pool_bytes + off + c * 128 + seg * 16;
                                     const uint32_t dst = dst0 + r * 128 + ((seg ^ (r & 7)) << 4);
                                     cp_async16(dst, src);
                                 }
@@ -731,11 +758,27 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
 }
 
 template <int HH>
-size_t smem_bytes_for(int K)
+__host__ __device__ inline size_t fixed_smem_bytes(int K)
 {
     const size_t Kp = (size_t)((K + 3) & ~3);
-    return 1024 + (size_t)a_stages_for(K) * kATile + kQStages * (HH * 128) + Kp * 4 * (2 * kMeta + 4) +
-           sizeof(TgtSmem<HH>) + 64;
+    return 1024 + kQStages * (HH * 128) + Kp * 4 * (2 * kMeta + 4) + sizeof(TgtSmem<HH>) + 64;
+}
+
+// Deepest A-stage ring that fits the per-block smem limit (0 if none does).
+template <int HH>
+int stages_for(int K, int smem_limit)
+{
+    const long room = (long)smem_limit - (long)fixed_smem_bytes<HH>(K);
+    long n = room / (long)kATile;
+    if (n > kMaxAStages)
+        n = kMaxAStages;
+    return n >= 4 ? (int)n : 0;
+}
+
+template <int HH>
+size_t smem_bytes_for(int K, int stages)
+{
+    return fixed_smem_bytes<HH>(K) + (size_t)stages * kATile;
 }
 
 template <int HH>
@@ -749,7 +792,7 @@ cudaError_t launch_h(const CUtensorMap &mapQ, const TgtTcArgs &a, int grid, cuda
         return e;
     if (fa.numRegs != kLaunchRegs)
         return cudaErrorInvalidConfiguration;
-    const size_t smem = smem_bytes_for<HH>(a.K);
+    const size_t smem = smem_bytes_for<HH>(a.K, a.n_astages);
     e = cudaFuncSetAttribute(target_tc_kernel<HH>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess)
         return e;
@@ -759,13 +802,13 @@ cudaError_t launch_h(const CUtensorMap &mapQ, const TgtTcArgs &a, int grid, cuda
 
 }  // namespace
 
-size_t target_tc_smem_bytes(int H, int K)
+int target_tc_stages(int H, int K, int smem_limit)
 {
     switch (H) {
-    case 16: return smem_bytes_for<16>(K);
-    case 32: return smem_bytes_for<32>(K);
-    case 64: return smem_bytes_for<64>(K);
-    case 128: return smem_bytes_for<128>(K);
+    case 16: return stages_for<16>(K, smem_limit);
+    case 32: return stages_for<32>(K, smem_limit);
+    case 64: return stages_for<64>(K, smem_limit);
+    case 128: return stages_for<128>(K, smem_limit);
     default: return 0;
     }
 }

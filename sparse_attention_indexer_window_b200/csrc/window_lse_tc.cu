@@ -207,39 +207,57 @@ __global__ void __launch_bounds__(kWinThreads, 1)
             }
             const int c_begin = wlo >> 4, c_end = min(ncol16 - 1, whi >> 4);
             const uint32_t taddr = tmem + wg * 256 + ((uint32_t)(q * 32) << 16);
+            // two passes (max, then sum of exponentials) over the row's window
+            // columns, three 16-column TMEM loads per wait
             float mx = -INFINITY;
-            for (int cc = c_begin; cc <= c_end; ++cc) {
-                uint32_t v[16];
-                tmem_ld16(taddr + cc * 16, v);
+            for (int cb = c_begin; cb <= c_end; cb += 3) {
+                uint32_t v[3][16];
+#pragma unroll
+                for (int u = 0; u < 3; ++u)
+                    if (cb + u <= c_end)
+                        tmem_ld16(taddr + (cb + u) * 16, v[u]);
                 tmem_ld_wait();
-                const int c0 = cc * 16;
-                if (c0 >= clo && c0 + 15 <= chi) {
 #pragma unroll
-                    for (int e = 0; e < 16; ++e)
-                        mx = fmaxf(mx, __uint_as_float(v[e]));
-                } else {
+                for (int u = 0; u < 3; ++u) {
+                    const int c0 = (cb + u) * 16;
+                    if (cb + u > c_end)
+                        break;
+                    if (c0 >= clo && c0 + 15 <= chi) {
 #pragma unroll
-                    for (int e = 0; e < 16; ++e)
-                        if (c0 + e >= clo && c0 + e <= chi)
-                            mx = fmaxf(mx, __uint_as_float(v[e]));
+                        for (int e = 0; e < 16; ++e)
+                            mx = fmaxf(mx, __uint_as_float(v[u][e]));
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 16; ++e)
+                            if (c0 + e >= clo && c0 + e <= chi)
+                                mx = fmaxf(mx, __uint_as_float(v[u][e]));
+                    }
                 }
             }
             const float m2 = mx * s2;
             float sum = 0.f;
-            for (int cc = c_begin; cc <= c_end; ++cc) {
-                uint32_t v[16];
-                tmem_ld16(taddr + cc * 16, v);
+            for (int cb = c_begin; cb <= c_end; cb += 3) {
+                uint32_t v[3][16];
+#pragma unroll
+                for (int u = 0; u < 3; ++u)
+                    if (cb + u <= c_end)
+                        tmem_ld16(taddr + (cb + u) * 16, v[u]);
                 tmem_ld_wait();
-                const int c0 = cc * 16;
-                if (c0 >= clo && c0 + 15 <= chi) {
 #pragma unroll
-                    for (int e = 0; e < 16; ++e)
-                        sum += ex2_approx(fmaf(__uint_as_float(v[e]), s2, -m2));
-                } else {
+                for (int u = 0; u < 3; ++u) {
+                    const int c0 = (cb + u) * 16;
+                    if (cb + u > c_end)
+                        break;
+                    if (c0 >= clo && c0 + 15 <= chi) {
 #pragma unroll
-                    for (int e = 0; e < 16; ++e)
-                        if (c0 + e >= clo && c0 + e <= chi)
-                            sum += ex2_approx(fmaf(__uint_as_float(v[e]), s2, -m2));
+                        for (int e = 0; e < 16; ++e)
+                            sum += ex2_approx(fmaf(__uint_as_float(v[u][e]), s2, -m2));
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 16; ++e)
+                            if (c0 + e >= clo && c0 + e <= chi)
+                                sum += ex2_approx(fmaf(__uint_as_float(v[u][e]), s2, -m2));
+                    }
                 }
             }
             tc_fence_before();

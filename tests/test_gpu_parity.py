@@ -138,6 +138,19 @@ def test_random_slot_order_permutes_outputs(sai):
     np.testing.assert_allclose(d2.cpu().numpy(), d1.cpu().numpy()[..., perm], rtol=0, atol=1e-9)
 
 
+def test_many_tiles_few_heads(sai):
+    """H=16 with up to 700 selected slots per token: six 128-slot tiles in one
+    TMEM group (row offsets read from shared memory). Sampled tokens."""
+    w = workload("small_s4096_k700", name="small", S=4096, K=700, B=1)
+    t = to_dev(w)
+    wl, p, loss, ds = run_chain(sai, w, t)
+    tok = np.unique(np.concatenate([np.arange(w.S - 24, w.S), synth.sample_tokens(w.B, w.S, 40)]))
+    owl, op, _, ods, bad = oracle.run_all(w, tok)
+    assert_close("window_lse", wl.cpu().numpy().reshape(-1, w.H)[tok] - owl, 0 * owl, tol_wl(owl))
+    assert_close("p", p.cpu().numpy().reshape(-1, w.K)[tok], op, TOL_P)
+    assert_close("dscores", ds.cpu().numpy().reshape(-1, w.K)[tok], ods, TOL_DS)
+
+
 def test_multi_group_tokens(sai):
     """More than 512 selected slots per token at H=64 (two TMEM groups, the
     two-pass statistics path). Sampled late tokens against the oracle."""
