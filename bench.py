@@ -95,16 +95,21 @@ def load_peaks():
 
 def traffic_record(kernel_src: str):
     """dram bytes per launch from a committed ncu summary, if it was taken on
-    the current source of the kernel (else null)."""
+    the current sources of the kernel (else null)."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
     with open(path) as f:
         rec = json.load(f)
-    src = os.path.join(ROOT, "sparse_attention_indexer_window_b200", "csrc", kernel_src)
-    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
     r = rec.get(kernel_src)
-    if not r or r.get("src_sha256_16") != h:
+    if not r:
+        return None
+    csrc = os.path.join(ROOT, "sparse_attention_indexer_window_b200", "csrc")
+    m = hashlib.sha256()
+    for name in r.get("sources", [kernel_src]):
+        with open(os.path.join(csrc, name), "rb") as f:
+            m.update(f.read())
+    if r.get("src_sha256_16") != m.hexdigest()[:16]:
         return None
     return r.get("dram_bytes_per_launch")
 
@@ -231,9 +236,11 @@ def main():
     dev = torch.device("cuda", local)
 
     import sparse_attention_indexer_window_b200 as sai
+    from sparse_attention_indexer_window_b200 import shard
     import synth
 
-    w = synth.make(WORKLOAD, seed=synth.CONFIGS[WORKLOAD].seed + rank)
+    # weak scaling: every rank runs its own full batch of the workload
+    w = synth.make(WORKLOAD, seed=shard.rank_seed(synth.CONFIGS[WORKLOAD].seed, rank))
     t = to_dev(w, dev)
     B, S, H, D, K = w.B, w.S, w.H, w.D, w.K
     wl = torch.empty((B, S, H), device=dev)
@@ -281,11 +288,7 @@ def main():
     k_win = [e[0].elapsed_time(e[1]) for e in ev]
     k_tgt = [e[1].elapsed_time(e[2]) for e in ev]
     k_kl = [e[2].elapsed_time(e[3]) for e in ev]
-    total_ms = float(sum(e[0].elapsed_time(e[3]) for e in ev))
-    if world > 1:
-        tt = torch.tensor([total_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        total_ms = float(tt.item())
+    total_ms = shard.max_over_ranks(float(sum(e[0].elapsed_time(e[3]) for e in ev)), device=dev)
     assert int(err.item()) == 0
     ms_step = total_ms / nsteps
     tokens_total = B * S * world * nsteps
@@ -293,7 +296,7 @@ def main():
 
     # ---------------------------------------------------------------- e2e
     host = {}
-    for k in ("Q", "Kw", "pool", "idx", "sink", "scores", "valid"):
+    for k in ("Q", "Kw", "pool", "idx", "sink", "doc_start", "scores", "valid"):
         if t[k] is not None:
             host[k] = t[k].cpu().pin_memory()
     out_loss = torch.empty(1).pin_memory()
@@ -305,9 +308,9 @@ def main():
     def e2e_step():
         for k, v in host.items():
             dq[k].copy_(v, non_blocking=True)
-        sai.window_lse(dq["Q"], dq["Kw"], w.W, w.scale, None, out=wl)
+        sai.window_lse(dq["Q"], dq["Kw"], w.W, w.scale, dq.get("doc_start"), out=wl)
         sai.distill_target(dq["Q"], dq["pool"], dq["idx"], wl, w.cr, w.scale, sink=dq.get("sink"),
-                           err=err, out=p)
+                           doc_start=dq.get("doc_start"), err=err, out=p)
         sai.distill_kl(p, dq["scores"], dq["valid"], w.coeff, workspace=ws, loss=loss, dscores=ds)
         out_loss.copy_(loss, non_blocking=True)
         out_ds.copy_(ds, non_blocking=True)
@@ -323,18 +326,12 @@ def main():
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize(dev)
-    e2e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        tt = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_ms = float(tt.item())
+    e2e_ms = shard.max_over_ranks(e0.elapsed_time(e1), device=dev)
     e2e_value = B * S * world * args.e2e_steps / (e2e_ms / 1e3)
 
-    # mean loss over ranks, for the record (not part of the timed path)
-    lv = torch.tensor([float(loss.item())], device=dev, dtype=torch.float64)
-    if world > 1:
-        dist.all_reduce(lv)
-        lv /= world
+    # batch-wide loss over all ranks, for the record (not part of the timed path)
+    n_rows = int(t["valid"].reshape(-1, K).any(dim=1).sum().item())
+    loss_all, _ = shard.global_mean_loss(float(loss.item()), n_rows, device=dev)
 
     if rank == 0:
         peak_tf, hbm_gbs, peak_src = load_peaks()
@@ -379,7 +376,8 @@ def main():
             "kernels_roofline": {
                 "window_lse": {"bound": "hbm", "achieved_gbs": win_bytes / (win_ms / 1e3) / 1e9,
                                "peak_gbs": hbm_gbs, "frac": win_bytes / (win_ms / 1e3) / 1e9 / hbm_gbs,
-                               "tflops": fl_win / (win_ms / 1e3) / 1e12},
+                               "tflops": fl_win / (win_ms / 1e3) / 1e12,
+                               "traffic": traffic_record("window_lse_tc.cu")},
                 "distill_kl": {"bound": "hbm", "achieved_gbs": kl_bytes / (kl_ms / 1e3) / 1e9,
                                "peak_gbs": hbm_gbs, "frac": kl_bytes / (kl_ms / 1e3) / 1e9 / hbm_gbs},
             },
@@ -387,7 +385,7 @@ def main():
                     "steps": args.e2e_steps},
             "gpu_launches": 4 * nsteps,
             "clocks": clk,
-            "loss": float(lv.item()),
+            "loss": loss_all,
         }
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)

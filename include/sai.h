@@ -57,9 +57,10 @@ int sai_version(void);
 /*
  * sai_window_lse -- sliding-window log-mass per (token, head).
  *
- * Source: Primus page, second commit message ("the cost is computing the mass,
- * a [S, window] score matrix per head ... indexer_distill_window_lse keeps the
- * scores in registers and loads only the key band a query block spans").
+ * Source: Primus page, second commit message (the joint target needs each
+ * head's log-mass over its window keys; indexer_distill_window_lse computes it
+ * without writing the window logits to memory, reading for each block of
+ * queries only the keys that block can see).
  *
  *   window_lse[b,t,h] = log sum_{s=lo}^{t} exp(scale * <Q[b,t,h,:], Kw[b,s,:]>)
  *   lo = max(d0, t - W + 1),  d0 = clamp(doc_start[b,t], 0, t) or 0 if NULL.
@@ -84,12 +85,12 @@ sai_status sai_window_lse(const uint16_t *Q, const uint16_t *Kw, const int32_t *
 /*
  * sai_distill_target -- the indexer's teacher target p[b,t,:].
  *
- * Source: Primus page, first commit message ("indexer_distill_target indexes
- * the pool inside the kernel, so the gather never exists and the softmax and
- * head sum happen in registers") and second commit message / "Why the target
- * was wrong" (one softmax over window keys, selected compressed entries and
- * the per-head sink; each head's share exp(compressed_lse - full_lse); floor
- * float32 tiny). Causal block rule: MaxText page "Add Indexer Loss
+ * Source: Primus page, first commit message (indexer_distill_target reads
+ * pool rows by index inside the kernel, so no gathered copy is written, and
+ * keeps the softmax and the sum over heads on chip) and second commit message
+ * / "Why the target was wrong" (each head normalises jointly over window keys,
+ * chosen pool rows and its sink; the pool rows' share of head h is
+ * exp(clse - lse_full); the L1 floor is the smallest normal float32). Causal block rule: MaxText page "Add Indexer Loss
  * [Deepseek v4]", commit messages (block j is visible to token t iff
  * (j+1)*cr - 1 <= t; cross-document blocks masked).
  *
@@ -127,10 +128,10 @@ size_t sai_distill_kl_workspace_bytes(int B, int S, int K);
 /*
  * sai_distill_kl -- KL(attention || indexer) and its gradient in one pass.
  *
- * Source: Primus page, first commit message ("indexer_distill_kl fuses the
- * KL tail with an analytic backward, so nothing beyond the inputs is saved
- * for it"); MaxText page review (log-softmax gives the exact gradient Q - P;
- * the valid mask includes the indexer mask).
+ * Source: Primus page, first commit message (indexer_distill_kl computes the
+ * KL and its closed-form gradient together and keeps no state between them);
+ * MaxText page review (the gradient of a log-softmax KL is q - p; the indexer's
+ * own mask is part of the valid mask).
  *
  * Per token row over its valid slots (valid[b,t,k] != 0):
  *   log q[k]  = scores[k] - log sum_{valid k'} exp scores[k']

@@ -22,7 +22,7 @@
  * Pins (tests under tests/): the window log-mass is pinned by closed forms
  * (one-key window, zero queries, document clipping) and by the full causal
  * log-sum-exp when the window covers the sequence; the target by the
- * joint softmax written out the long way, closed forms and invariants; the
+ * joint softmax spelled out term by term, closed forms and invariants; the
  * KL by its zero at matching targets, a hand-computed two-slot value and
  * central finite differences. The normalisation of the loss by the number
  * of valid tokens is a reading of the pages (they do not state it): parity
@@ -96,8 +96,8 @@ static int64_t doc_begin(const int32_t *doc_start, int64_t g, int64_t t)
 }
 
 /*
- * Sliding-window log-mass [P1, third commit message: "the cost is computing the
- * mass, a [S, window] score matrix per head"; indexer_distill_window_lse]:
+ * Sliding-window log-mass [P1, third commit message: the extra work of the
+ * joint target is this per-head window mass; indexer_distill_window_lse]:
  *
  *   window_lse[b,t,h] = log sum_{s = max(d0, t-W+1)}^{t} exp(scale * <Q[b,t,h,:], Kw[b,s,:]>)
  *
@@ -135,10 +135,10 @@ void orc_window_lse(const uint16_t *Q, const uint16_t *Kw, const int32_t *doc_st
 
 /*
  * Distillation target [P1, first and third commit messages, "Why the target
- * was wrong"]. One softmax runs over the concatenation of the window keys, the
- * selected compressed entries and the per-head sink; the target is that joint
- * softmax's mass on the selected compressed entries, summed over heads and
- * L1-renormalised with a float32-tiny floor.
+ * was wrong"]. Each head has a single softmax whose logits are the window
+ * keys, the chosen pool rows and a sink logit; the target keeps the part of
+ * that distribution that falls on the chosen pool rows, adds it up over heads
+ * and L1-normalises the result, flooring the sum at FLT_MIN.
  *
  *   slot k of token (b,t) is selected iff 0 <= idx < P, the block lies wholly
  *   at or before the token, (idx+1)*cr - 1 <= t  [P3: causal block mask, with
@@ -147,11 +147,11 @@ void orc_window_lse(const uint16_t *Q, const uint16_t *Kw, const int32_t *doc_st
  *   z[h,k]       = scale * <Q[b,t,h,:], pool[b, idx[k], :]>   (selected k)
  *   clse[h]      = log sum_k exp z[h,k]                       (-inf if none)
  *   lse_full[h]  = log( exp wl[h] + exp clse[h] + exp sink[h] )  (no sink term
- *                  when sink is NULL)  ["exp(compressed_lse - full_lse)"]
+ *                  when sink is NULL)  [head share exp(clse - lse_full)]
  *   u[k]         = sum_h exp(z[h,k] - lse_full[h])           [head sum]
  *   m            = sum_k u[k]
- *   p[k]         = u[k] / max(m, FLT_MIN)  (0 on masked slots) [floor moved
- *                  from 1e-10 to float32 tiny]
+ *   p[k]         = u[k] / max(m, FLT_MIN)  (0 on masked slots) [the floor is the
+ *                  smallest normal float32, no longer 1e-10]
  *
  * wl: [n, H] window log-mass rows aligned with the token list.
  * Returns the number of idx entries outside {-1} U [0, P) (data errors; those
@@ -229,9 +229,9 @@ int64_t orc_count_valid_rows(const uint8_t *valid, int64_t n_rows, int64_t K)
 
 /*
  * KL(attention || indexer) with its analytic gradient [P1, first commit
- * message: "indexer_distill_kl fuses the KL tail with an analytic backward";
- * P3 review: log-softmax gives the exact gradient Q - P, and the valid mask
- * must include the indexer mask so no row is all -inf].
+ * message: indexer_distill_kl computes the KL and its gradient in closed form
+ * in one pass; P3 review: the gradient of a log-softmax KL is q - p, and rows
+ * must be masked by the indexer's own mask so none is all -inf].
  *
  * Per row (token) over its valid slots:
  *   log q[k]  = s[k] - log sum_{valid k'} exp s[k']

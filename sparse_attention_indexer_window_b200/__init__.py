@@ -142,7 +142,7 @@ def distill_target(Q: torch.Tensor, pool: torch.Tensor, idx: torch.Tensor, wl: t
     if sink is not None:
         # The Primus page: a sink must hold one value per head (else ValueError).
         if sink.numel() != H:
-            raise ValueError(f"sink must hold {H} head values, got {sink.numel()}")
+            raise ValueError(f"sink needs one logit per head: expected {H} values, found {sink.numel()}")
         _want(sink, "sink", torch.float32)
     _want(doc_start, "doc_start", torch.int32, (B, S))
     _want(err, "err", torch.int32)

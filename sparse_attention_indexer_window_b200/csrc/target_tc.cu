@@ -4,8 +4,8 @@
 // For every token (b,t) (Primus page "perf(deepseek-v4): fuse and enable the
 // indexer distillation loss": first commit message -- the pool is indexed
 // inside the kernel so the [B,S,K,D] gather never exists; second commit
-// message / "Why the target was wrong" -- one softmax over window keys,
-// selected compressed entries and the per-head sink):
+// message / "Why the target was wrong" -- each head normalises jointly over
+// its window keys, its chosen pool rows and its sink logit):
 //
 //   z[k,h]      = scale <pool[idx[k]], Q[t,h]>       selected slots k
 //   clse[h]     = log sum_k exp z[k,h]
@@ -19,7 +19,7 @@
 //
 // Gather. A dedicated warp compacts each token's idx row (selected slots
 // first, masked slots last), up to two tokens ahead; the idx rows arrive by a
-// 1-D bulk copy. Eight gather warps then copy the selected rows into the
+// 1-D bulk copy. Ten gather warps then copy the selected rows into the
 // swizzled K-major operand layout with 16-byte cp.async (eight lanes per row,
 // four rows per instruction, every 128-byte row segment one coalesced
 // request); each thread's cp.async.mbarrier arrival publishes a stage. On
@@ -46,9 +46,9 @@
 //        = u'[k] exp(A - log FLT_MIN)   otherwise (the float32-tiny floor),
 // so no intermediate is subnormal however small each head's compressed share.
 //
-// Warp roles (576 threads): warp 0 idx staging and compaction, warps 1..8
-// row gathers (warp 1 also loads Q), warp 9 MMA issuer and TMEM owner, warps
-// 10..13 and 14..17 the two epilogue groups. Persistent CTAs walk tokens from the last
+// Warp roles (640 threads): warp 0 idx staging and compaction, warps 1..7 and
+// 9..11 row gathers (warp 1 also loads Q), warp 8 MMA issuer and TMEM owner,
+// warps 12..15 and 16..19 the two epilogue groups. Persistent CTAs walk tokens from the last
 // (heaviest) to the first. All mbarrier waits are bounded; a timeout is
 // reported through err and the CTA unwinds. Named barriers are only used
 // where every participating thread is guaranteed to arrive.

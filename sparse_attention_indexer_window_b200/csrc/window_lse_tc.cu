@@ -4,9 +4,9 @@
 // lo = max(d0, t-W+1): the log mass of the sliding-window keys that the joint
 // softmax of a CSA layer carries in its denominator (Primus page "perf(
 // deepseek-v4): fuse and enable the indexer distillation loss", second commit
-// message: the window mass is a [S, window] score matrix per head, and the
-// fused kernel keeps the scores on chip and loads only the key band a query
-// block spans).
+// message: computing the window mass eagerly materialises per-head window
+// logits that are mostly masked; the fused kernel never writes them and reads
+// only the keys each tile of queries can see).
 //
 // Tile: M = 128 rows = TQ = 128/H consecutive tokens x H heads, contiguous in
 // Q viewed as [B*S*H, D]. The key band of the tile is the NB = roundup16(W +

@@ -1,9 +1,9 @@
 """The distillation target written out the long way (numpy, fp64).
 
 The Primus page ("perf(deepseek-v4): fuse and enable the indexer distillation
-loss", second commit message and "Test plan") pins its fused target against a
-joint softmax written out the long way. This is that check, restated from the
-page's description: for every (token, head) build ONE logit vector that
+loss", second commit message and "Test plan") checks its fused target against
+the joint softmax computed term by term. This is that check in our own form:
+for every (token, head) build ONE logit vector that
 concatenates the window logits, the selected compressed logits and the sink,
 take a softmax over it, keep the compressed part, sum it over heads and
 L1-renormalise with the float32-tiny floor.

@@ -2,8 +2,8 @@
 
 Each test ties one part of the oracle to something fixed independently: a
 value a source page prints (fixtures under tests/golden/), a closed form, a
-special case that reduces to a library routine, the joint softmax written out
-the long way, or an invariant. They are chosen so that a plausible slip in the
+special case that reduces to a library routine, the joint softmax computed
+term by term, or an invariant. They are chosen so that a plausible slip in the
 oracle (an off-by-one window bound, a dropped sink or window term, a wrong
 causal rule, a transposed operand, a sign error in the gradient) fails one.
 """
