@@ -1,6 +1,7 @@
 // C-ABI entry points of libsai (declared in include/sai.h): argument
 // validation, kernel selection by shape, TMA descriptor encoding and launch.
 // Nothing here allocates device memory or synchronises the stream.
+#include <algorithm>
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
@@ -177,6 +178,7 @@ sai_status sai_distill_target(const uint16_t *Q, const uint16_t *pool, const int
         a.tiles_per_group = 256 / H;
         a.idx_bulk = ((K % 4) == 0 && al16(idx)) ? 1 : 0;
         a.n_astages = n_astages;
+        a.pool_box_rows = (int)std::min<int64_t>(128, (int64_t)B * P);
         a.scale = scale;
         a.pool = pool;
         a.idx = idx;
@@ -185,15 +187,16 @@ sai_status sai_distill_target(const uint16_t *Q, const uint16_t *pool, const int
         a.doc_start = doc_start;
         a.p = p;
         a.err = d_err;
-        CUtensorMap mq;
-        if (!make_map_bf16(&mq, Q, (uint64_t)B * S * H, D, (uint32_t)H))
+        CUtensorMap mq, mp;
+        if (!make_map_bf16(&mq, Q, (uint64_t)B * S * H, D, (uint32_t)H) ||
+            !make_map_bf16(&mp, pool, (uint64_t)B * P, D, (uint32_t)a.pool_box_rows))
             return SAI_ERR_CUDA;
         int grid = sm_count();
         if (grid <= 0)
             return SAI_ERR_CUDA;
         if (grid > a.n_tok)
             grid = a.n_tok;
-        return cuda_status(sai::launch_target_tc(mq, a, grid, st));
+        return cuda_status(sai::launch_target_tc(mq, mp, a, grid, st));
     }
     if ((int)sai::target_simt_smem_bytes(H, D, K) <= smem_cap)
         return cuda_status(sai::launch_target_simt(Q, pool, idx, window_lse, sink, doc_start, B, S, H, D, K, cr,

@@ -31,6 +31,7 @@ struct TgtTcArgs {
     int tiles_per_group;  // 128-slot tiles per TMEM accumulator (256 / H)
     int idx_bulk;         // idx rows are 16-byte aligned (K % 4 == 0): stage them by bulk copy
     int n_astages;        // depth of the gathered-row stage ring
+    int pool_box_rows;    // rows of the pool's TMA box (min(128, B*P))
     float scale;
     const uint16_t *pool;
     const int32_t *idx;
@@ -42,7 +43,8 @@ struct TgtTcArgs {
 };
 // Deepest gathered-row stage ring that fits `smem_limit` bytes (0: none).
 int target_tc_stages(int H, int K, int smem_limit);
-cudaError_t launch_target_tc(const CUtensorMap &mapQ, const TgtTcArgs &a, int grid, cudaStream_t stream);
+cudaError_t launch_target_tc(const CUtensorMap &mapQ, const CUtensorMap &mapP, const TgtTcArgs &a, int grid,
+                             cudaStream_t stream);
 
 // ------------------------------------------- generic CUDA-core kernels
 // For shapes the tensor-core kernels do not take (small H or D).

@@ -19,14 +19,19 @@
 //
 // Gather. A dedicated warp compacts each token's idx row (selected slots
 // first, masked slots last), up to two tokens ahead; the idx rows arrive by a
-// 1-D bulk copy. Ten gather warps then copy the selected rows into the
-// swizzled K-major operand layout with 16-byte cp.async (eight lanes per row,
-// four rows per instruction, every 128-byte row segment one coalesced
-// request); each thread's cp.async.mbarrier arrival publishes a stage. On
-// B200 a random-row gather from L2 saturates near 45 bytes/clock per SM this
-// way with eight or more warps (TMA tile::gather4 near 20), so the gather, not
-// the tensor core, bounds this kernel. Q[t] chunks (contiguous) arrive by TMA
-// tile loads. Masked slots are never loaded.
+// 1-D bulk copy, and the compaction turns pool rows into byte offsets. Nine
+// gather warps each own one 16 KB slot of the A ring and fill every stage
+// that lands in it: 128 selected rows x one 128-byte chunk of D, copied into
+// the swizzled K-major operand layout with 16-byte cp.async (eight lanes per
+// row, four rows per instruction, every 128-byte row segment one coalesced
+// request), then wait for their own copies and publish the stage with a
+// single mbarrier arrival. Per-stage synchronisation is thus one wait and one
+// arrival per stage, not per warp and stage; with many warps each sharing
+// every stage that bookkeeping, not the copies, set the pace. A separate warp
+// loads the Q[t] chunks (contiguous) by TMA several chunks ahead. A tile
+// whose selected rows are consecutive pool rows (every tile of an early token
+// under a sorted top-k, whose selection is all causal blocks) is one TMA box
+// instead. Masked slots are never loaded.
 //
 // The epilogue needs the per-head log-sum-exp over ALL selected slots before
 // it can form u, so a token's scores stay in TMEM until it is done: up to
@@ -46,8 +51,8 @@
 //        = u'[k] exp(A - log FLT_MIN)   otherwise (the float32-tiny floor),
 // so no intermediate is subnormal however small each head's compressed share.
 //
-// Warp roles (640 threads): warp 0 idx staging and compaction, warps 1..7 and
-// 9..11 row gathers (warp 1 also loads Q), warp 8 MMA issuer and TMEM owner,
+// Warp roles (640 threads): warp 0 idx staging and compaction, warps 1..7,
+// 9 and 10 row gathers, warp 11 Q loads, warp 8 MMA issuer and TMEM owner,
 // warps 12..15 and 16..19 the two epilogue groups. Persistent CTAs walk tokens from the last
 // (heaviest) to the first. All mbarrier waits are bounded; a timeout is
 // reported through err and the CTA unwinds. Named barriers are only used
@@ -58,11 +63,13 @@
 namespace sai {
 namespace {
 
-// Warpgroups 0..2 (warps 0..11): warp 0 compaction, warp 8 MMA, the other
-// ten warps row gathers; warpgroups 3 and 4 (warps 12..19): epilogue.
+// Warpgroups 0..2 (warps 0..11): warp 0 compaction, warp 8 MMA, warp 11 Q
+// loads, the other nine warps row gathers; warpgroups 3 and 4 (warps
+// 12..19): epilogue.
 constexpr int kMetaWarp = 0;
 constexpr int kMmaWarp = 8;
-constexpr int kGatherWarps = 10;
+constexpr int kQWarp = 11;
+constexpr int kGatherWarps = 9;
 constexpr int kEpiWarp0 = 12;
 constexpr int kTgtThreads = 20 * 32;                // 640
 // Register split (setmaxnreg): launched at kLaunchRegs a thread; warpgroups
@@ -72,8 +79,11 @@ constexpr int kLaunchRegs = 96;
 constexpr int kLowRegs = 56;
 constexpr int kHighRegs = 152;
 static_assert(384 * kLowRegs + 256 * kHighRegs <= kTgtThreads * kLaunchRegs, "register split");
-constexpr int kMaxAStages = 12;
-constexpr int kQStages = 3;
+constexpr int kMaxAStages = kGatherWarps;          // one A ring slot per gather warp
+constexpr int kQStagesMax = 6;
+// Q[t] chunk ring depth: the Q warp runs this many 64-column chunks ahead
+template <int HH>
+constexpr int q_stages() { return HH <= 64 ? 6 : 3; }
 constexpr int kMeta = 3;                            // compaction runs up to two tokens ahead
 constexpr uint32_t kATile = 128 * 128;              // 128 rows x 128 bytes
 constexpr float kLog2e = 1.4426950408889634f;
@@ -94,7 +104,7 @@ struct EpiState {                 // one per epilogue warpgroup
 template <int HH>
 struct TgtSmem {
     uint64_t a_full[kMaxAStages], a_empty[kMaxAStages];
-    uint64_t q_full[kQStages], q_empty[kQStages];
+    uint64_t q_full[kQStagesMax], q_empty[kQStagesMax];
     uint64_t acc_full[2], acc_empty[2];
     uint64_t meta_full[kMeta], meta_empty[kMeta];
     uint64_t idx_full[2];
@@ -123,7 +133,8 @@ __device__ __forceinline__ bool selected(int j, int t, int d0, int P, int cr)
 
 template <int HH>
 __global__ void __launch_bounds__(kTgtThreads, 1)
-    target_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const TgtTcArgs a)
+    target_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapP,
+                     const TgtTcArgs a)
 {
     constexpr int TB = 256 / HH;                 // tiles per accumulator
     constexpr int IB = TB < 2 ? TB : 2;          // tiles per TMEM load batch
@@ -136,9 +147,11 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
     const int Kp = (K + 3) & ~3;
     const int NA = a.n_astages;              // A-stage ring depth (sized on the host)
     uint8_t *a_buf = base;                                                   // NA x 16 KB
-    uint8_t *q_buf = a_buf + NA * kATile;                                    // kQStages x H*128
-    int32_t *rowid = reinterpret_cast<int32_t *>(q_buf + kQStages * kQTile); // [kMeta][Kp]
-    int32_t *slot = rowid + kMeta * Kp;                                      // [kMeta][Kp]
+    constexpr int QS = q_stages<HH>();
+    uint8_t *q_buf = a_buf + NA * kATile;                                    // QS x H*128
+    // byte offset in pool of every selected slot's row, compacted per token
+    uint32_t *rowoff = reinterpret_cast<uint32_t *>(q_buf + QS * kQTile);    // [kMeta][Kp]
+    int32_t *slot = reinterpret_cast<int32_t *>(rowoff + kMeta * Kp);        // [kMeta][Kp]
     int32_t *idxs = slot + kMeta * Kp;                                       // [2][Kp] staged idx rows
     float *ubuf = reinterpret_cast<float *>(idxs + 2 * Kp);                  // [2][Kp]
     TgtSmem<HH> *sm = reinterpret_cast<TgtSmem<HH> *>(ubuf + 2 * Kp);
@@ -150,10 +163,10 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < NA; ++s) {
-            mbar_init(&sm->a_full[s], kGatherWarps * 32);  // one arrival per gather thread
+            mbar_init(&sm->a_full[s], 1);        // the owning gather warp's lane 0
             mbar_init(&sm->a_empty[s], 1);
         }
-        for (int s = 0; s < kQStages; ++s) {
+        for (int s = 0; s < QS; ++s) {
             mbar_init(&sm->q_full[s], 1);
             mbar_init(&sm->q_empty[s], 1);
         }
@@ -230,7 +243,7 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
             }
             // selected slots in order at the front, masked slots from the back;
             // lane L takes 4 consecutive slots
-            int32_t *rw = rowid + m3 * Kp;
+            uint32_t *rw = rowoff + m3 * Kp;
             int32_t *sl = slot + m3 * Kp;
             const int32_t *grow = a.idx + (size_t)g * K;
             int nsel = 0, nmask = 0;
@@ -274,7 +287,7 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     if (sel[e]) {
-                        rw[ps] = b * a.P + j[e];
+                        rw[ps] = (uint32_t)(b * a.P + j[e]) * (uint32_t)(a.D * 2);
                         sl[ps] = k + e;
                         ++ps;
                     } else if (k + e < K) {
@@ -299,20 +312,17 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
                     mbar_drain(&sm->idx_full[s], (i_last >> s) & 1u);
         }
         __syncwarp();
-    } else if (warp != kMmaWarp && warp < kEpiWarp0) {
-        // ============================================================ gathers
-        const int gw = warp < kMmaWarp ? warp - 1 : warp - 2;   // 0..9
-        const bool q_loader = (gw == 0);         // also loads the Q[t] chunks by TMA
-        if (q_loader && lane == 0)
-            tma_prefetch_desc(&mapQ);
-        int as = 0, qs = 0;
-        uint32_t aph = 0, qph = 0;
+    } else if (warp == kQWarp) {
+        // ============================================================ Q[t] chunks
+        // Every (pass, group, chunk) of a token uses the chunk's H x 64 slice
+        // of Q[t]; this warp loads them by TMA, QS chunks ahead of the MMA.
+        int qs = 0;
+        uint32_t qph = 0;
         uint32_t q_issued = 0, q_last = 0;
         bool ok = true;
         int it = 0;
-        const char *pool_bytes = reinterpret_cast<const char *>(a.pool);
-        const int seg = lane & 7;                // 16-byte segment of a 128-byte row chunk
-        const int r_in = lane >> 3;              // row within a 4-row group
+        if (lane == 0)
+            tma_prefetch_desc(&mapQ);
         for (int gt = blockIdx.x; gt < a.n_tok && ok; gt += gridDim.x, ++it) {
             const int g = a.n_tok - 1 - gt;
             const int m3 = it % kMeta;
@@ -322,143 +332,168 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
             if (!ok)
                 break;
             const int nsel = sm->nsel[m3];
-            const int32_t *rw = rowid + m3 * Kp;
-            const int nt = (nsel + 127) / 128;
             const int G = n_groups(nsel, TB);
-            const int passes = G > 1 ? 2 : 1;
-            for (int pass = 0; pass < passes && ok; ++pass) {
-                for (int grp = 0; grp < G && ok; ++grp) {
-                    const int i0 = grp * TB;
-                    const int ntg = min(nt, i0 + TB) - i0;
-                    // byte offsets of this lane's rows in every tile of the group,
-                    // held in registers when the group has at most four tiles
-                    // (all-ones marks a row past the selected slots)
-                    constexpr int NGI = (32 + kGatherWarps - 1) / kGatherWarps;
-                    constexpr int RT = TB < 4 ? TB : 4;
-                    uint32_t roff[RT][NGI];
-#pragma unroll
-                    for (int i = 0; i < RT; ++i)
-#pragma unroll
-                        for (int u = 0; u < NGI; ++u) {
-                            const int gi = gw + u * kGatherWarps;
-                            const int r = 4 * gi + r_in;
-                            const int k = (i0 + i) * 128 + r;
-                            roff[i][u] = (gi < 32 && i < ntg && k < nsel) ? (uint32_t)rw[k] * (uint32_t)(a.D * 2)
-                                                                          : 0xffffffffu;
-                        }
-                    for (int c = 0; c < n_chunks && ok; ++c) {
-                        if (q_loader) {
-                            if (lane == 0) {
-                                ok = mbar_wait(&sm->q_empty[qs], qph ^ 1u, abort_flag, a.err);
-                                if (ok) {
-                                    mbar_arrive_expect_tx(&sm->q_full[qs], kQTile);
-                                    tma_load_2d(q_buf + qs * kQTile, &mapQ, &sm->q_full[qs], c * 64, g * HH);
-                                    q_issued |= 1u << qs;
-                                    q_last = (q_last & ~(1u << qs)) | (qph << qs);
+            const int nq = (G > 1 ? 2 : 1) * G * n_chunks;
+            for (int qi = 0; qi < nq && ok; ++qi) {
+                const int c = qi % n_chunks;
+                if (lane == 0) {
+                    ok = mbar_wait(&sm->q_empty[qs], qph ^ 1u, abort_flag, a.err);
+                    if (ok) {
+                        mbar_arrive_expect_tx(&sm->q_full[qs], kQTile);
+                        tma_load_2d(q_buf + qs * kQTile, &mapQ, &sm->q_full[qs], c * 64, g * HH);
+                        q_issued |= 1u << qs;
+                        q_last = (q_last & ~(1u << qs)) | (qph << qs);
+                    }
+                }
+                ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+                if (++qs == QS) {
+                    qs = 0;
+                    qph ^= 1u;
+                }
+            }
+        }
+        if (!ok && lane == 0) {
+            for (int s = 0; s < QS; ++s)
+                if (q_issued & (1u << s))
+                    mbar_drain(&sm->q_full[s], (q_last >> s) & 1u);
+        }
+        __syncwarp();
+    } else if (warp != kMmaWarp && warp < kEpiWarp0) {
+        // ============================================================ gathers
+        // Gather warp gw owns A ring slot gw: it fills every stage that lands
+        // there (stages gw, gw + NA, gw + 2 NA, ... of the MMA's sequence),
+        // waits for its own copies and publishes the stage with one arrival.
+        // Each slot has a single producer, so its phases are seen in order.
+        const int gw = warp < kMmaWarp ? warp - 1 : warp - 2;   // 0..8
+        if (gw < NA) {
+            const char *pool_bytes = reinterpret_cast<const char *>(a.pool);
+            const int seg = lane & 7;            // 16-byte segment of a 128-byte row chunk
+            const int r_in = lane >> 3;          // row within a 4-row group
+            const uint32_t dst0 = smem_u32(a_buf + gw * kATile);
+            const uint32_t row_bytes = (uint32_t)a.D * 2u;
+            if (lane == 0)
+                tma_prefetch_desc(&mapP);
+            uint32_t ph = 0;
+            int s = 0;                           // stage index modulo NA
+            bool ok = true;
+            int it = 0;
+            for (int gt = blockIdx.x; gt < a.n_tok && ok; gt += gridDim.x, ++it) {
+                const int m3 = it % kMeta;
+                if (lane == 0)
+                    ok = mbar_wait(&sm->meta_full[m3], (it / kMeta) & 1, abort_flag, a.err);
+                ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+                if (!ok)
+                    break;
+                const int nsel = sm->nsel[m3];
+                const uint32_t *rw = rowoff + m3 * Kp;
+                const int nt = (nsel + 127) / 128;
+                const int G = n_groups(nsel, TB);
+                const int passes = G > 1 ? 2 : 1;
+                for (int pass = 0; pass < passes && ok; ++pass) {
+                    for (int grp = 0; grp < G && ok; ++grp) {
+                        const int i0 = grp * TB;
+                        const int ntg = min(nt, i0 + TB) - i0;
+                        for (int c = 0; c < n_chunks && ok; ++c) {
+                            for (int i = 0; i < ntg; ++i) {
+                                const bool mine = (s == gw);
+                                if (++s == NA)
+                                    s = 0;
+                                if (!mine)
+                                    continue;
+                                if (lane == 0)
+                                    ok = mbar_wait(&sm->a_empty[gw], ph ^ 1u, abort_flag, a.err);
+                                ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+                                if (!ok)
+                                    break;
+                                const int tile_row0 = (i0 + i) * 128;
+                                const int rows = min(128, nsel - tile_row0);
+                                const uint32_t *ro = rw + tile_row0;
+                                // a tile whose rows are consecutive pool rows is one TMA box
+                                const uint32_t ro0 = ro[0];
+                                bool run = true;
+                                for (int q = lane; q < rows; q += 32)
+                                    run = run && ro[q] == ro0 + (uint32_t)q * row_bytes;
+                                if (__all_sync(0xffffffffu, run)) {
+                                    if (lane == 0) {
+                                        mbar_arrive_expect_tx(&sm->a_full[gw], (uint32_t)a.pool_box_rows * 128u);
+                                        tma_load_2d(a_buf + gw * kATile, &mapP, &sm->a_full[gw], c * 64,
+                                                    (int32_t)(ro0 / row_bytes));
+                                    }
+                                    __syncwarp();
+                                } else {
+                                    const char *src0 = pool_bytes + c * 128 + seg * 16;
+#pragma unroll 8
+                                    for (int j = 0; j < 32; ++j) {
+                                        const int r = 4 * j + r_in;
+                                        if (r < rows)
+                                            cp_async16(dst0 + r * 128 + ((seg ^ (r & 7)) << 4), src0 + ro[r]);
+                                    }
+                                    cp_async_commit();
+                                    cp_async_wait<0>();
+                                    fence_proxy_async_smem();
+                                    __syncwarp();
+                                    if (lane == 0)
+                                        mbar_arrive(&sm->a_full[gw]);
                                 }
-                            }
-                            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-                            if (!ok)
-                                break;
-                            if (++qs == kQStages) {
-                                qs = 0;
-                                qph ^= 1u;
-                            }
-                        }
-                        for (int i = 0; i < ntg; ++i) {
-                            if (lane == 0)
-                                ok = mbar_wait(&sm->a_empty[as], aph ^ 1u, abort_flag, a.err);
-                            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-                            if (!ok)
-                                break;
-                            const int tile_row0 = (i0 + i) * 128;
-                            const int rows = min(128, nsel - tile_row0);
-                            const uint32_t dst0 = smem_u32(a_buf + as * kATile);
-#pragma unroll
-                            for (int u = 0; u < NGI; ++u) {
-                                const int gi = gw + u * kGatherWarps;
-                                const int r = 4 * gi + r_in;
-                                uint32_t off = 0xffffffffu;
-                                if (TB <= 4) {
-#pragma unroll
-                                    for (int ii = 0; ii < RT; ++ii)
-                                        if (ii == i)
-                                            off = roff[ii][u];
-                                } else if (gi < 32 && r < rows) {
-                                    off = (uint32_t)rw[tile_row0 + r] * (uint32_t)(a.D * 2);
-                                }
-                                if (gi < 32 && r < rows && off != 0xffffffffu) {
-                                    const char *src = pool_bytes + off + c * 128 + seg * 16;
-                                    const uint32_t dst = dst0 + r * 128 + ((seg ^ (r & 7)) << 4);
-                                    cp_async16(dst, src);
-                                }
-                            }
-                            // arrives once this thread's copies so far have landed
-                            cp_async_mbar_arrive_noinc(&sm->a_full[as]);
-                            if (++as == NA) {
-                                as = 0;
-                                aph ^= 1u;
+                                ph ^= 1u;
                             }
                         }
                     }
                 }
             }
         }
-        cp_async_wait<0>();
-        if (!ok && q_loader && lane == 0) {
-            for (int s = 0; s < kQStages; ++s)
-                if (q_issued & (1u << s))
-                    mbar_drain(&sm->q_full[s], (q_last >> s) & 1u);
-        }
         __syncwarp();
     } else if (warp == kMmaWarp) {
         // ============================================================ MMA
-        const uint32_t idesc = idesc_bf16_f32(128, HH);
-        int as = 0, qs = 0;
-        uint32_t aph = 0, qph = 0;
-        bool ok = true, issued = false;
-        int it = 0;
-        int jobs0 = 0, jobs1 = 0;
-        for (int gt = blockIdx.x; gt < a.n_tok && ok; gt += gridDim.x, ++it) {
-            const int mb = it & 1;
-            const int m3 = it % kMeta;
-            if (!mbar_wait(&sm->meta_full[m3], (it / kMeta) & 1, abort_flag, a.err)) {
-                ok = false;
-                break;
-            }
-            const int nsel = sm->nsel[m3];
-            const int nt = (nsel + 127) / 128;
-            const int G = n_groups(nsel, TB);
-            const int passes = G > 1 ? 2 : 1;
-            const uint32_t dbase = tmem + mb * 256;
-            for (int pass = 0; pass < passes && ok; ++pass) {
-                for (int grp = 0; grp < G && ok; ++grp) {
-                    const int i0 = grp * TB;
-                    const int ntg = min(nt, i0 + TB) - i0;
-                    const int jb = mb ? jobs1 : jobs0;
-                    if (!mbar_wait(&sm->acc_empty[mb], (jb & 1) ^ 1u, abort_flag, a.err)) {
-                        ok = false;
-                        break;
-                    }
-                    if (mb)
-                        ++jobs1;
-                    else
-                        ++jobs0;
-                    tc_fence_after();
-                    for (int c = 0; c < n_chunks && ok; ++c) {
-                        if (!mbar_wait(&sm->q_full[qs], qph, abort_flag, a.err)) {
+        // One thread issues everything, stage by stage. (Issuing a chunk's
+        // MMAs back to back measured slower: at N = H the MMAs are bound by
+        // shared-memory operand reads, and bursts of them starve the gathers'
+        // shared-memory writes.)
+        if (lane == 0) {
+            const uint32_t idesc = idesc_bf16_f32(128, HH);
+            int as = 0, qs = 0;
+            uint32_t aph = 0, qph = 0;
+            bool ok = true, issued = false;
+            int it = 0;
+            int jobs0 = 0, jobs1 = 0;
+            for (int gt = blockIdx.x; gt < a.n_tok && ok; gt += gridDim.x, ++it) {
+                const int mb = it & 1;
+                const int m3 = it % kMeta;
+                if (!mbar_wait(&sm->meta_full[m3], (it / kMeta) & 1, abort_flag, a.err)) {
+                    ok = false;
+                    break;
+                }
+                const int nsel = sm->nsel[m3];
+                const int nt = (nsel + 127) / 128;
+                const int G = n_groups(nsel, TB);
+                const int passes = G > 1 ? 2 : 1;
+                const uint32_t dbase = tmem + mb * 256;
+                for (int pass = 0; pass < passes && ok; ++pass) {
+                    for (int grp = 0; grp < G && ok; ++grp) {
+                        const int i0 = grp * TB;
+                        const int ntg = min(nt, i0 + TB) - i0;
+                        const int jb = mb ? jobs1 : jobs0;
+                        if (!mbar_wait(&sm->acc_empty[mb], (jb & 1) ^ 1u, abort_flag, a.err)) {
                             ok = false;
                             break;
                         }
-                        tc_fence_after();
-                        const uint64_t dq = sdesc_k_sw128(smem_u32(q_buf + qs * kQTile));
-                        for (int i = 0; i < ntg; ++i) {
-                            if (!mbar_wait(&sm->a_full[as], aph, abort_flag, a.err)) {
+                        if (mb)
+                            ++jobs1;
+                        else
+                            ++jobs0;
+                        for (int c = 0; c < n_chunks && ok; ++c) {
+                            if (!mbar_wait(&sm->q_full[qs], qph, abort_flag, a.err)) {
                                 ok = false;
                                 break;
                             }
-                            tc_fence_after();
-                            if (lane == 0) {
+                            // are all of this chunk's stages published already?
+                            const uint64_t dq = sdesc_k_sw128(smem_u32(q_buf + qs * kQTile));
+                            for (int i = 0; i < ntg; ++i) {
+                                if (!mbar_wait(&sm->a_full[as], aph, abort_flag, a.err)) {
+                                    ok = false;
+                                    break;
+                                }
+                                tc_fence_after();
                                 const uint64_t da = sdesc_k_sw128(smem_u32(a_buf + as * kATile));
                                 const uint32_t d_tmem = dbase + i * HH;
 #pragma unroll
@@ -466,34 +501,29 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
                                     umma_bf16(d_tmem, da + 2 * kk, dq + 2 * kk, idesc, (c | kk) != 0);
                                 umma_commit(&sm->a_empty[as]);
                                 issued = true;
+                                if (++as == NA) {
+                                    as = 0;
+                                    aph ^= 1u;
+                                }
                             }
-                            __syncwarp();
-                            if (++as == NA) {
-                                as = 0;
-                                aph ^= 1u;
+                            if (!ok)
+                                break;
+                            umma_commit(&sm->q_empty[qs]);
+                            if (++qs == QS) {
+                                qs = 0;
+                                qph ^= 1u;
                             }
                         }
                         if (!ok)
                             break;
-                        if (lane == 0)
-                            umma_commit(&sm->q_empty[qs]);
-                        __syncwarp();
-                        if (++qs == kQStages) {
-                            qs = 0;
-                            qph ^= 1u;
-                        }
-                    }
-                    if (!ok)
-                        break;
-                    if (lane == 0)
                         umma_commit(&sm->acc_full[mb]);
-                    __syncwarp();
+                    }
                 }
             }
-        }
-        if (!ok && lane == 0 && issued) {
-            umma_commit(&sm->drain);
-            mbar_drain(&sm->drain, 0);
+            if (!ok && issued) {
+                umma_commit(&sm->drain);
+                mbar_drain(&sm->drain, 0);
+            }
         }
         __syncwarp();
     }
@@ -761,7 +791,7 @@ template <int HH>
 __host__ __device__ inline size_t fixed_smem_bytes(int K)
 {
     const size_t Kp = (size_t)((K + 3) & ~3);
-    return 1024 + kQStages * (HH * 128) + Kp * 4 * (2 * kMeta + 4) + sizeof(TgtSmem<HH>) + 64;
+    return 1024 + q_stages<HH>() * (HH * 128) + Kp * 4 * (2 * kMeta + 4) + sizeof(TgtSmem<HH>) + 64;
 }
 
 // Deepest A-stage ring that fits the per-block smem limit (0 if none does).
@@ -782,7 +812,8 @@ size_t smem_bytes_for(int K, int stages)
 }
 
 template <int HH>
-cudaError_t launch_h(const CUtensorMap &mapQ, const TgtTcArgs &a, int grid, cudaStream_t stream)
+cudaError_t launch_h(const CUtensorMap &mapQ, const CUtensorMap &mapP, const TgtTcArgs &a, int grid,
+                     cudaStream_t stream)
 {
     // The register split above is only safe if every thread was launched with
     // exactly kLaunchRegs registers; refuse to launch otherwise.
@@ -796,7 +827,7 @@ cudaError_t launch_h(const CUtensorMap &mapQ, const TgtTcArgs &a, int grid, cuda
     e = cudaFuncSetAttribute(target_tc_kernel<HH>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess)
         return e;
-    target_tc_kernel<HH><<<grid, kTgtThreads, smem, stream>>>(mapQ, a);
+    target_tc_kernel<HH><<<grid, kTgtThreads, smem, stream>>>(mapQ, mapP, a);
     return cudaGetLastError();
 }
 
@@ -813,13 +844,14 @@ int target_tc_stages(int H, int K, int smem_limit)
     }
 }
 
-cudaError_t launch_target_tc(const CUtensorMap &mapQ, const TgtTcArgs &a, int grid, cudaStream_t stream)
+cudaError_t launch_target_tc(const CUtensorMap &mapQ, const CUtensorMap &mapP, const TgtTcArgs &a, int grid,
+                             cudaStream_t stream)
 {
     switch (a.H) {
-    case 16: return launch_h<16>(mapQ, a, grid, stream);
-    case 32: return launch_h<32>(mapQ, a, grid, stream);
-    case 64: return launch_h<64>(mapQ, a, grid, stream);
-    case 128: return launch_h<128>(mapQ, a, grid, stream);
+    case 16: return launch_h<16>(mapQ, mapP, a, grid, stream);
+    case 32: return launch_h<32>(mapQ, mapP, a, grid, stream);
+    case 64: return launch_h<64>(mapQ, mapP, a, grid, stream);
+    case 128: return launch_h<128>(mapQ, mapP, a, grid, stream);
     default: return cudaErrorInvalidValue;
     }
 }
