@@ -18,8 +18,9 @@
 // 64-element (128-byte, swizzled) chunks.
 //
 // Gather. A dedicated warp compacts each token's idx row (selected slots
-// first, masked slots last), up to two tokens ahead; the idx rows arrive by a
-// 1-D bulk copy, and the compaction turns pool rows into byte offsets. Nine
+// first, masked slots last), up to two tokens ahead; the idx rows arrive by
+// its own cp.async copies, and the compaction turns pool rows into byte
+// offsets. Nine
 // gather warps each own one 16 KB slot of the A ring and fill every stage
 // that lands in it: 128 selected rows x one 128-byte chunk of D, copied into
 // the swizzled K-major operand layout with 16-byte cp.async (eight lanes per
@@ -107,7 +108,6 @@ struct TgtSmem {
     uint64_t q_full[kQStagesMax], q_empty[kQStagesMax];
     uint64_t acc_full[2], acc_empty[2];
     uint64_t meta_full[kMeta], meta_empty[kMeta];
-    uint64_t idx_full[2];
     uint64_t drain;
     uint32_t tmem_base;
     int abort_flag;
@@ -152,8 +152,8 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
     // byte offset in pool of every selected slot's row, compacted per token
     uint32_t *rowoff = reinterpret_cast<uint32_t *>(q_buf + QS * kQTile);    // [kMeta][Kp]
     int32_t *slot = reinterpret_cast<int32_t *>(rowoff + kMeta * Kp);        // [kMeta][Kp]
-    int32_t *idxs = slot + kMeta * Kp;                                       // [2][Kp] staged idx rows
-    float *ubuf = reinterpret_cast<float *>(idxs + 2 * Kp);                  // [2][Kp]
+    int32_t *idxs = slot + kMeta * Kp;                                       // [3][Kp] staged idx rows
+    float *ubuf = reinterpret_cast<float *>(idxs + 3 * Kp);                  // [2][Kp]
     TgtSmem<HH> *sm = reinterpret_cast<TgtSmem<HH> *>(ubuf + 2 * Kp);
 
     const int warp = threadIdx.x >> 5;
@@ -173,7 +173,6 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
         for (int b = 0; b < 2; ++b) {
             mbar_init(&sm->acc_full[b], 1);
             mbar_init(&sm->acc_empty[b], 4);
-            mbar_init(&sm->idx_full[b], 1);
         }
         for (int b = 0; b < kMeta; ++b) {
             mbar_init(&sm->meta_full[b], 1);
@@ -198,39 +197,34 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
     regs_dec<kLowRegs>();
     if (warp == kMetaWarp) {
         // ====================================================== idx compaction
-        if (lane == 0 && idx_bulk && (int)blockIdx.x < a.n_tok) {
-            const int g0 = a.n_tok - 1 - blockIdx.x;
-            mbar_arrive_expect_tx(&sm->idx_full[0], (uint32_t)K * 4u);
-            bulk_load(idxs, a.idx + (size_t)g0 * K, (uint32_t)K * 4u, &sm->idx_full[0]);
-        }
-        uint32_t i_issued = 0, i_last = 0;
+        // idx rows are staged into shared memory with this warp's own
+        // 16-byte cp.async copies, two tokens ahead (three buffers). (A TMA
+        // bulk copy here queued behind the Q and pool TMA traffic of the same
+        // SM and arrived late.)
+        const int n_vec = K / 4;                 // 16-byte pieces of an idx row (idx_bulk: K % 4 == 0)
+        auto stage_idx = [&](int gts, int buf) {
+            if (idx_bulk && gts < a.n_tok) {
+                const int gs = a.n_tok - 1 - gts;
+                const char *src = reinterpret_cast<const char *>(a.idx + (size_t)gs * K);
+                const uint32_t dst = smem_u32(idxs + buf * Kp);
+                for (int v = lane; v < n_vec; v += 32)
+                    cp_async16(dst + v * 16, src + v * 16);
+            }
+            cp_async_commit();
+        };
+        stage_idx(blockIdx.x, 0);
+        stage_idx(blockIdx.x + gridDim.x, 1);
         bool ok = true;
         int it = 0;
         for (int gt = blockIdx.x; gt < a.n_tok && ok; gt += gridDim.x, ++it) {
             const int g = a.n_tok - 1 - gt;
             const int b = g / a.S;
             const int t = g - b * a.S;
-            const int ib2 = it & 1;
             const int m3 = it % kMeta;
-            int32_t *ib = idxs + ib2 * Kp;
-            if (idx_bulk) {
-                // this token's idx row has landed; start the next token's copy
-                if (lane == 0) {
-                    ok = mbar_wait(&sm->idx_full[ib2], (it >> 1) & 1, abort_flag, a.err);
-                    const int gtn = gt + gridDim.x;
-                    if (ok && gtn < a.n_tok) {
-                        const int gn = a.n_tok - 1 - gtn;
-                        const int nb = ib2 ^ 1;
-                        mbar_arrive_expect_tx(&sm->idx_full[nb], (uint32_t)K * 4u);
-                        bulk_load(idxs + nb * Kp, a.idx + (size_t)gn * K, (uint32_t)K * 4u, &sm->idx_full[nb]);
-                        i_issued |= 1u << nb;
-                        i_last = (i_last & ~(1u << nb)) | ((((it + 1) >> 1) & 1u) << nb);
-                    }
-                }
-                ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-                if (!ok)
-                    break;
-            }
+            int32_t *ib = idxs + (it % 3) * Kp;
+            stage_idx(gt + 2 * (int)gridDim.x, (it + 2) % 3);
+            cp_async_wait<2>();                  // this token's row has landed
+            __syncwarp();
             if (lane == 0)
                 ok = mbar_wait(&sm->meta_empty[m3], ((it / kMeta) & 1) ^ 1u, abort_flag, a.err);
             ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
@@ -306,11 +300,7 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
             if (lane == 0)
                 mbar_arrive(&sm->meta_full[m3]);
         }
-        if (!ok && lane == 0) {
-            for (int s = 0; s < 2; ++s)
-                if (i_issued & (1u << s))
-                    mbar_drain(&sm->idx_full[s], (i_last >> s) & 1u);
-        }
+        cp_async_wait<0>();
         __syncwarp();
     } else if (warp == kQWarp) {
         // ============================================================ Q[t] chunks
@@ -791,7 +781,7 @@ template <int HH>
 __host__ __device__ inline size_t fixed_smem_bytes(int K)
 {
     const size_t Kp = (size_t)((K + 3) & ~3);
-    return 1024 + q_stages<HH>() * (HH * 128) + Kp * 4 * (2 * kMeta + 4) + sizeof(TgtSmem<HH>) + 64;
+    return 1024 + q_stages<HH>() * (HH * 128) + Kp * 4 * (2 * kMeta + 5) + sizeof(TgtSmem<HH>) + 64;
 }
 
 // Deepest A-stage ring that fits the per-block smem limit (0 if none does).
