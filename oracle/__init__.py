@@ -40,7 +40,7 @@ def _load():
         Dd = ctypes.c_double
         lib.orc_window_lse.argtypes = [P, P, P, I, I, I, I, I, Dd, P, I, P]
         lib.orc_window_lse.restype = None
-        lib.orc_distill_target.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, Dd, P, I, P]
+        lib.orc_distill_target.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, Dd, P, I, ctypes.c_int, P]
         lib.orc_distill_target.restype = I
         lib.orc_count_valid_rows.argtypes = [P, I, I]
         lib.orc_count_valid_rows.restype = I
@@ -83,17 +83,27 @@ def window_lse(Q, Kw, doc_start, W: int, scale: float, tokens=None) -> np.ndarra
     return out
 
 
-def distill_target(Q, pool, idx, wl, sink, doc_start, cr: int, scale: float, tokens=None):
-    """(p [n, K] fp64, bad_index_count) for the flat token ids in ``tokens``."""
+def distill_target(Q, pool, idx, wl, sink, doc_start, cr: int, scale: float, tokens=None,
+                   per_branch: bool = False):
+    """(p [n, K] fp64, bad_index_count) for the flat token ids in ``tokens``.
+
+    per_branch selects the earlier per-branch target (every head normalised
+    over the selected entries alone, floor 1e-10); wl and sink are then
+    unused and may be None."""
     B, S, H, D = Q.shape
     K = idx.shape[-1]
     Q = _c(Q, np.uint16); pool = _c(pool, np.uint16); idx = _c(idx, np.int32)
     wl = _c(wl, np.float64); sink = _c(sink, np.float32); ds = _c(doc_start, np.int32)
     tk, n = _tokens(tokens, B, S)
-    assert wl.shape == (n, H)
+    if per_branch:
+        wl = None
+        sink = None
+    else:
+        assert wl.shape == (n, H)
     p = np.empty((n, K), dtype=np.float64)
     bad = _load().orc_distill_target(_ptr(Q), _ptr(pool), _ptr(idx), _ptr(wl), _ptr(sink), _ptr(ds),
-                                     B, S, H, D, K, cr, float(scale), _ptr(tk), n, _ptr(p))
+                                     B, S, H, D, K, cr, float(scale), _ptr(tk), n, 1 if per_branch else 0,
+                                     _ptr(p))
     return p, int(bad)
 
 

@@ -47,6 +47,7 @@ int orc_num_threads(void)
 }
 
 #define ORC_FLT_MIN 1.1754943508222875e-38 /* float32 tiny, 2^-126 */
+#define ORC_OLD_FLOOR 1e-10                 /* the per-branch target's floor */
 
 static double bf16_val(uint16_t bits)
 {
@@ -153,6 +154,13 @@ void orc_window_lse(const uint16_t *Q, const uint16_t *Kw, const int32_t *doc_st
  *   p[k]         = u[k] / max(m, FLT_MIN)  (0 on masked slots) [the floor is the
  *                  smallest normal float32, no longer 1e-10]
  *
+ * per_branch != 0 selects the earlier per-branch target that the Primus page
+ * keeps behind an A/B switch and the MaxText page prints [P1, second commit
+ * message: PRIMUS_V4_DISTILL_NONCOMP_LSE=0 restores it; P3 commit messages]:
+ * every head is normalised over the selected compressed entries alone,
+ *   lse_full[h] = clse[h]   (window and sink ignored; wl and sink may be NULL)
+ * and the floor is the old 1e-10: p[k] = u[k] / max(m, 1e-10).
+ *
  * wl: [n, H] window log-mass rows aligned with the token list.
  * Returns the number of idx entries outside {-1} U [0, P) (data errors; those
  * slots are masked).
@@ -160,7 +168,7 @@ void orc_window_lse(const uint16_t *Q, const uint16_t *Kw, const int32_t *doc_st
 int64_t orc_distill_target(const uint16_t *Q, const uint16_t *pool, const int32_t *idx,
                            const double *wl, const float *sink, const int32_t *doc_start,
                            int64_t B, int64_t S, int64_t H, int64_t D, int64_t K, int64_t cr,
-                           double scale, const int64_t *tokens, int64_t n_tokens, double *p)
+                           double scale, const int64_t *tokens, int64_t n_tokens, int per_branch, double *p)
 {
     int64_t n = tokens ? n_tokens : B * S;
     int64_t P = S / cr;
@@ -185,6 +193,10 @@ int64_t orc_distill_target(const uint16_t *Q, const uint16_t *pool, const int32_
             for (int64_t k = 0; k < K; ++k)
                 z[h * K + k] = sel[k] ? scale * dot_bf16(q, pool + (b * P + row[k]) * D, D) : -INFINITY;
             double clse = lse_list(z + h * K, K);
+            if (per_branch) {
+                lse_full[h] = clse;
+                continue;
+            }
             double parts[3];
             int np = 0;
             parts[np++] = wl[i * H + h];
@@ -203,7 +215,8 @@ int64_t orc_distill_target(const uint16_t *Q, const uint16_t *pool, const int32_
             u[k] = acc;
             m += acc;
         }
-        double den = m > ORC_FLT_MIN ? m : ORC_FLT_MIN;
+        const double floor_ = per_branch ? ORC_OLD_FLOOR : ORC_FLT_MIN;
+        double den = m > floor_ ? m : floor_;
         for (int64_t k = 0; k < K; ++k)
             u[k] = sel[k] ? u[k] / den : 0.0;
         free(sel);

@@ -221,6 +221,50 @@ def test_target_per_branch_limit_is_maxtext_formula():
         np.testing.assert_allclose(p.reshape(32, 6)[t][ok], ref, rtol=1e-9, atol=1e-12)
 
 
+@pytest.mark.parametrize("seed,docs", [(30, False), (31, True)])
+def test_per_branch_mode_is_maxtext_formula(seed, docs):
+    """The per-branch mode is the MaxText page's formula as printed:
+    L1_Normalize(Sum_h Softmax_k(z)) over the selected entries, computed here
+    with scipy's softmax from the same inputs; window and sink play no part."""
+    from scipy.special import softmax
+    S, H, D, K, cr = 32, 3, 16, 6, 4
+    Q, _, pool, idx, snk, ds = _rand_problem(seed, B=1, S=S, H=H, D=D, K=K, cr=cr, docs=docs)
+    scale = 0.3
+    p, bad = oracle.distill_target(Q, pool, idx, None, None, ds, cr, scale, per_branch=True)
+    assert bad == 0
+    q, pl = _f64(Q)[0], _f64(pool)[0]
+    p = p.reshape(S, K)
+    for t in range(S):
+        d0 = 0 if ds is None else min(max(int(ds[0, t]), 0), t)
+        j = idx[0, t].astype(int)
+        ok = (j >= 0) & ((j + 1) * cr - 1 <= t) & (j * cr >= d0)
+        if not ok.any():
+            assert np.all(p[t] == 0.0)
+            continue
+        z = scale * q[t] @ pl[j[ok]].T                 # [H, n]
+        ref = softmax(z, axis=1).sum(axis=0)
+        ref = ref / ref.sum()
+        np.testing.assert_allclose(p[t][ok], ref, rtol=1e-12, atol=1e-15)
+        assert np.all(p[t][~ok] == 0.0)
+
+
+def test_per_branch_mode_ignores_window_and_sink_and_sums_to_one():
+    """Changing the window log-mass or the sink cannot move the per-branch
+    target, while it does move the joint one; every non-empty row sums to 1
+    (each head contributes a full distribution, so the 1e-10 floor is idle)."""
+    Q, Kw, pool, idx, snk, _ = _rand_problem(32, B=1, S=32, H=3, D=16, K=6)
+    wl = oracle.window_lse(Q, Kw, None, 5, 0.25)
+    p1, _ = oracle.distill_target(Q, pool, idx, wl, snk, None, 4, 0.25, per_branch=True)
+    p2, _ = oracle.distill_target(Q, pool, idx, wl + 5.0, snk * 0 + 30.0, None, 4, 0.25, per_branch=True)
+    np.testing.assert_array_equal(p1, p2)
+    j1, _ = oracle.distill_target(Q, pool, idx, wl, snk, None, 4, 0.25)
+    j2, _ = oracle.distill_target(Q, pool, idx, wl + 5.0, snk, None, 4, 0.25)
+    assert np.abs(j1 - j2).max() > 1e-3
+    rows = p1.sum(axis=1)
+    nonempty = rows > 0
+    np.testing.assert_allclose(rows[nonempty], 1.0, rtol=1e-12)
+
+
 def test_target_invariants():
     Q, Kw, pool, idx, snk, ds = _rand_problem(30, B=2, S=32, H=4, D=16, K=8, docs=True)
     scale = 0.25
