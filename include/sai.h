@@ -104,7 +104,12 @@ sai_status sai_window_lse(const uint16_t *Q, const uint16_t *Kw, const int32_t *
  *
  *   Q          [B,S,H,D] bf16, 16-byte aligned
  *   pool       [B,P,D]   bf16 compressed entries, 16-byte aligned
- *   idx        [B,S,K]   int32 top-k rows, -1 = empty slot
+ *   idx        [B,S,K]   int32 top-k rows, -1 = empty slot; or NULL for the
+ *              dense warm-up stage (MaxText page "Add Indexer Loss
+ *              [Deepseek v4]": teacher over all causal blocks before sparse
+ *              training), where slot k is compressed block k (idx[b,t,k] = k
+ *              implicitly; with K = S/cr every block; the causal and document
+ *              rules still mask the slots a token cannot see)
  *   window_lse [B,S,H]   fp32 (from sai_window_lse)
  *   sink       [H] fp32 per-head sink logits, or NULL for no sink
  *   doc_start  [B,S] int32 or NULL
@@ -121,6 +126,31 @@ sai_status sai_distill_target(const uint16_t *Q, const uint16_t *pool, const int
                               const float *window_lse, const float *sink, const int32_t *doc_start,
                               int B, int S, int H, int D, int K, int cr, float scale,
                               float *p, int32_t *d_err, void *stream);
+
+/* Flags of sai_distill_target_ex. */
+#define SAI_TARGET_PER_BRANCH 1u
+
+/*
+ * sai_distill_target_ex -- sai_distill_target with a flags word.
+ *
+ * flags == 0 is exactly sai_distill_target. SAI_TARGET_PER_BRANCH selects
+ * the earlier per-branch target, which the Primus page keeps as an A/B
+ * switch (second commit message: PRIMUS_V4_DISTILL_NONCOMP_LSE=0) and the
+ * MaxText page "Add Indexer Loss [Deepseek v4]" prints in its commit
+ * messages: every head is normalised over the selected compressed entries
+ * alone and the L1 floor is the earlier 1e-10,
+ *
+ *   lse_full[h] = clse[h],   p[b,t,k] = u[k] / max(m, 1e-10),
+ *
+ * i.e. p is the head mean of the per-head softmaxes over the selected slots.
+ * window_lse and sink are not read in that mode and may be NULL.
+ * Unknown flag bits return SAI_ERR_UNSUPPORTED; everything else (layouts,
+ * sizes, errors, ownership) is as for sai_distill_target.
+ */
+sai_status sai_distill_target_ex(const uint16_t *Q, const uint16_t *pool, const int32_t *idx,
+                                 const float *window_lse, const float *sink, const int32_t *doc_start,
+                                 int B, int S, int H, int D, int K, int cr, float scale, unsigned flags,
+                                 float *p, int32_t *d_err, void *stream);
 
 /* Bytes of device workspace sai_distill_kl needs for these sizes. */
 size_t sai_distill_kl_workspace_bytes(int B, int S, int K);

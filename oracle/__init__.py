@@ -89,8 +89,11 @@ def distill_target(Q, pool, idx, wl, sink, doc_start, cr: int, scale: float, tok
 
     per_branch selects the earlier per-branch target (every head normalised
     over the selected entries alone, floor 1e-10); wl and sink are then
-    unused and may be None."""
+    unused and may be None. idx=None is the dense warm-up stage: slot k is
+    compressed block k for every token (K = S/cr)."""
     B, S, H, D = Q.shape
+    if idx is None:
+        idx = np.broadcast_to(np.arange(S // cr, dtype=np.int32), (B, S, S // cr))
     K = idx.shape[-1]
     Q = _c(Q, np.uint16); pool = _c(pool, np.uint16); idx = _c(idx, np.int32)
     wl = _c(wl, np.float64); sink = _c(sink, np.float32); ds = _c(doc_start, np.int32)

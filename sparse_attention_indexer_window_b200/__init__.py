@@ -45,6 +45,10 @@ _lib.sai_window_lse.argtypes = [_P, _P, _P, _I, _I, _I, _I, _I, _F, _P, _P]
 _lib.sai_window_lse.restype = _I
 _lib.sai_distill_target.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P]
 _lib.sai_distill_target.restype = _I
+_lib.sai_distill_target_ex.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, ctypes.c_uint,
+                                       _P, _P, _P]
+_lib.sai_distill_target_ex.restype = _I
+TARGET_PER_BRANCH = 1   # flag of sai_distill_target_ex: the earlier per-branch target
 _lib.sai_distill_kl_workspace_bytes.argtypes = [_I, _I, _I]
 _lib.sai_distill_kl_workspace_bytes.restype = ctypes.c_size_t
 _lib.sai_distill_kl.argtypes = [_P, _P, _P, _I, _I, _I, _F, _P, _P, _P, ctypes.c_size_t, _P]
@@ -128,16 +132,25 @@ def window_lse(Q: torch.Tensor, Kw: torch.Tensor, W: int, scale: float,
     return out
 
 
-def distill_target(Q: torch.Tensor, pool: torch.Tensor, idx: torch.Tensor, wl: torch.Tensor, cr: int,
+def distill_target(Q: torch.Tensor, pool: torch.Tensor, idx: Optional[torch.Tensor], wl: Optional[torch.Tensor], cr: int,
                    scale: float, sink: Optional[torch.Tensor] = None, doc_start: Optional[torch.Tensor] = None,
-                   err: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+                   err: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
+                   per_branch: bool = False) -> torch.Tensor:
+    """p[B,S,K] through sai_distill_target_ex. per_branch=True selects the
+    earlier per-branch target; wl and sink are then not used (may be None).
+    idx=None is the dense warm-up stage: every compressed block is a slot
+    (K = S/cr, slot k = block k)."""
     B, S, H, D = Q.shape
-    K = idx.shape[-1]
+    K = idx.shape[-1] if idx is not None else S // cr
     Q = _bf16_bits(Q, "Q")
     pool = _bf16_bits(pool, "pool")
     if tuple(pool.shape) != (B, S // cr, D):
         raise ValueError("pool must be [B,S/cr,D]")
     _want(idx, "idx", torch.int32, (B, S, K))
+    if per_branch:
+        wl, sink = None, None
+    elif wl is None:
+        raise ValueError("window_lse is required unless per_branch")
     _want(wl, "window_lse", torch.float32, (B, S, H))
     if sink is not None:
         # The Primus page: a sink must hold one value per head (else ValueError).
@@ -149,9 +162,10 @@ def distill_target(Q: torch.Tensor, pool: torch.Tensor, idx: torch.Tensor, wl: t
     if out is None:
         out = torch.empty((B, S, K), dtype=torch.float32, device=Q.device)
     _want(out, "out", torch.float32, (B, S, K))
-    st = _lib.sai_distill_target(_ptr(Q), _ptr(pool), _ptr(idx), _ptr(wl), _ptr(sink), _ptr(doc_start),
-                                 B, S, H, D, K, int(cr), float(scale), _ptr(out), _ptr(err), _stream(Q.device))
-    _check(st, "sai_distill_target")
+    st = _lib.sai_distill_target_ex(_ptr(Q), _ptr(pool), _ptr(idx), _ptr(wl), _ptr(sink), _ptr(doc_start),
+                                    B, S, H, D, K, int(cr), float(scale), TARGET_PER_BRANCH if per_branch else 0,
+                                    _ptr(out), _ptr(err), _stream(Q.device))
+    _check(st, "sai_distill_target_ex")
     return out
 
 

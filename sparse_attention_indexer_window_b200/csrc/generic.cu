@@ -15,6 +15,7 @@ namespace {
 
 constexpr int kGenThreads = 128;
 constexpr float kLnFltMinG = -87.33654475055310898657f;
+constexpr float kLnOldFloorG = -23.025850929940457f;  // log(1e-10), the per-branch target's floor
 
 __device__ __forceinline__ float bf16f(uint16_t b) { return __uint_as_float(((uint32_t)b) << 16); }
 
@@ -83,7 +84,7 @@ __global__ void __launch_bounds__(kGenThreads)
     target_generic_kernel(const uint16_t *__restrict__ Q, const uint16_t *__restrict__ pool,
                           const int32_t *__restrict__ idx, const float *__restrict__ wl,
                           const float *__restrict__ sink, const int32_t *__restrict__ doc_start, int S, int H,
-                          int D, int K, int cr, float scale, float *__restrict__ p, int32_t *err)
+                          int D, int K, int cr, float scale, int per_branch, float *__restrict__ p, int32_t *err)
 {
     extern __shared__ float gsm[];
     float *qs = gsm;                              // [H][D]
@@ -110,7 +111,7 @@ __global__ void __launch_bounds__(kGenThreads)
     __syncthreads();
     float *prow = p + (size_t)g * K;
     for (int k = threadIdx.x; k < K; k += blockDim.x) {
-        const int j = idx[(size_t)g * K + k];
+        const int j = idx ? idx[(size_t)g * K + k] : k;   // NULL: dense, slot k is block k
         const bool inr = j >= 0 && j < P;
         if (!(j == -1 || inr) && err)
             atomicExch(err, kErrIndex);
@@ -143,6 +144,11 @@ __global__ void __launch_bounds__(kGenThreads)
         for (int j = 0; j < nsel; ++j)
             se += expf(zs[j * H + h] - M);
         const float clse = M + logf(se);
+        hM[h] = M;
+        if (per_branch) {
+            hA[h] = M - clse;                     // each head normalised over its selected entries
+            continue;
+        }
         const float w = wl[(size_t)g * H + h];
         float mm = fmaxf(w, clse);
         if (sink)
@@ -150,7 +156,6 @@ __global__ void __launch_bounds__(kGenThreads)
         float acc = expf(w - mm) + expf(clse - mm);
         if (sink)
             acc += expf(sink[h] - mm);
-        hM[h] = M;
         hA[h] = M - (mm + logf(acc));
     }
     __syncthreads();
@@ -166,8 +171,9 @@ __global__ void __launch_bounds__(kGenThreads)
         mpart += u;
     }
     const float mt = block_sum(mpart, scratch);
-    const bool plain = logf(mt) + At >= kLnFltMinG;
-    const float f = plain ? 0.f : expf(At - kLnFltMinG);
+    const float ln_floor = per_branch ? kLnOldFloorG : kLnFltMinG;
+    const bool plain = logf(mt) + At >= ln_floor;
+    const float f = plain ? 0.f : expf(At - ln_floor);
     for (int j = threadIdx.x; j < nsel; j += blockDim.x)
         prow[slots[j]] = plain ? us[j] / mt : us[j] * f;
 }
@@ -195,7 +201,8 @@ size_t target_simt_smem_bytes(int H, int D, int K)
 
 cudaError_t launch_target_simt(const uint16_t *Q, const uint16_t *pool, const int32_t *idx, const float *wl,
                                const float *sink, const int32_t *doc_start, int B, int S, int H, int D, int K,
-                               int cr, float scale, float *p, int32_t *err, cudaStream_t stream)
+                               int cr, float scale, int per_branch, float *p, int32_t *err,
+                               cudaStream_t stream)
 {
     const size_t smem = target_simt_smem_bytes(H, D, K);
     cudaError_t e =
@@ -203,7 +210,7 @@ cudaError_t launch_target_simt(const uint16_t *Q, const uint16_t *pool, const in
     if (e != cudaSuccess)
         return e;
     target_generic_kernel<<<B * S, kGenThreads, smem, stream>>>(Q, pool, idx, wl, sink, doc_start, S, H, D, K, cr,
-                                                                scale, p, err);
+                                                                scale, per_branch, p, err);
     return cudaGetLastError();
 }
 

@@ -146,7 +146,23 @@ sai_status sai_distill_target(const uint16_t *Q, const uint16_t *pool, const int
                               const float *sink, const int32_t *doc_start, int B, int S, int H, int D, int K,
                               int cr, float scale, float *p, int32_t *d_err, void *stream)
 {
-    if (!Q || !pool || !idx || !window_lse || !p)
+    return sai_distill_target_ex(Q, pool, idx, window_lse, sink, doc_start, B, S, H, D, K, cr, scale, 0u, p, d_err,
+                                 stream);
+}
+
+sai_status sai_distill_target_ex(const uint16_t *Q, const uint16_t *pool, const int32_t *idx,
+                                 const float *window_lse, const float *sink, const int32_t *doc_start, int B, int S,
+                                 int H, int D, int K, int cr, float scale, unsigned flags, float *p, int32_t *d_err,
+                                 void *stream)
+{
+    if (flags & ~SAI_TARGET_PER_BRANCH)
+        return SAI_ERR_UNSUPPORTED;
+    const bool per_branch = (flags & SAI_TARGET_PER_BRANCH) != 0;
+    if (per_branch) {
+        window_lse = nullptr;   // not read in this mode
+        sink = nullptr;
+    }
+    if (!Q || !pool || (!window_lse && !per_branch) || !p)     // idx NULL: dense over all blocks
         return SAI_ERR_NULL;
     if (B < 1 || S < 1 || H < 1 || D < 1 || K < 1 || cr < 1 || (D % 8) != 0 || (S % cr) != 0 ||
         !isfinite(scale) || scale <= 0.f)
@@ -156,8 +172,8 @@ sai_status sai_distill_target(const uint16_t *Q, const uint16_t *pool, const int
         return SAI_ERR_SHAPE;
     if ((int64_t)B * S * H * D > INT32_MAX || (int64_t)B * S * K > INT32_MAX)
         return SAI_ERR_SHAPE;
-    if (!al16(Q) || !al16(pool) || !al4(idx) || !al4(window_lse) || !al4(p) || (sink && !al4(sink)) ||
-        (doc_start && !al4(doc_start)) || (d_err && !al4(d_err)))
+    if (!al16(Q) || !al16(pool) || (idx && !al4(idx)) || (window_lse && !al4(window_lse)) || !al4(p) ||
+        (sink && !al4(sink)) || (doc_start && !al4(doc_start)) || (d_err && !al4(d_err)))
         return SAI_ERR_ALIGN;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const int smem_cap = max_smem_optin();
@@ -176,8 +192,9 @@ sai_status sai_distill_target(const uint16_t *Q, const uint16_t *pool, const int
         a.P = P;
         a.n_tok = B * S;
         a.tiles_per_group = 256 / H;
-        a.idx_bulk = ((K % 4) == 0 && al16(idx)) ? 1 : 0;
+        a.idx_bulk = (idx && (K % 4) == 0 && al16(idx)) ? 1 : 0;
         a.n_astages = n_astages;
+        a.per_branch = per_branch ? 1 : 0;
         a.pool_box_rows = (int)std::min<int64_t>(128, (int64_t)B * P);
         a.scale = scale;
         a.pool = pool;
@@ -200,7 +217,7 @@ sai_status sai_distill_target(const uint16_t *Q, const uint16_t *pool, const int
     }
     if ((int)sai::target_simt_smem_bytes(H, D, K) <= smem_cap)
         return cuda_status(sai::launch_target_simt(Q, pool, idx, window_lse, sink, doc_start, B, S, H, D, K, cr,
-                                                   scale, p, d_err, st));
+                                                   scale, per_branch ? 1 : 0, p, d_err, st));
     return SAI_ERR_UNSUPPORTED;
 }
 

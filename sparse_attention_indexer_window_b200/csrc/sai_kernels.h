@@ -32,6 +32,7 @@ struct TgtTcArgs {
     int idx_bulk;         // idx rows are 16-byte aligned (K % 4 == 0): stage them by bulk copy
     int n_astages;        // depth of the gathered-row stage ring
     int pool_box_rows;    // rows of the pool's TMA box (min(128, B*P))
+    int per_branch;       // 1: per-branch target (lse_full = clse, floor 1e-10); wl and sink unused
     float scale;
     const uint16_t *pool;
     const int32_t *idx;
@@ -54,7 +55,8 @@ cudaError_t launch_window_lse_simt(const uint16_t *Q, const uint16_t *Kw, const 
 size_t target_simt_smem_bytes(int H, int D, int K);
 cudaError_t launch_target_simt(const uint16_t *Q, const uint16_t *pool, const int32_t *idx, const float *wl,
                                const float *sink, const int32_t *doc_start, int B, int S, int H, int D, int K,
-                               int cr, float scale, float *p, int32_t *err, cudaStream_t stream);
+                               int cr, float scale, int per_branch, float *p, int32_t *err,
+                               cudaStream_t stream);
 
 // ---------------------------------------------------------------- distill_kl
 struct KlPlan {

@@ -89,6 +89,7 @@ constexpr int kMeta = 3;                            // compaction runs up to two
 constexpr uint32_t kATile = 128 * 128;              // 128 rows x 128 bytes
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLnFltMin = -87.33654475055310898657f;  // log(2^-126)
+constexpr float kLnOldFloor = -23.025850929940457f;      // log(1e-10), the per-branch target's floor
 
 template <int HH>
 struct EpiState {                 // one per epilogue warpgroup
@@ -239,7 +240,7 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
             // lane L takes 4 consecutive slots
             uint32_t *rw = rowoff + m3 * Kp;
             int32_t *sl = slot + m3 * Kp;
-            const int32_t *grow = a.idx + (size_t)g * K;
+            const int32_t *grow = a.idx ? a.idx + (size_t)g * K : nullptr;   // NULL: slot k is block k
             int nsel = 0, nmask = 0;
             bool bad = false;
             for (int k0 = 0; k0 < K; k0 += 128) {
@@ -256,7 +257,7 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
                 } else {
 #pragma unroll
                     for (int e = 0; e < 4; ++e)
-                        j[e] = (k + e < K) ? __ldg(grow + k + e) : -1;
+                        j[e] = (k + e < K) ? (grow ? __ldg(grow + k + e) : k + e) : -1;
                 }
                 int cs = 0, cm = 0;
                 bool sel[4];
@@ -536,7 +537,7 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
             const int g = a.n_tok - 1 - gt;
             const int m3 = it % kMeta;
             // window log-mass of this token's heads, fetched early
-            const float wl_h = (et < HH) ? a.wl[(size_t)g * HH + et] : 0.f;
+            const float wl_h = (et < HH && a.wl) ? a.wl[(size_t)g * HH + et] : 0.f;
             // leader waits; the named barrier hands the outcome to the group
             if (et == 0)
                 st.flag = mbar_wait(&sm->meta_full[m3], (it / kMeta) & 1, abort_flag, a.err) ? 1 : 0;
@@ -670,11 +671,16 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
                             if (et < HH) {
                                 const float M = st.colM[et] * 0.69314718055994531f;  // natural log units
                                 const float clse = M + logf(st.colS[et]);
-                                float mm = fmaxf(fmaxf(wl_h, clse), sink_h);
-                                float acc = expf(wl_h - mm) + expf(clse - mm);
-                                if (a.sink)
-                                    acc += expf(sink_h - mm);
-                                st.head_a[et] = M - (mm + logf(acc));
+                                if (a.per_branch) {
+                                    // each head normalised over its selected entries alone
+                                    st.head_a[et] = M - clse;
+                                } else {
+                                    float mm = fmaxf(fmaxf(wl_h, clse), sink_h);
+                                    float acc = expf(wl_h - mm) + expf(clse - mm);
+                                    if (a.sink)
+                                        acc += expf(sink_h - mm);
+                                    st.head_a[et] = M - (mm + logf(acc));
+                                }
                             }
                             named_bar_sync(bar_id, 128);
                             float x = -INFINITY;
@@ -755,8 +761,9 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
             named_bar_sync(bar_id, 128);
             const float mtot = st.red_m[0] + st.red_m[1] + st.red_m[2] + st.red_m[3];
             if (nsel > 0) {
-                const bool plain = logf(mtot) + At >= kLnFltMin;
-                const float f = plain ? 1.0f / mtot : expf(At - kLnFltMin);
+                const float ln_floor = a.per_branch ? kLnOldFloor : kLnFltMin;
+                const bool plain = logf(mtot) + At >= ln_floor;
+                const float f = plain ? 1.0f / mtot : expf(At - ln_floor);
                 for (int jj = et; jj < K; jj += 128)
                     prow[sl[jj]] = (jj < nsel) ? ub[jj] * f : 0.f;
             } else {

@@ -78,6 +78,17 @@ def test_distill_target_host_errors(sai):
     assert f(FAKE, FAKE_MIS, FAKE, FAKE, None, None, 1, 64, 4, 32, 8, 4, 0.1, FAKE, None, None) == 7
 
 
+def test_distill_target_ex_host_errors(sai):
+    """The flags variant: unknown flag bits are refused; the joint target
+    (flags 0) needs window_lse. Only paths that return before any launch."""
+    f = sai.lib().sai_distill_target_ex
+    args = lambda wl, flags: (FAKE, FAKE, FAKE, wl, None, None, 1, 64, 4, 32, 8, 4, 0.1, flags, FAKE, None, None)
+    assert f(*args(FAKE, 2)) == 3                     # unknown flag bit
+    assert f(*args(FAKE, 0x80000000)) == 3
+    assert f(*args(None, 0)) == 1                     # joint target without window_lse
+    assert f(*args(FAKE, 1)[:6], 1, 64, 4, 32, 8, 3, 0.1, 1, FAKE, None, None) == 2   # S % cr, per-branch
+
+
 def test_distill_kl_host_errors(sai):
     f = sai.lib().sai_distill_kl
     need = sai.lib().sai_distill_kl_workspace_bytes(1, 64, 8)

@@ -180,6 +180,38 @@ def test_target_long_way_on_tiny_workload():
     np.testing.assert_allclose(p, ref, rtol=0, atol=1e-12)
 
 
+@pytest.mark.parametrize("docs", [False, True])
+def test_dense_mode_is_every_causal_block(docs):
+    """Dense warm-up (idx omitted): slot k is compressed block k. The target
+    equals the joint softmax written out the long way over the explicit
+    index row 0..P-1, puts exactly zero on blocks a token cannot see (the
+    MaxText page's rule: with t=4, cr=4 block 0 visible, block 1 masked), and
+    with every block visible equals the sparse target that selects them all."""
+    S, H, D, cr, W = 32, 3, 16, 4, 5
+    Q, Kw, pool, _, snk, ds = _rand_problem(40, B=1, S=S, H=H, D=D, K=6, cr=cr, docs=docs)
+    P = S // cr
+    scale = 0.25
+    wl = oracle.window_lse(Q, Kw, ds, W, scale)
+    p, bad = oracle.distill_target(Q, pool, None, wl, snk, ds, cr, scale)
+    assert bad == 0 and p.shape == (S, P)
+    arange = np.broadcast_to(np.arange(P, dtype=np.int32), (1, S, P)).copy()
+    ref = target_long_way(Q, Kw, pool, arange, snk, ds, W, cr, scale)
+    np.testing.assert_allclose(p, ref, rtol=0, atol=1e-12)
+    t = 4
+    assert p[t, 0] > 0 and np.all(p[t, 1:] == 0)
+    for t in range(S):
+        d0 = 0 if ds is None else min(max(int(ds[0, t]), 0), t)
+        for j in range(P):
+            if (j + 1) * cr - 1 > t or j * cr < d0:
+                assert p[t, j] == 0.0
+    if not docs:
+        t = S - 1
+        idx = np.full((1, S, P), -1, dtype=np.int32)
+        idx[0, t] = np.arange(P)[::-1]                 # all blocks, another slot order
+        ps, _ = oracle.distill_target(Q, pool, idx, wl, snk, None, cr, scale)
+        np.testing.assert_allclose(ps[t][::-1], p[t], rtol=1e-13, atol=0)
+
+
 def test_target_long_way_on_small_workload_sample():
     """The local-branch-dominates workload (sink +8, q aligned to the key)."""
     w = synth.make("small")
