@@ -20,7 +20,7 @@
 // Gather. A dedicated warp compacts each token's idx row (selected slots
 // first, masked slots last), up to two tokens ahead; the idx rows arrive by
 // its own cp.async copies, and the compaction turns pool rows into byte
-// offsets. Nine
+// offsets. Eight
 // gather warps each own one 16 KB slot of the A ring and fill every stage
 // that lands in it: 128 selected rows x one 128-byte chunk of D, copied into
 // the swizzled K-major operand layout with 16-byte cp.async (eight lanes per
@@ -52,9 +52,9 @@
 //        = u'[k] exp(A - log FLT_MIN)   otherwise (the float32-tiny floor),
 // so no intermediate is subnormal however small each head's compressed share.
 //
-// Warp roles (640 threads): warp 0 idx staging and compaction, warps 1..7,
-// 9 and 10 row gathers, warp 11 Q loads, warp 8 MMA issuer and TMEM owner,
-// warps 12..15 and 16..19 the two epilogue groups. Persistent CTAs walk tokens from the last
+// Warp roles (640 threads): warp 0 idx staging and compaction, warps 1..7
+// and 9 row gathers, warp 11 Q loads, warps 8 (also the TMEM owner) and 10
+// the two MMA issuers, warps 12..15 and 16..19 the two epilogue groups. Persistent CTAs walk tokens from the last
 // (heaviest) to the first. All mbarrier waits are bounded; a timeout is
 // reported through err and the CTA unwinds. Named barriers are only used
 // where every participating thread is guaranteed to arrive.
@@ -64,13 +64,14 @@
 namespace sai {
 namespace {
 
-// Warpgroups 0..2 (warps 0..11): warp 0 compaction, warp 8 MMA, warp 11 Q
-// loads, the other nine warps row gathers; warpgroups 3 and 4 (warps
-// 12..19): epilogue.
+// Warpgroups 0..2 (warps 0..11): warp 0 compaction, warps 8 and 10 MMA,
+// warp 11 Q loads, the other eight warps row gathers; warpgroups 3 and 4
+// (warps 12..19): epilogue.
 constexpr int kMetaWarp = 0;
-constexpr int kMmaWarp = 8;
+constexpr int kMmaWarp = 8;                         // MMA thread 0, TMEM owner
+constexpr int kMmaWarp2 = 10;                       // MMA thread 1
 constexpr int kQWarp = 11;
-constexpr int kGatherWarps = 9;
+constexpr int kGatherWarps = 8;
 constexpr int kEpiWarp0 = 12;
 constexpr int kTgtThreads = 20 * 32;                // 640
 // Register split (setmaxnreg): launched at kLaunchRegs a thread; warpgroups
@@ -109,7 +110,7 @@ struct TgtSmem {
     uint64_t q_full[kQStagesMax], q_empty[kQStagesMax];
     uint64_t acc_full[2], acc_empty[2];
     uint64_t meta_full[kMeta], meta_empty[kMeta];
-    uint64_t drain;
+    uint64_t drain[2];
     uint32_t tmem_base;
     int abort_flag;
     int nsel[kMeta];
@@ -169,17 +170,18 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
         }
         for (int s = 0; s < QS; ++s) {
             mbar_init(&sm->q_full[s], 1);
-            mbar_init(&sm->q_empty[s], 1);
+            mbar_init(&sm->q_empty[s], 2);      // both MMA threads release a Q chunk
         }
         for (int b = 0; b < 2; ++b) {
-            mbar_init(&sm->acc_full[b], 1);
+            mbar_init(&sm->acc_full[b], 2);     // both MMA threads commit a group
             mbar_init(&sm->acc_empty[b], 4);
         }
         for (int b = 0; b < kMeta; ++b) {
             mbar_init(&sm->meta_full[b], 1);
             mbar_init(&sm->meta_empty[b], 1);
         }
-        mbar_init(&sm->drain, 1);
+        mbar_init(&sm->drain[0], 1);
+        mbar_init(&sm->drain[1], 1);
         sm->abort_flag = 0;
         fence_mbar_init();
     }
@@ -349,13 +351,13 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
                     mbar_drain(&sm->q_full[s], (q_last >> s) & 1u);
         }
         __syncwarp();
-    } else if (warp != kMmaWarp && warp < kEpiWarp0) {
+    } else if (warp != kMmaWarp && warp != kMmaWarp2 && warp < kEpiWarp0) {
         // ============================================================ gathers
         // Gather warp gw owns A ring slot gw: it fills every stage that lands
         // there (stages gw, gw + NA, gw + 2 NA, ... of the MMA's sequence),
         // waits for its own copies and publishes the stage with one arrival.
         // Each slot has a single producer, so its phases are seen in order.
-        const int gw = warp < kMmaWarp ? warp - 1 : warp - 2;   // 0..8
+        const int gw = warp < kMmaWarp ? warp - 1 : warp - 2;   // 0..7
         if (gw < NA) {
             const char *pool_bytes = reinterpret_cast<const char *>(a.pool);
             const int seg = lane & 7;            // 16-byte segment of a 128-byte row chunk
@@ -434,12 +436,16 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
             }
         }
         __syncwarp();
-    } else if (warp == kMmaWarp) {
+    } else if (warp == kMmaWarp || warp == kMmaWarp2) {
         // ============================================================ MMA
-        // One thread issues everything, stage by stage. (Issuing a chunk's
-        // MMAs back to back measured slower: at N = H the MMAs are bound by
-        // shared-memory operand reads, and bursts of them starve the gathers'
-        // shared-memory writes.)
+        // Two threads issue the MMAs: thread mt takes the tiles i with
+        // i % 2 == mt, so each accumulator's chain (chunk 0 initialises, the
+        // later chunks accumulate) stays with one thread, while the other
+        // thread's MMAs fill the tensor pipe during this one's barrier waits,
+        // fences and commits (each of which costs the issuing thread on the
+        // order of 150 cycles on this part). Both walk the whole stage
+        // sequence and both release every Q chunk and every TMEM group.
+        const int mt = (warp == kMmaWarp) ? 0 : 1;
         if (lane == 0) {
             const uint32_t idesc = idesc_bf16_f32(128, HH);
             int as = 0, qs = 0;
@@ -477,21 +483,22 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
                                 ok = false;
                                 break;
                             }
-                            // are all of this chunk's stages published already?
                             const uint64_t dq = sdesc_k_sw128(smem_u32(q_buf + qs * kQTile));
                             for (int i = 0; i < ntg; ++i) {
-                                if (!mbar_wait(&sm->a_full[as], aph, abort_flag, a.err)) {
-                                    ok = false;
-                                    break;
-                                }
-                                tc_fence_after();
-                                const uint64_t da = sdesc_k_sw128(smem_u32(a_buf + as * kATile));
-                                const uint32_t d_tmem = dbase + i * HH;
+                                if ((i & 1) == mt) {
+                                    if (!mbar_wait(&sm->a_full[as], aph, abort_flag, a.err)) {
+                                        ok = false;
+                                        break;
+                                    }
+                                    tc_fence_after();
+                                    const uint64_t da = sdesc_k_sw128(smem_u32(a_buf + as * kATile));
+                                    const uint32_t d_tmem = dbase + i * HH;
 #pragma unroll
-                                for (int kk = 0; kk < 4; ++kk)
-                                    umma_bf16(d_tmem, da + 2 * kk, dq + 2 * kk, idesc, (c | kk) != 0);
-                                umma_commit(&sm->a_empty[as]);
-                                issued = true;
+                                    for (int kk = 0; kk < 4; ++kk)
+                                        umma_bf16(d_tmem, da + 2 * kk, dq + 2 * kk, idesc, (c | kk) != 0);
+                                    umma_commit(&sm->a_empty[as]);
+                                    issued = true;
+                                }
                                 if (++as == NA) {
                                     as = 0;
                                     aph ^= 1u;
@@ -512,8 +519,8 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
                 }
             }
             if (!ok && issued) {
-                umma_commit(&sm->drain);
-                mbar_drain(&sm->drain, 0);
+                umma_commit(&sm->drain[mt]);
+                mbar_drain(&sm->drain[mt], 0);
             }
         }
         __syncwarp();
