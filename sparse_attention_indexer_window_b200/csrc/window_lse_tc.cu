@@ -19,7 +19,7 @@
 // Warp roles (320 threads): warp 0 TMA producer (and TMEM owner), warp 1 MMA
 // issuer, warps 2..5 and 6..9 two epilogue groups that take alternate tiles,
 // each with its own 256-column TMEM accumulator. The kernel is bound by
-// reading Q from HBM once; six 34 KB stages keep enough bytes in flight.
+// reading Q from HBM once; the stage ring keeps about 200 KB in flight.
 // Every wait is bounded; on timeout the kernel writes NaN rows and unwinds.
 #include "sai_device.cuh"
 #include "sai_kernels.h"
@@ -48,8 +48,14 @@ __global__ void __launch_bounds__(kWinThreads, 1)
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t b_bytes = a.b_stage_bytes;  // NB x 128, rounded to 1024
-    const uint32_t stage_bytes = kATileBytes + b_bytes;
-    WinSmem *sm = reinterpret_cast<WinSmem *>(base + kWinStages * stage_bytes);
+    const uint32_t chunk_bytes = kATileBytes + b_bytes;   // one 64-column chunk of D: Q tile + key band
+    // A stage carries two chunks when D allows it (three stages), else one
+    // (six stages): the same bytes in flight, half the barrier waits, fences
+    // and commits per MMA, which cost the issuing thread ~150 cycles each.
+    const int cps = ((a.D / 64) % 2 == 0) ? 2 : 1;
+    const int n_stages = kWinStages / cps;
+    const uint32_t stage_bytes = cps * chunk_bytes;
+    WinSmem *sm = reinterpret_cast<WinSmem *>(base + kWinStages * chunk_bytes);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -95,25 +101,28 @@ __global__ void __launch_bounds__(kWinThreads, 1)
                 const int t0 = g0 - b * a.S;
                 const int rowQ = g0 * a.H;
                 const int rowK = b * a.S + t0 - a.W + 1;
-                for (int c = 0; c < n_chunks; ++c) {
+                for (int c = 0; c < n_chunks; c += cps) {
                     if (!mbar_wait(&sm->empty[stage], phase ^ 1u, abort_flag, nullptr)) {
                         ok = false;
                         break;
                     }
                     uint8_t *sa = base + stage * stage_bytes;
-                    mbar_arrive_expect_tx(&sm->full[stage], kATileBytes + a.NB * 128u);
-                    tma_load_2d(sa, &mapQ, &sm->full[stage], c * 64, rowQ);
-                    tma_load_2d(sa + kATileBytes, &mapK, &sm->full[stage], c * 64, rowK);
+                    mbar_arrive_expect_tx(&sm->full[stage], (uint32_t)cps * (kATileBytes + a.NB * 128u));
+                    for (int cc = 0; cc < cps; ++cc) {
+                        tma_load_2d(sa + cc * chunk_bytes, &mapQ, &sm->full[stage], (c + cc) * 64, rowQ);
+                        tma_load_2d(sa + cc * chunk_bytes + kATileBytes, &mapK, &sm->full[stage], (c + cc) * 64,
+                                    rowK);
+                    }
                     issued_mask |= 1u << stage;
                     last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
-                    if (++stage == kWinStages) {
+                    if (++stage == n_stages) {
                         stage = 0;
                         phase ^= 1u;
                     }
                 }
             }
             if (!ok) {
-                for (int s = 0; s < kWinStages; ++s)
+                for (int s = 0; s < n_stages; ++s)
                     if (issued_mask & (1u << s))
                         mbar_drain(&sm->full[s], (last_parity >> s) & 1u);
             }
@@ -135,24 +144,26 @@ __global__ void __launch_bounds__(kWinThreads, 1)
             }
             tc_fence_after();
             const uint32_t d_tmem = tmem + buf * 256;
-            for (int c = 0; c < n_chunks; ++c) {
+            for (int c = 0; c < n_chunks; c += cps) {
                 if (!mbar_wait(&sm->full[stage], phase, abort_flag, nullptr)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
                 if (lane == 0) {
-                    const uint32_t sa = smem_u32(base + stage * stage_bytes);
-                    const uint64_t da = sdesc_k_sw128(sa);
-                    const uint64_t db = sdesc_k_sw128(sa + kATileBytes);
+                    for (int cc = 0; cc < cps; ++cc) {
+                        const uint32_t sa = smem_u32(base + stage * stage_bytes + cc * chunk_bytes);
+                        const uint64_t da = sdesc_k_sw128(sa);
+                        const uint64_t db = sdesc_k_sw128(sa + kATileBytes);
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        umma_bf16(d_tmem, da + 2 * kk, db + 2 * kk, idesc, (c | kk) != 0);
+                        for (int kk = 0; kk < 4; ++kk)
+                            umma_bf16(d_tmem, da + 2 * kk, db + 2 * kk, idesc, ((c + cc) | kk) != 0);
+                    }
                     umma_commit(&sm->empty[stage]);
                     issued = true;
                 }
                 __syncwarp();
-                if (++stage == kWinStages) {
+                if (++stage == n_stages) {
                     stage = 0;
                     phase ^= 1u;
                 }

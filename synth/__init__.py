@@ -190,13 +190,16 @@ def _idx_topk_sorted(rng, S, cr, K, doc_start, b) -> np.ndarray:
 
 def make(name: str, *, seed: Optional[int] = None, with_sink: bool = True,
          S: Optional[int] = None, B: Optional[int] = None, K: Optional[int] = None,
-         W: Optional[int] = None) -> Workload:
-    """Draw the named workload. ``S``/``B``/``K``/``W`` override the sizes
-    (same recipe and value distributions)."""
+         W: Optional[int] = None, H: Optional[int] = None, D: Optional[int] = None) -> Workload:
+    """Draw the named workload. ``S``/``B``/``K``/``W``/``H``/``D`` override the
+    sizes (same recipe and value distributions; H=128 is the V4-Pro head
+    count)."""
     sp = CONFIGS[name]
     B_ = B if B is not None else sp.B
     S_ = S if S is not None else sp.S
-    H, D, cr = sp.H, sp.D, sp.cr
+    H = sp.H if H is None else H
+    D = sp.D if D is None else D
+    cr = sp.cr
     K = sp.K if K is None else K
     W = sp.W if W is None else W
     assert K <= S_ // cr

@@ -74,6 +74,22 @@ def test_flash_recipe_ragged_tiles(sai):
     check_full(sai, workload("flash_s1024_k200", name="flash", S=1024, K=200))
 
 
+def test_pro_heads_h128(sai):
+    # V4-Pro head count: a window tile is one token, two score tiles per TMEM
+    # group, so 300 selected slots take two groups
+    check_full(sai, workload("pro_s1280_k300", name="flash", S=1280, K=300, H=128))
+
+
+def test_h32_d256(sai):
+    # four tokens per window tile, eight score tiles per TMEM group, D/64 = 4
+    check_full(sai, workload("h32_d256", name="flash", S=512, K=96, H=32, D=256))
+
+
+def test_h64_d128(sai):
+    # two 64-column chunks of D: one two-chunk window stage per tile
+    check_full(sai, workload("h64_d128", name="flash", S=512, K=100, D=128))
+
+
 def test_flash_recipe_odd_k(sai):
     """K not a multiple of 4: idx rows are read directly, not staged."""
     check_full(sai, synth.make("flash", S=512, K=101, seed=4242))
