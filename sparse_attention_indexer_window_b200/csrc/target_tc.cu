@@ -36,9 +36,10 @@
 //
 // The epilogue needs the per-head log-sum-exp over ALL selected slots before
 // it can form u, so a token's scores stay in TMEM until it is done: up to
-// 256/H tiles (512 slots at H=64) per accumulator. Two epilogue warpgroups
-// take alternate tokens, each with its own 256-column accumulator, so one
-// token's epilogue overlaps the next token's MMA. Tokens with more selected
+// 256/H tiles (512 slots at H=64) per accumulator. Tokens alternate between
+// two 256-column accumulators, so one token's epilogue overlaps the next
+// token's MMA; both epilogue warpgroups work on each token (half the tiles
+// each), which keeps the epilogue shorter than the MMAs of a token. Tokens with more selected
 // slots run in groups: a first pass over the groups merges per-head (max,
 // sum-exp) statistics, a second pass recomputes each group and forms u.
 //
@@ -54,7 +55,8 @@
 //
 // Warp roles (640 threads): warp 0 idx staging and compaction, warps 1..7
 // and 9 row gathers, warp 11 Q loads, warps 8 (also the TMEM owner) and 10
-// the two MMA issuers, warps 12..15 and 16..19 the two epilogue groups. Persistent CTAs walk tokens from the last
+// the two MMA issuers, warps 12..19 the epilogue (two warpgroups that split
+// each token's tiles). Persistent CTAs walk tokens from the last
 // (heaviest) to the first. All mbarrier waits are bounded; a timeout is
 // reported through err and the CTA unwinds. Named barriers are only used
 // where every participating thread is guaranteed to arrive.
@@ -94,13 +96,13 @@ constexpr float kLnOldFloor = -23.025850929940457f;      // log(1e-10), the per-
 
 template <int HH>
 struct EpiState {                 // one per epilogue warpgroup
-    float red_max[4][HH];
-    float red_sum[4][HH];
+    float red_max[8][HH];
+    float red_sum[8][HH];
     float colM[HH];
     float colS[HH];
     float head_a[HH];
     float wprime[HH];
-    float red_m[4];
+    float red_m[8];
     int flag;
 };
 
@@ -114,7 +116,7 @@ struct TgtSmem {
     uint32_t tmem_base;
     int abort_flag;
     int nsel[kMeta];
-    EpiState<HH> epi[2];
+    EpiState<HH> epi[1];
 };
 
 // Bytes of dynamic smem other than the A-stage ring.
@@ -139,7 +141,6 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
                      const TgtTcArgs a)
 {
     constexpr int TB = 256 / HH;                 // tiles per accumulator
-    constexpr int IB = TB < 2 ? TB : 2;          // tiles per TMEM load batch
     constexpr uint32_t kQTile = HH * 128;        // H rows x 128 bytes
     constexpr int NC16 = HH / 16;
 
@@ -155,8 +156,8 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
     uint32_t *rowoff = reinterpret_cast<uint32_t *>(q_buf + QS * kQTile);    // [kMeta][Kp]
     int32_t *slot = reinterpret_cast<int32_t *>(rowoff + kMeta * Kp);        // [kMeta][Kp]
     int32_t *idxs = slot + kMeta * Kp;                                       // [3][Kp] staged idx rows
-    float *ubuf = reinterpret_cast<float *>(idxs + 3 * Kp);                  // [2][Kp]
-    TgtSmem<HH> *sm = reinterpret_cast<TgtSmem<HH> *>(ubuf + 2 * Kp);
+    float *ubuf = reinterpret_cast<float *>(idxs + 3 * Kp);                  // [Kp] u' of a token
+    TgtSmem<HH> *sm = reinterpret_cast<TgtSmem<HH> *>(ubuf + Kp);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -174,7 +175,7 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&sm->acc_full[b], 2);     // both MMA threads commit a group
-            mbar_init(&sm->acc_empty[b], 4);
+            mbar_init(&sm->acc_empty[b], 8);    // lane 0 of each epilogue warp
         }
         for (int b = 0; b < kMeta; ++b) {
             mbar_init(&sm->meta_full[b], 1);
@@ -527,28 +528,38 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
     }
     } else {
         // ============================================================ epilogue
+        // Both epilogue warpgroups work on every token: warpgroup hf takes the
+        // tiles [hf*TBH, (hf+1)*TBH) of each TMEM group, so a token's scores
+        // are drained in about half the time of one warpgroup and the TMEM
+        // buffer returns to the MMA threads sooner. Per-head statistics are
+        // combined across the eight warps through shared memory.
         // warpgroups 3 and 4 execute this one setmaxnreg together
         regs_inc<kHighRegs>();
-        const int wg = (warp - kEpiWarp0) >> 2;  // epilogue group: tokens with it & 1 == wg
-        const int q = warp & 3;              // TMEM lane quarter
-        const int r = q * 32 + lane;         // row within a 128-slot tile
-        const int et = (warp - kEpiWarp0 - 4 * wg) * 32 + lane;  // 0..127 within the group
-        const uint32_t bar_id = 1 + wg;
-        EpiState<HH> &st = sm->epi[wg];
-        float *ub = ubuf + wg * Kp;
-        const float s2 = a.scale * kLog2e;   // scale > 0 (checked on the host)
+        constexpr int TBH = TB / 2;           // tiles per warpgroup and group
+        constexpr int IBH = TBH < 2 ? TBH : 2; // tiles per TMEM load batch
+        const int ew = warp - kEpiWarp0;      // 0..7
+        const int hf = ew >> 2;               // which half of the tiles
+        const int q = warp & 3;               // TMEM lane quarter
+        const int r = q * 32 + lane;          // row within a 128-slot tile
+        const int et = ew * 32 + lane;        // 0..255
+        constexpr uint32_t bar_id = 1;
+        constexpr int kEpiThreads = 256;
+        EpiState<HH> &st = sm->epi[0];
+        float *ub = ubuf;
+        const float s2 = a.scale * kLog2e;    // scale > 0 (checked on the host)
         const float sink_h = (a.sink && et < HH) ? a.sink[et] : -INFINITY;
-        int jobs = 0;
-        for (int it = wg; blockIdx.x + it * (int)gridDim.x < a.n_tok; it += 2) {
+        int jobs0 = 0, jobs1 = 0;
+        for (int it = 0; blockIdx.x + it * (int)gridDim.x < a.n_tok; ++it) {
             const int gt = blockIdx.x + it * gridDim.x;
             const int g = a.n_tok - 1 - gt;
             const int m3 = it % kMeta;
+            const int mb = it & 1;
             // window log-mass of this token's heads, fetched early
             const float wl_h = (et < HH && a.wl) ? a.wl[(size_t)g * HH + et] : 0.f;
-            // leader waits; the named barrier hands the outcome to the group
+            // leader waits; the named barrier hands the outcome to everyone
             if (et == 0)
                 st.flag = mbar_wait(&sm->meta_full[m3], (it / kMeta) & 1, abort_flag, a.err) ? 1 : 0;
-            named_bar_sync(bar_id, 128);
+            named_bar_sync(bar_id, kEpiThreads);
             if (!st.flag)
                 break;
             const int nsel = sm->nsel[m3];
@@ -557,7 +568,7 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
             const int passes = G > 1 ? 2 : 1;
             float *prow = a.p + (size_t)g * K;
             const int32_t *sl = slot + m3 * Kp;
-            const uint32_t tbase = tmem + wg * 256 + ((uint32_t)(q * 32) << 16);
+            const uint32_t tbase = tmem + mb * 256 + ((uint32_t)(q * 32) << 16);
             float m_part = 0.f;
             float At = 0.f;
             bool ok = true;
@@ -565,15 +576,23 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
                 for (int grp = 0; grp < G; ++grp) {
                     const int i0 = grp * TB;
                     const int ntg = min(nt, i0 + TB) - i0;
-                    named_bar_sync(bar_id, 128);   // st.flag is free again
-                    if (et == 0)
-                        st.flag = mbar_wait(&sm->acc_full[wg], jobs & 1, abort_flag, a.err) ? 1 : 0;
-                    named_bar_sync(bar_id, 128);
+                    // this warpgroup's tiles of the group: [t0, t1) (possibly empty)
+                    const int t0 = hf * TBH;
+                    const int t1 = min(ntg, t0 + TBH);
+                    named_bar_sync(bar_id, kEpiThreads);   // st.flag is free again
+                    if (et == 0) {
+                        const int jb = mb ? jobs1 : jobs0;
+                        st.flag = mbar_wait(&sm->acc_full[mb], jb & 1, abort_flag, a.err) ? 1 : 0;
+                    }
+                    named_bar_sync(bar_id, kEpiThreads);
+                    if (mb)
+                        ++jobs1;
+                    else
+                        ++jobs0;
                     if (!st.flag) {
                         ok = false;
                         break;
                     }
-                    ++jobs;
                     tc_fence_after();
                     const bool single = (G == 1);
                     if (pass == 0) {
@@ -583,16 +602,16 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
 #pragma unroll
                             for (int e = 0; e < 16; ++e)
                                 v16[e] = -INFINITY;
-                            for (int ib = 0; ib < ntg; ib += IB) {
-                                uint32_t v[IB][16];
+                            for (int ib = t0; ib < t1; ib += IBH) {
+                                uint32_t v[IBH][16];
 #pragma unroll
-                                for (int i = 0; i < IB; ++i)
-                                    if (ib + i < ntg)
+                                for (int i = 0; i < IBH; ++i)
+                                    if (ib + i < t1)
                                         tmem_ld16(tbase + (ib + i) * HH + cc * 16, v[i]);
                                 tmem_ld_wait();
 #pragma unroll
-                                for (int i = 0; i < IB; ++i) {
-                                    if (ib + i < ntg && (i0 + ib + i) * 128 + r < nsel) {
+                                for (int i = 0; i < IBH; ++i) {
+                                    if (ib + i < t1 && (i0 + ib + i) * 128 + r < nsel) {
 #pragma unroll
                                         for (int e = 0; e < 16; ++e)
                                             v16[e] = fmaxf(v16[e], __uint_as_float(v[i][e]));
@@ -601,13 +620,17 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
                             }
                             const float red = warp_colreduce16(v16, OpMax());
                             if (lane < 16)
-                                st.red_max[q][cc * 16 + lane] = red;
+                                st.red_max[ew][cc * 16 + lane] = red;
                         }
-                        named_bar_sync(bar_id, 128);
-                        if (et < HH)
-                            st.head_a[et] = fmaxf(fmaxf(st.red_max[0][et], st.red_max[1][et]),
-                                                  fmaxf(st.red_max[2][et], st.red_max[3][et])) * s2;
-                        named_bar_sync(bar_id, 128);
+                        named_bar_sync(bar_id, kEpiThreads);
+                        if (et < HH) {
+                            float mx = st.red_max[0][et];
+#pragma unroll
+                            for (int w = 1; w < 8; ++w)
+                                mx = fmaxf(mx, st.red_max[w][et]);
+                            st.head_a[et] = mx * s2;
+                        }
+                        named_bar_sync(bar_id, kEpiThreads);
                         // ---- e = 2^(v s2 - max s2), column sums; one group: keep e in TMEM
                         for (int cc = 0; cc < NC16; ++cc) {
                             float s16[16], m16[16];
@@ -616,16 +639,16 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
                                 s16[e] = 0.f;
                                 m16[e] = st.head_a[cc * 16 + e];
                             }
-                            for (int ib = 0; ib < ntg; ib += IB) {
-                                uint32_t v[IB][16];
+                            for (int ib = t0; ib < t1; ib += IBH) {
+                                uint32_t v[IBH][16];
 #pragma unroll
-                                for (int i = 0; i < IB; ++i)
-                                    if (ib + i < ntg)
+                                for (int i = 0; i < IBH; ++i)
+                                    if (ib + i < t1)
                                         tmem_ld16(tbase + (ib + i) * HH + cc * 16, v[i]);
                                 tmem_ld_wait();
 #pragma unroll
-                                for (int i = 0; i < IB; ++i) {
-                                    if (ib + i < ntg) {
+                                for (int i = 0; i < IBH; ++i) {
+                                    if (ib + i < t1) {
                                         if ((i0 + ib + i) * 128 + r < nsel) {
 #pragma unroll
                                             for (int e = 0; e < 16; ++e) {
@@ -643,23 +666,25 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
                                 }
                                 if (single) {
 #pragma unroll
-                                    for (int i = 0; i < IB; ++i)
-                                        if (ib + i < ntg)
+                                    for (int i = 0; i < IBH; ++i)
+                                        if (ib + i < t1)
                                             tmem_st16(tbase + (ib + i) * HH + cc * 16, v[i]);
                                 }
                             }
                             const float red = warp_colreduce16(s16, OpAdd());
                             if (lane < 16)
-                                st.red_sum[q][cc * 16 + lane] = red;
+                                st.red_sum[ew][cc * 16 + lane] = red;
                         }
                         if (single)
                             tmem_st_wait();
-                        named_bar_sync(bar_id, 128);
+                        named_bar_sync(bar_id, kEpiThreads);
                         if (et < HH) {
                             // group statistics in the log2 domain: max M2, sum S
                             const float gm = st.head_a[et];
-                            const float gs = st.red_sum[0][et] + st.red_sum[1][et] + st.red_sum[2][et] +
-                                             st.red_sum[3][et];
+                            float gs = 0.f;
+#pragma unroll
+                            for (int w = 0; w < 8; ++w)
+                                gs += st.red_sum[w][et];
                             if (grp == 0) {
                                 st.colM[et] = gm;
                                 st.colS[et] = gs;
@@ -670,7 +695,7 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
                                 st.colM[et] = M1;
                             }
                         }
-                        named_bar_sync(bar_id, 128);
+                        named_bar_sync(bar_id, kEpiThreads);
                     }
                     if (pass == passes - 1) {
                         if (grp == 0) {
@@ -689,7 +714,7 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
                                     st.head_a[et] = M - (mm + logf(acc));
                                 }
                             }
-                            named_bar_sync(bar_id, 128);
+                            named_bar_sync(bar_id, kEpiThreads);
                             float x = -INFINITY;
                             for (int h = lane; h < HH; h += 32)
                                 x = fmaxf(x, st.head_a[h]);
@@ -699,12 +724,12 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
                             At = x;
                             if (et < HH)
                                 st.wprime[et] = expf(st.head_a[et] - At);
-                            named_bar_sync(bar_id, 128);
+                            named_bar_sync(bar_id, kEpiThreads);
                         }
                         // ---- u'[k] = sum_h e[k,h] w[h]
-                        float u[TB];
+                        float u[TBH];
 #pragma unroll
-                        for (int i = 0; i < TB; ++i)
+                        for (int i = 0; i < TBH; ++i)
                             u[i] = 0.f;
                         for (int cc = 0; cc < NC16; ++cc) {
                             float w16[16];
@@ -712,18 +737,18 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
                             for (int e = 0; e < 16; ++e)
                                 w16[e] = st.wprime[cc * 16 + e];
 #pragma unroll
-                            for (int ib = 0; ib < TB; ib += IB) {
-                                if (ib >= ntg)
+                            for (int ib = 0; ib < TBH; ib += IBH) {
+                                if (t0 + ib >= t1)
                                     break;
-                                uint32_t v[IB][16];
+                                uint32_t v[IBH][16];
 #pragma unroll
-                                for (int i = 0; i < IB; ++i)
-                                    if (ib + i < ntg)
-                                        tmem_ld16(tbase + (ib + i) * HH + cc * 16, v[i]);
+                                for (int i = 0; i < IBH; ++i)
+                                    if (t0 + ib + i < t1)
+                                        tmem_ld16(tbase + (t0 + ib + i) * HH + cc * 16, v[i]);
                                 tmem_ld_wait();
 #pragma unroll
-                                for (int i = 0; i < IB; ++i) {
-                                    if (ib + i < ntg) {
+                                for (int i = 0; i < IBH; ++i) {
+                                    if (t0 + ib + i < t1) {
                                         float acc = u[ib + i];
                                         if (single) {
 #pragma unroll
@@ -742,9 +767,9 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
                             }
                         }
 #pragma unroll
-                        for (int i = 0; i < TB; ++i) {
-                            const int j = (i0 + i) * 128 + r;
-                            if (i < ntg && j < nsel) {
+                        for (int i = 0; i < TBH; ++i) {
+                            const int j = (i0 + t0 + i) * 128 + r;
+                            if (t0 + i < t1 && j < nsel) {
                                 ub[j] = u[i];
                                 m_part += u[i];
                             }
@@ -753,7 +778,7 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0)
-                        mbar_arrive(&sm->acc_empty[wg]);
+                        mbar_arrive(&sm->acc_empty[mb]);
                 }
             }
             if (!ok)
@@ -764,20 +789,23 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
             for (int o = 16; o >= 1; o >>= 1)
                 mt += __shfl_xor_sync(0xffffffffu, mt, o);
             if (lane == 0)
-                st.red_m[q] = mt;
-            named_bar_sync(bar_id, 128);
-            const float mtot = st.red_m[0] + st.red_m[1] + st.red_m[2] + st.red_m[3];
+                st.red_m[ew] = mt;
+            named_bar_sync(bar_id, kEpiThreads);
+            float mtot = 0.f;
+#pragma unroll
+            for (int w = 0; w < 8; ++w)
+                mtot += st.red_m[w];
             if (nsel > 0) {
                 const float ln_floor = a.per_branch ? kLnOldFloor : kLnFltMin;
                 const bool plain = logf(mtot) + At >= ln_floor;
                 const float f = plain ? 1.0f / mtot : expf(At - ln_floor);
-                for (int jj = et; jj < K; jj += 128)
+                for (int jj = et; jj < K; jj += kEpiThreads)
                     prow[sl[jj]] = (jj < nsel) ? ub[jj] * f : 0.f;
             } else {
-                for (int jj = et; jj < K; jj += 128)
+                for (int jj = et; jj < K; jj += kEpiThreads)
                     prow[jj] = 0.f;
             }
-            named_bar_sync(bar_id, 128);
+            named_bar_sync(bar_id, kEpiThreads);
             if (et == 0)
                 mbar_arrive(&sm->meta_empty[m3]);
         }
@@ -795,7 +823,7 @@ template <int HH>
 __host__ __device__ inline size_t fixed_smem_bytes(int K)
 {
     const size_t Kp = (size_t)((K + 3) & ~3);
-    return 1024 + q_stages<HH>() * (HH * 128) + Kp * 4 * (2 * kMeta + 5) + sizeof(TgtSmem<HH>) + 64;
+    return 1024 + q_stages<HH>() * (HH * 128) + Kp * 4 * (2 * kMeta + 4) + sizeof(TgtSmem<HH>) + 64;
 }
 
 // Deepest A-stage ring that fits the per-block smem limit (0 if none does).
