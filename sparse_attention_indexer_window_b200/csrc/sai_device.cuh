@@ -1,5 +1,5 @@
 // Device helpers for the sm_100a kernels: mbarriers with bounded waits, TMA
-// tile and gather4 loads, tcgen05 (TMEM allocation, MMA, loads/stores).
+// tile loads, tcgen05 (TMEM allocation, MMA, loads/stores).
 // Inline PTX only; no library code.
 #pragma once
 
@@ -80,20 +80,6 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *bar, uint32_t pari
     return ok != 0;
 }
 
-// Non-blocking test of the phase with the given parity.
-__device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity)
-{
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-
 // Wait for the phase with the given parity to complete. Gives up (returns
 // false) when the CTA's abort flag is raised or after kWaitLimitNs, in which
 // case it raises the abort flag and records kErrTimeout in *err (if any).
@@ -147,16 +133,6 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, u
         : "memory");
 }
 
-// 1-D bulk copy global -> smem (both 16-byte aligned, bytes % 16 == 0).
-__device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar)
-{
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-            smem_u32(dst)),
-        "l"(src), "r"(bytes), "r"(smem_u32(bar))
-        : "memory");
-}
-
 // 16-byte global -> smem copy through L2 (LSU path, not cached in L1).
 __device__ __forceinline__ void cp_async16(uint32_t dst_smem, const void *src)
 {
@@ -168,29 +144,11 @@ __device__ __forceinline__ void cp_async_wait()
 {
     asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
-// Arrive on an mbarrier once all prior cp.async copies of this thread have
-// landed (the arrival counts toward the barrier's expected count).
-__device__ __forceinline__ void cp_async_mbar_arrive_noinc(uint64_t *bar)
-{
-    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
 // Make this thread's generic-proxy smem writes visible to the async proxy
 // (tcgen05.mma operand reads).
 __device__ __forceinline__ void fence_proxy_async_smem()
 {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
-// Gather of four rows (r0..r3) of a 2-D map whose box is one row high; the
-// four rows land contiguously in smem, swizzled like a tiled load.
-__device__ __forceinline__ void tma_gather4(void *dst, const CUtensorMap *map, uint64_t *bar, int32_t x,
-                                            int32_t r0, int32_t r1, int32_t r2, int32_t r3)
-{
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(dst)),
-        "l"(map), "r"(smem_u32(bar)), "r"(x), "r"(r0), "r"(r1), "r"(r2), "r"(r3)
-        : "memory");
 }
 
 // ----------------------------------------------------------------- tcgen05
