@@ -52,7 +52,8 @@ def workload_config(w, n):
     return {
         "workload": f"{WORKLOAD}: B={w.B} S={w.S} H={w.H} D={w.D} cr={w.cr} K={w.K} W={w.W}, "
                     f"top-K of a random causal score, sorted ascending; bf16 Q/Kw/pool N(0,1), "
-                    f"fp32 sink N(0,1), scores N(0,2); seed 1003",
+                    f"fp32 sink N(0,1), scores N(0,2); "
+                    + ("seed 1003" if n == 1 else f"seeds 1003..{1003 + n - 1}, one batch per rank"),
         "global_batch": w.B * n,
         "seq_len": w.S,
         "parallelism": f"dp{n}" if n > 1 else "single",
@@ -145,9 +146,16 @@ class Clocks:
         except Exception:
             self.proc.kill()
         self.f.close()
+        with open(self.path) as f:
+            return self.parse(f)
+
+    @staticmethod
+    def parse(lines):
+        """Summary of nvidia-smi rows in the order of Q: median SM clock, max
+        clock, and every slowdown reason seen active in any sample."""
         sm, mx, reasons, n = [], None, set(), 0
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in open(self.path):
+        for line in lines:
             parts = [x.strip() for x in line.split(",")]
             if len(parts) < 9:
                 continue
@@ -383,7 +391,7 @@ def main():
             },
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "steps": args.e2e_steps},
-            "gpu_launches": 4 * nsteps,
+            "gpu_launches": 4 * nsteps * world,   # window, target, KL count, KL rows; every rank
             "clocks": clk,
             "loss": loss_all,
         }
