@@ -152,6 +152,38 @@ sai_status sai_distill_target_ex(const uint16_t *Q, const uint16_t *pool, const 
                                  int B, int S, int H, int D, int K, int cr, float scale, unsigned flags,
                                  float *p, int32_t *d_err, void *stream);
 
+/* Bytes of device workspace sai_distill_target_kl needs for these sizes. */
+size_t sai_distill_target_kl_workspace_bytes(int B, int S, int K);
+
+/*
+ * sai_distill_target_kl -- the target and the KL stage in one call.
+ *
+ * Computes what sai_distill_target_ex followed by sai_distill_kl computes.
+ * Where the tensor-core target kernel runs and K <= 512, the KL row, its
+ * gradient and the per-block KL sums come from the target kernel's epilogue
+ * while the row is still in shared memory, so p need not be written to or
+ * read back from device memory. This is the KL half of the single fused pass
+ * the Primus page describes (first commit message: the KL tail is fused and
+ * keeps no state between forward and backward). Before it, a small kernel
+ * counts the rows with a valid slot (N).
+ *
+ *   arguments as in sai_distill_target_ex and sai_distill_kl;
+ *   p          [B,S,K] fp32 target, written if not NULL. It may be NULL only
+ *              where the fused route applies (else SAI_ERR_UNSUPPORTED);
+ *   workspace  device scratch of sai_distill_target_kl_workspace_bytes(B,S,K)
+ *              bytes, 16-byte aligned, owned by the caller; no initialisation
+ *              needed; calls that share it must not overlap.
+ *
+ * Errors: as sai_distill_target_ex and sai_distill_kl (SAI_ERR_WORKSPACE for
+ * a short or misaligned workspace). The loss is deterministic run to run.
+ */
+sai_status sai_distill_target_kl(const uint16_t *Q, const uint16_t *pool, const int32_t *idx,
+                                 const float *window_lse, const float *sink, const int32_t *doc_start,
+                                 int B, int S, int H, int D, int K, int cr, float scale, unsigned flags,
+                                 const float *scores, const uint8_t *valid, float coeff,
+                                 float *p, float *loss, float *dscores,
+                                 void *workspace, size_t ws_bytes, int32_t *d_err, void *stream);
+
 /* Bytes of device workspace sai_distill_kl needs for these sizes. */
 size_t sai_distill_kl_workspace_bytes(int B, int S, int K);
 

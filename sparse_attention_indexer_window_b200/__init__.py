@@ -49,6 +49,11 @@ _lib.sai_distill_target_ex.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _
                                        _P, _P, _P]
 _lib.sai_distill_target_ex.restype = _I
 TARGET_PER_BRANCH = 1   # flag of sai_distill_target_ex: the earlier per-branch target
+_lib.sai_distill_target_kl_workspace_bytes.argtypes = [_I, _I, _I]
+_lib.sai_distill_target_kl_workspace_bytes.restype = ctypes.c_size_t
+_lib.sai_distill_target_kl.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, ctypes.c_uint,
+                                       _P, _P, _F, _P, _P, _P, _P, ctypes.c_size_t, _P, _P]
+_lib.sai_distill_target_kl.restype = _I
 _lib.sai_distill_kl_workspace_bytes.argtypes = [_I, _I, _I]
 _lib.sai_distill_kl_workspace_bytes.restype = ctypes.c_size_t
 _lib.sai_distill_kl.argtypes = [_P, _P, _P, _I, _I, _I, _F, _P, _P, _P, ctypes.c_size_t, _P]
@@ -167,6 +172,61 @@ def distill_target(Q: torch.Tensor, pool: torch.Tensor, idx: Optional[torch.Tens
                                     _ptr(out), _ptr(err), _stream(Q.device))
     _check(st, "sai_distill_target_ex")
     return out
+
+
+def target_kl_workspace_bytes(B: int, S: int, K: int) -> int:
+    return int(_lib.sai_distill_target_kl_workspace_bytes(B, S, K))
+
+
+def distill_target_kl(Q: torch.Tensor, pool: torch.Tensor, idx: Optional[torch.Tensor], wl: Optional[torch.Tensor],
+                      cr: int, scale: float, scores: torch.Tensor, valid: torch.Tensor, coeff: float,
+                      sink: Optional[torch.Tensor] = None, doc_start: Optional[torch.Tensor] = None,
+                      err: Optional[torch.Tensor] = None, p: Optional[torch.Tensor] = None,
+                      per_branch: bool = False, workspace: Optional[torch.Tensor] = None,
+                      loss: Optional[torch.Tensor] = None, dscores: Optional[torch.Tensor] = None
+                      ) -> Tuple[torch.Tensor, torch.Tensor]:
+    """(loss, dscores) through sai_distill_target_kl: the target and the KL
+    stage in one call. p (optional [B,S,K] fp32 output) receives the target
+    when given; without it the target never leaves the GPU's on-chip memory
+    where the fused route applies."""
+    B, S, H, D = Q.shape
+    K = idx.shape[-1] if idx is not None else S // cr
+    Q = _bf16_bits(Q, "Q")
+    pool = _bf16_bits(pool, "pool")
+    if tuple(pool.shape) != (B, S // cr, D):
+        raise ValueError("pool must be [B,S/cr,D]")
+    _want(idx, "idx", torch.int32, (B, S, K))
+    if per_branch:
+        wl, sink = None, None
+    elif wl is None:
+        raise ValueError("window_lse is required unless per_branch")
+    _want(wl, "window_lse", torch.float32, (B, S, H))
+    if sink is not None:
+        if sink.numel() != H:
+            raise ValueError(f"sink needs one logit per head: expected {H} values, found {sink.numel()}")
+        _want(sink, "sink", torch.float32)
+    _want(doc_start, "doc_start", torch.int32, (B, S))
+    _want(err, "err", torch.int32)
+    _want(scores, "scores", torch.float32, (B, S, K))
+    if valid.dtype == torch.bool:
+        valid = valid.view(torch.uint8)
+    _want(valid, "valid", torch.uint8, (B, S, K))
+    _want(p, "p", torch.float32, (B, S, K))
+    need = target_kl_workspace_bytes(B, S, K)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=Q.device)
+    if loss is None:
+        loss = torch.empty(1, dtype=torch.float32, device=Q.device)
+    if dscores is None:
+        dscores = torch.empty((B, S, K), dtype=torch.float32, device=Q.device)
+    _want(dscores, "dscores", torch.float32, (B, S, K))
+    st = _lib.sai_distill_target_kl(_ptr(Q), _ptr(pool), _ptr(idx), _ptr(wl), _ptr(sink), _ptr(doc_start),
+                                    B, S, H, D, K, int(cr), float(scale), TARGET_PER_BRANCH if per_branch else 0,
+                                    _ptr(scores), _ptr(valid), float(coeff), _ptr(p), _ptr(loss), _ptr(dscores),
+                                    _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(err),
+                                    _stream(Q.device))
+    _check(st, "sai_distill_target_kl")
+    return loss, dscores
 
 
 def kl_workspace_bytes(B: int, S: int, K: int) -> int:

@@ -308,6 +308,12 @@ KlPlan kl_plan(int B, int S, int K)
     return pl;
 }
 
+cudaError_t launch_kl_count(const KlPlan &pl, const uint8_t *valid, void *ws, cudaStream_t stream)
+{
+    kl_count_kernel<<<pl.count_blocks, kKlThreads, 0, stream>>>(valid, pl.rows, pl.K, ws, pl.count_blocks);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_distill_kl(const KlPlan &pl, const float *p, const float *scores, const uint8_t *valid,
                               float coeff, float *loss, float *dscores, void *ws, cudaStream_t stream)
 {

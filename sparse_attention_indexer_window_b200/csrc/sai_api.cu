@@ -150,10 +150,33 @@ sai_status sai_distill_target(const uint16_t *Q, const uint16_t *pool, const int
                                  stream);
 }
 
-sai_status sai_distill_target_ex(const uint16_t *Q, const uint16_t *pool, const int32_t *idx,
-                                 const float *window_lse, const float *sink, const int32_t *doc_start, int B, int S,
-                                 int H, int D, int K, int cr, float scale, unsigned flags, float *p, int32_t *d_err,
-                                 void *stream)
+namespace {
+
+// Fused KL arguments of sai_distill_target_kl (NULL: target only).
+struct KlFuse {
+    const float *scores;
+    const uint8_t *valid;
+    float coeff;
+    float *loss;
+    float *dscores;
+    void *ws;
+    sai::KlPlan plan;
+};
+
+// Workspace of sai_distill_target_kl: the KL workspace (completion counter,
+// per-block valid-row counts, per-block KL sums) with room for one KL sum per
+// CTA of the target kernel (at most kMaxTargetCtas).
+constexpr int kMaxTargetCtas = 1024;
+size_t fused_ws_bytes(const sai::KlPlan &pl)
+{
+    const size_t a = 16 + (((size_t)pl.count_blocks * 4 + 15) & ~size_t(15));
+    const size_t parts = (size_t)(pl.row_blocks > kMaxTargetCtas ? pl.row_blocks : kMaxTargetCtas) * 8;
+    return a + parts;
+}
+
+sai_status target_impl(const uint16_t *Q, const uint16_t *pool, const int32_t *idx, const float *window_lse,
+                       const float *sink, const int32_t *doc_start, int B, int S, int H, int D, int K, int cr,
+                       float scale, unsigned flags, float *p, int32_t *d_err, cudaStream_t st, const KlFuse *kf)
 {
     if (flags & ~SAI_TARGET_PER_BRANCH)
         return SAI_ERR_UNSUPPORTED;
@@ -162,7 +185,8 @@ sai_status sai_distill_target_ex(const uint16_t *Q, const uint16_t *pool, const 
         window_lse = nullptr;   // not read in this mode
         sink = nullptr;
     }
-    if (!Q || !pool || (!window_lse && !per_branch) || !p)     // idx NULL: dense over all blocks
+    // idx NULL: dense over all blocks; p may be NULL only when the KL is fused
+    if (!Q || !pool || (!window_lse && !per_branch) || (!p && !kf))
         return SAI_ERR_NULL;
     if (B < 1 || S < 1 || H < 1 || D < 1 || K < 1 || cr < 1 || (D % 8) != 0 || (S % cr) != 0 ||
         !isfinite(scale) || scale <= 0.f)
@@ -172,15 +196,18 @@ sai_status sai_distill_target_ex(const uint16_t *Q, const uint16_t *pool, const 
         return SAI_ERR_SHAPE;
     if ((int64_t)B * S * H * D > INT32_MAX || (int64_t)B * S * K > INT32_MAX)
         return SAI_ERR_SHAPE;
-    if (!al16(Q) || !al16(pool) || (idx && !al4(idx)) || (window_lse && !al4(window_lse)) || !al4(p) ||
+    if (!al16(Q) || !al16(pool) || (idx && !al4(idx)) || (window_lse && !al4(window_lse)) || (p && !al4(p)) ||
         (sink && !al4(sink)) || (doc_start && !al4(doc_start)) || (d_err && !al4(d_err)))
         return SAI_ERR_ALIGN;
-    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const int smem_cap = max_smem_optin();
 
     // the tensor-core kernel addresses pool rows with 32-bit byte offsets
     const bool pool_fits = (uint64_t)B * P * D * 2 < 0xffffffffull;
     const int n_astages = tc_heads(H) && (D % 64) == 0 && pool_fits ? sai::target_tc_stages(H, K, smem_cap) : 0;
+    // the epilogue computes the KL from two slots per thread (K <= 512)
+    const bool fuse_here = kf && n_astages > 0 && K <= 512;
+    if (kf && !fuse_here && !p)
+        return SAI_ERR_UNSUPPORTED;   // the unfused route needs p to pass the target on
     if (n_astages > 0) {
         sai::TgtTcArgs a;
         a.B = B;
@@ -204,6 +231,15 @@ sai_status sai_distill_target_ex(const uint16_t *Q, const uint16_t *pool, const 
         a.doc_start = doc_start;
         a.p = p;
         a.err = d_err;
+        a.kl_scores = nullptr;
+        a.kl_valid = nullptr;
+        a.kl_dscores = nullptr;
+        a.kl_loss = nullptr;
+        a.kl_coeff = 0.f;
+        a.kl_count_part = nullptr;
+        a.kl_count_blocks = 0;
+        a.kl_part = nullptr;
+        a.kl_done = nullptr;
         CUtensorMap mq, mp;
         if (!make_map_bf16(&mq, Q, (uint64_t)B * S * H, D, (uint32_t)H) ||
             !make_map_bf16(&mp, pool, (uint64_t)B * P, D, (uint32_t)a.pool_box_rows))
@@ -213,14 +249,83 @@ sai_status sai_distill_target_ex(const uint16_t *Q, const uint16_t *pool, const 
             return SAI_ERR_CUDA;
         if (grid > a.n_tok)
             grid = a.n_tok;
-        return cuda_status(sai::launch_target_tc(mq, mp, a, grid, st));
+        if (grid > kMaxTargetCtas)
+            grid = kMaxTargetCtas;
+        if (fuse_here) {
+            // N first: per-block valid-row counts (this also zeroes the counter)
+            sai_status e = cuda_status(sai::launch_kl_count(kf->plan, kf->valid, kf->ws, st));
+            if (e != SAI_OK)
+                return e;
+            uint8_t *w = reinterpret_cast<uint8_t *>(kf->ws);
+            a.kl_scores = kf->scores;
+            a.kl_valid = kf->valid;
+            a.kl_dscores = kf->dscores;
+            a.kl_loss = kf->loss;
+            a.kl_coeff = kf->coeff;
+            a.kl_done = reinterpret_cast<uint32_t *>(w);
+            a.kl_count_part = reinterpret_cast<const int32_t *>(w + 16);
+            a.kl_count_blocks = kf->plan.count_blocks;
+            a.kl_part = reinterpret_cast<double *>(w + 16 + (((size_t)kf->plan.count_blocks * 4 + 15) & ~size_t(15)));
+        }
+        sai_status e = cuda_status(sai::launch_target_tc(mq, mp, a, grid, st));
+        if (e != SAI_OK || fuse_here || !kf)
+            return e;
+    } else if ((int)sai::target_simt_smem_bytes(H, D, K) <= smem_cap) {
+        sai_status e = cuda_status(sai::launch_target_simt(Q, pool, idx, window_lse, sink, doc_start, B, S, H, D, K,
+                                                           cr, scale, per_branch ? 1 : 0, p, d_err, st));
+        if (e != SAI_OK || !kf)
+            return e;
+    } else {
+        return SAI_ERR_UNSUPPORTED;
     }
-    if ((int)sai::target_simt_smem_bytes(H, D, K) <= smem_cap)
-        return cuda_status(sai::launch_target_simt(Q, pool, idx, window_lse, sink, doc_start, B, S, H, D, K, cr,
-                                                   scale, per_branch ? 1 : 0, p, d_err, st));
-    return SAI_ERR_UNSUPPORTED;
+    // the KL as its own pass over the target just written to p
+    return cuda_status(sai::launch_distill_kl(kf->plan, p, kf->scores, kf->valid, kf->coeff, kf->loss, kf->dscores,
+                                              kf->ws, st));
 }
 
+}  // namespace
+
+sai_status sai_distill_target_ex(const uint16_t *Q, const uint16_t *pool, const int32_t *idx,
+                                 const float *window_lse, const float *sink, const int32_t *doc_start, int B, int S,
+                                 int H, int D, int K, int cr, float scale, unsigned flags, float *p, int32_t *d_err,
+                                 void *stream)
+{
+    return target_impl(Q, pool, idx, window_lse, sink, doc_start, B, S, H, D, K, cr, scale, flags, p, d_err,
+                       reinterpret_cast<cudaStream_t>(stream), nullptr);
+}
+
+size_t sai_distill_target_kl_workspace_bytes(int B, int S, int K)
+{
+    if (B < 1 || S < 1 || K < 1)
+        return 0;
+    return fused_ws_bytes(sai::kl_plan(B, S, K));
+}
+
+sai_status sai_distill_target_kl(const uint16_t *Q, const uint16_t *pool, const int32_t *idx,
+                                 const float *window_lse, const float *sink, const int32_t *doc_start, int B, int S,
+                                 int H, int D, int K, int cr, float scale, unsigned flags, const float *scores,
+                                 const uint8_t *valid, float coeff, float *p, float *loss, float *dscores,
+                                 void *workspace, size_t ws_bytes, int32_t *d_err, void *stream)
+{
+    if (!scores || !valid || !loss || !dscores)
+        return SAI_ERR_NULL;
+    if (B < 1 || S < 1 || K < 1 || !isfinite(coeff))
+        return SAI_ERR_SHAPE;
+    if (!al16(scores) || !al16(valid) || !al4(loss) || !al16(dscores))
+        return SAI_ERR_ALIGN;
+    KlFuse kf;
+    kf.scores = scores;
+    kf.valid = valid;
+    kf.coeff = coeff;
+    kf.loss = loss;
+    kf.dscores = dscores;
+    kf.ws = workspace;
+    kf.plan = sai::kl_plan(B, S, K);
+    if (!workspace || !al16(workspace) || ws_bytes < fused_ws_bytes(kf.plan))
+        return SAI_ERR_WORKSPACE;
+    return target_impl(Q, pool, idx, window_lse, sink, doc_start, B, S, H, D, K, cr, scale, flags, p, d_err,
+                       reinterpret_cast<cudaStream_t>(stream), &kf);
+}
 size_t sai_distill_kl_workspace_bytes(int B, int S, int K)
 {
     if (B < 1 || S < 1 || K < 1)

@@ -39,8 +39,19 @@ struct TgtTcArgs {
     const float *wl;
     const float *sink;
     const int32_t *doc_start;
-    float *p;
+    float *p;             // may be NULL when the KL is fused (kl_scores set)
     int32_t *err;
+    // KL fused into the epilogue (kl_scores NULL: not fused). N comes from the
+    // per-block valid-row counts of kl_count_kernel, run before on the stream.
+    const float *kl_scores;     // [n_tok, K]
+    const uint8_t *kl_valid;    // [n_tok, K]
+    float *kl_dscores;          // [n_tok, K]
+    float *kl_loss;             // device scalar
+    float kl_coeff;
+    const int32_t *kl_count_part;
+    int kl_count_blocks;
+    double *kl_part;            // [grid] per-CTA KL sums
+    uint32_t *kl_done;          // completion counter, zeroed by kl_count_kernel
 };
 // Deepest gathered-row stage ring that fits `smem_limit` bytes (0: none).
 int target_tc_stages(int H, int K, int smem_limit);
@@ -66,6 +77,9 @@ struct KlPlan {
     size_t ws_bytes;
 };
 KlPlan kl_plan(int B, int S, int K);
+// Per-block counts of rows with a valid slot into the KL workspace (its
+// layout: completion counter at byte 0, which this resets, counts at byte 16).
+cudaError_t launch_kl_count(const KlPlan &pl, const uint8_t *valid, void *ws, cudaStream_t stream);
 cudaError_t launch_distill_kl(const KlPlan &pl, const float *p, const float *scores, const uint8_t *valid,
                               float coeff, float *loss, float *dscores, void *ws, cudaStream_t stream);
 

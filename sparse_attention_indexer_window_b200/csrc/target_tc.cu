@@ -103,6 +103,7 @@ struct EpiState {                 // one per epilogue warpgroup
     float head_a[HH];
     float wprime[HH];
     float red_m[8];
+    float klred[8][3];   // fused KL: per-warp partials of the row reductions
     int flag;
 };
 
@@ -549,6 +550,28 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
         const float s2 = a.scale * kLog2e;    // scale > 0 (checked on the host)
         const float sink_h = (a.sink && et < HH) ? a.sink[et] : -INFINITY;
         int jobs0 = 0, jobs1 = 0;
+        // fused KL: the global count N of rows with a valid slot, and this
+        // CTA's running KL sum (thread et == 0, fixed token order)
+        const bool kl = a.kl_scores != nullptr;
+        float kl_c = 0.f;
+        int kl_n = 0;
+        double kl_acc = 0.0;
+        if (kl) {
+            int n = 0;
+            for (int i = et; i < a.kl_count_blocks; i += kEpiThreads)
+                n += a.kl_count_part[i];
+#pragma unroll
+            for (int o = 16; o >= 1; o >>= 1)
+                n += __shfl_xor_sync(0xffffffffu, n, o);
+            if (lane == 0)
+                st.red_m[ew] = __int_as_float(n);
+            named_bar_sync(bar_id, kEpiThreads);
+#pragma unroll
+            for (int w = 0; w < 8; ++w)
+                kl_n += __float_as_int(st.red_m[w]);
+            kl_c = a.kl_coeff / (float)(kl_n > 1 ? kl_n : 1);
+            named_bar_sync(bar_id, kEpiThreads);
+        }
         for (int it = 0; blockIdx.x + it * (int)gridDim.x < a.n_tok; ++it) {
             const int gt = blockIdx.x + it * gridDim.x;
             const int g = a.n_tok - 1 - gt;
@@ -569,6 +592,21 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
             float *prow = a.p + (size_t)g * K;
             const int32_t *sl = slot + m3 * Kp;
             const uint32_t tbase = tmem + mb * 256 + ((uint32_t)(q * 32) << 16);
+            // fused KL: this thread's scores and valid flags (slots et, et+256),
+            // loaded now so the latency is hidden behind the token's MMAs
+            constexpr int kKlReg = 2;
+            float kl_s[kKlReg];
+            uint8_t kl_v[kKlReg];
+            if (kl) {
+#pragma unroll
+                for (int i = 0; i < kKlReg; ++i) {
+                    const int jj = et + i * kEpiThreads;
+                    const bool in = jj < K;
+                    const size_t gi = (size_t)g * K + (in ? sl[jj] : 0);
+                    kl_s[i] = in ? a.kl_scores[gi] : 0.f;
+                    kl_v[i] = in ? a.kl_valid[gi] : 0;
+                }
+            }
             float m_part = 0.f;
             float At = 0.f;
             bool ok = true;
@@ -795,19 +833,120 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
 #pragma unroll
             for (int w = 0; w < 8; ++w)
                 mtot += st.red_m[w];
+            float f = 0.f;
             if (nsel > 0) {
                 const float ln_floor = a.per_branch ? kLnOldFloor : kLnFltMin;
                 const bool plain = logf(mtot) + At >= ln_floor;
-                const float f = plain ? 1.0f / mtot : expf(At - ln_floor);
+                f = plain ? 1.0f / mtot : expf(At - ln_floor);
+            }
+            if (a.p) {
                 for (int jj = et; jj < K; jj += kEpiThreads)
                     prow[sl[jj]] = (jj < nsel) ? ub[jj] * f : 0.f;
-            } else {
-                for (int jj = et; jj < K; jj += kEpiThreads)
-                    prow[jj] = 0.f;
+            }
+            if (kl) {
+                // ---- KL(p || softmax(scores)) over the row's valid slots and
+                // its gradient, straight from the target in shared memory
+                // (K <= 2 * 256 here: two slots per thread, in registers)
+                const size_t rowo = (size_t)g * K;
+                float pv[kKlReg];
+                int kk[kKlReg];
+                float mx = -INFINITY;
+                bool anyv = false;
+#pragma unroll
+                for (int i = 0; i < kKlReg; ++i) {
+                    const int jj = et + i * kEpiThreads;
+                    kk[i] = jj < K ? sl[jj] : 0;
+                    pv[i] = (jj < nsel) ? ub[jj] * f : 0.f;
+                    if (kl_v[i]) {
+                        mx = fmaxf(mx, kl_s[i]);
+                        anyv = true;
+                    }
+                }
+#pragma unroll
+                for (int o = 16; o >= 1; o >>= 1)
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+                const bool wany = __any_sync(0xffffffffu, anyv);
+                if (lane == 0) {
+                    st.klred[ew][0] = mx;
+                    st.klred[ew][1] = wany ? 1.f : 0.f;
+                }
+                named_bar_sync(bar_id, kEpiThreads);
+                float rmx = -INFINITY;
+                bool rany = false;
+#pragma unroll
+                for (int w = 0; w < 8; ++w) {
+                    rmx = fmaxf(rmx, st.klred[w][0]);
+                    rany = rany || st.klred[w][1] != 0.f;
+                }
+                named_bar_sync(bar_id, kEpiThreads);
+                float se = 0.f, ps = 0.f;
+#pragma unroll
+                for (int i = 0; i < kKlReg; ++i) {
+                    if (kl_v[i]) {
+                        se += __expf(kl_s[i] - rmx);
+                        ps += pv[i];
+                    }
+                }
+#pragma unroll
+                for (int o = 16; o >= 1; o >>= 1) {
+                    se += __shfl_xor_sync(0xffffffffu, se, o);
+                    ps += __shfl_xor_sync(0xffffffffu, ps, o);
+                }
+                if (lane == 0) {
+                    st.klred[ew][0] = se;
+                    st.klred[ew][1] = ps;
+                }
+                named_bar_sync(bar_id, kEpiThreads);
+                float rse = 0.f, rps = 0.f;
+#pragma unroll
+                for (int w = 0; w < 8; ++w) {
+                    rse += st.klred[w][0];
+                    rps += st.klred[w][1];
+                }
+                const float lse = rany ? rmx + __logf(rse) : 0.f;
+                float klv = 0.f;
+#pragma unroll
+                for (int i = 0; i < kKlReg; ++i) {
+                    const int jj = et + i * kEpiThreads;
+                    if (jj < K) {
+                        const bool v = rany && kl_v[i];
+                        const float logq = kl_s[i] - lse;
+                        if (v && pv[i] > 0.f)
+                            klv += pv[i] * (__logf(pv[i]) - logq);
+                        a.kl_dscores[rowo + kk[i]] = v ? kl_c * fmaf(__expf(logq), rps, -pv[i]) : 0.f;
+                    }
+                }
+#pragma unroll
+                for (int o = 16; o >= 1; o >>= 1)
+                    klv += __shfl_xor_sync(0xffffffffu, klv, o);
+                named_bar_sync(bar_id, kEpiThreads);   // klred[.][0..1] read by all before reuse
+                if (lane == 0)
+                    st.klred[ew][2] = klv;
+                named_bar_sync(bar_id, kEpiThreads);
+                if (et == 0) {
+                    float tk = 0.f;
+#pragma unroll
+                    for (int w = 0; w < 8; ++w)
+                        tk += st.klred[w][2];
+                    kl_acc += (double)tk;
+                }
             }
             named_bar_sync(bar_id, kEpiThreads);
             if (et == 0)
                 mbar_arrive(&sm->meta_empty[m3]);
+        }
+        if (kl && et == 0) {
+            // this CTA's KL sum; the last CTA to finish adds them in CTA order
+            a.kl_part[blockIdx.x] = kl_acc;
+            __threadfence();
+            if (atomicAdd(a.kl_done, 1u) == gridDim.x - 1) {
+                __threadfence();
+                const volatile double *kp = a.kl_part;
+                double tot = 0.0;
+                for (int i = 0; i < (int)gridDim.x; ++i)
+                    tot += kp[i];
+                *a.kl_loss = (float)((double)a.kl_coeff * tot / (double)(kl_n > 1 ? kl_n : 1));
+            }
         }
     }
 

@@ -89,6 +89,22 @@ def test_distill_target_ex_host_errors(sai):
     assert f(*args(FAKE, 1)[:6], 1, 64, 4, 32, 8, 3, 0.1, 1, FAKE, None, None) == 2   # S % cr, per-branch
 
 
+def test_distill_target_kl_host_errors(sai):
+    """The fused target + KL call refuses missing KL buffers and a short or
+    misaligned workspace before launching anything."""
+    lib = sai.lib()
+    f = lib.sai_distill_target_kl
+    need = lib.sai_distill_target_kl_workspace_bytes(1, 64, 8)
+    assert need > lib.sai_distill_kl_workspace_bytes(1, 64, 8)
+    head = (FAKE, FAKE, FAKE, FAKE, None, None, 1, 64, 4, 32, 8, 4, 0.1, 0)
+    assert f(*head, None, FAKE, 0.01, None, FAKE, FAKE, FAKE, need, None, None) == 1    # no scores
+    assert f(*head, FAKE, FAKE, 0.01, None, FAKE, None, FAKE, need, None, None) == 1    # no dscores
+    assert f(*head, FAKE, FAKE, 0.01, None, FAKE, FAKE, FAKE, need - 1, None, None) == 6
+    assert f(*head, FAKE, FAKE, 0.01, None, FAKE, FAKE, FAKE_MIS, need, None, None) == 6
+    assert f(*head, FAKE_MIS, FAKE, 0.01, None, FAKE, FAKE, FAKE, need, None, None) == 7
+    assert f(*head[:13], 2, FAKE, FAKE, 0.01, None, FAKE, FAKE, FAKE, need, None, None) == 3   # bad flag
+
+
 def test_distill_kl_host_errors(sai):
     f = sai.lib().sai_distill_kl
     need = sai.lib().sai_distill_kl_workspace_bytes(1, 64, 8)
