@@ -20,8 +20,8 @@
 // Gather. A dedicated warp compacts each token's idx row (selected slots
 // first, masked slots last), up to two tokens ahead; the idx rows arrive by
 // its own cp.async copies, and the compaction turns pool rows into byte
-// offsets. Eight
-// gather warps each own one 16 KB slot of the A ring and fill every stage
+// offsets. Eight gather warps each own one 16 KB slot of the A ring and fill
+// every stage
 // that lands in it: 128 selected rows x one 128-byte chunk of D, copied into
 // the swizzled K-major operand layout with 16-byte cp.async (eight lanes per
 // row, four rows per instruction, every 128-byte row segment one coalesced
@@ -39,9 +39,11 @@
 // 256/H tiles (512 slots at H=64) per accumulator. Tokens alternate between
 // two 256-column accumulators, so one token's epilogue overlaps the next
 // token's MMA; both epilogue warpgroups work on each token (half the tiles
-// each), which keeps the epilogue shorter than the MMAs of a token. Tokens with more selected
-// slots run in groups: a first pass over the groups merges per-head (max,
-// sum-exp) statistics, a second pass recomputes each group and forms u.
+// each), which keeps the epilogue shorter than the MMAs of a token. Tokens
+// with more selected slots run in groups: a first pass over the groups merges
+// per-head (max, sum-exp) statistics, a second pass recomputes each group and
+// forms u. When the KL stage is fused (sai_distill_target_kl), the epilogue
+// then computes each row's KL and dscores from the target in shared memory.
 //
 // Epilogue arithmetic (one exponential per score):
 //   M[h] = max_k z[k,h]  (column max: transposing warp butterfly + smem)
@@ -52,6 +54,8 @@
 //   p[k] = u'[k]/m'                     if log m' + A >= log FLT_MIN
 //        = u'[k] exp(A - log FLT_MIN)   otherwise (the float32-tiny floor),
 // so no intermediate is subnormal however small each head's compressed share.
+// The per-branch target (SAI_TARGET_PER_BRANCH) takes a[h] = M[h] - clse[h]
+// and the floor 1e-10.
 //
 // Warp roles (640 threads): warp 0 idx staging and compaction, warps 1..7
 // and 9 row gathers, warp 11 Q loads, warps 8 (also the TMEM owner) and 10
