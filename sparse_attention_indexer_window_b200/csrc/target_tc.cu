@@ -140,7 +140,9 @@ __device__ __forceinline__ bool selected(int j, int t, int d0, int P, int cr)
     return j >= 0 && j < P && (j + 1) * cr - 1 <= t && j * cr >= d0;
 }
 
-template <int HH>
+// FUSE_KL: the epilogue also computes the KL stage (sai_distill_target_kl);
+// a separate instantiation, so the plain target kernel carries none of it.
+template <int HH, bool FUSE_KL>
 __global__ void __launch_bounds__(kTgtThreads, 1)
     target_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapP,
                      const TgtTcArgs a)
@@ -556,7 +558,7 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
         int jobs0 = 0, jobs1 = 0;
         // fused KL: the global count N of rows with a valid slot, and this
         // CTA's running KL sum (thread et == 0, fixed token order)
-        const bool kl = a.kl_scores != nullptr;
+        const bool kl = FUSE_KL;
         float kl_c = 0.f;
         int kl_n = 0;
         double kl_acc = 0.0;
@@ -986,24 +988,32 @@ size_t smem_bytes_for(int K, int stages)
     return fixed_smem_bytes<HH>(K) + (size_t)stages * kATile;
 }
 
-template <int HH>
-cudaError_t launch_h(const CUtensorMap &mapQ, const CUtensorMap &mapP, const TgtTcArgs &a, int grid,
-                     cudaStream_t stream)
+template <int HH, bool FUSE_KL>
+cudaError_t launch_hk(const CUtensorMap &mapQ, const CUtensorMap &mapP, const TgtTcArgs &a, int grid,
+                      cudaStream_t stream)
 {
     // The register split above is only safe if every thread was launched with
     // exactly kLaunchRegs registers; refuse to launch otherwise.
     cudaFuncAttributes fa;
-    cudaError_t e = cudaFuncGetAttributes(&fa, target_tc_kernel<HH>);
+    cudaError_t e = cudaFuncGetAttributes(&fa, target_tc_kernel<HH, FUSE_KL>);
     if (e != cudaSuccess)
         return e;
     if (fa.numRegs != kLaunchRegs)
         return cudaErrorInvalidConfiguration;
     const size_t smem = smem_bytes_for<HH>(a.K, a.n_astages);
-    e = cudaFuncSetAttribute(target_tc_kernel<HH>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    e = cudaFuncSetAttribute(target_tc_kernel<HH, FUSE_KL>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess)
         return e;
-    target_tc_kernel<HH><<<grid, kTgtThreads, smem, stream>>>(mapQ, mapP, a);
+    target_tc_kernel<HH, FUSE_KL><<<grid, kTgtThreads, smem, stream>>>(mapQ, mapP, a);
     return cudaGetLastError();
+}
+
+template <int HH>
+cudaError_t launch_h(const CUtensorMap &mapQ, const CUtensorMap &mapP, const TgtTcArgs &a, int grid,
+                     cudaStream_t stream)
+{
+    return a.kl_scores ? launch_hk<HH, true>(mapQ, mapP, a, grid, stream)
+                       : launch_hk<HH, false>(mapQ, mapP, a, grid, stream);
 }
 
 }  // namespace
