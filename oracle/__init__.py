@@ -84,13 +84,16 @@ def window_lse(Q, Kw, doc_start, W: int, scale: float, tokens=None) -> np.ndarra
 
 
 def distill_target(Q, pool, idx, wl, sink, doc_start, cr: int, scale: float, tokens=None,
-                   per_branch: bool = False):
+                   per_branch: bool = False, full_lse: bool = False):
     """(p [n, K] fp64, bad_index_count) for the flat token ids in ``tokens``.
 
     per_branch selects the earlier per-branch target (every head normalised
     over the selected entries alone, floor 1e-10); wl and sink are then
-    unused and may be None. idx=None is the dense warm-up stage: slot k is
-    compressed block k for every token (K = S/cr)."""
+    unused and may be None. full_lse says that wl already holds lse_full,
+    the per-head log-normaliser of the whole attention row (window, selected
+    entries and sink) as a CSA attention forward returns it; sink is then
+    unused. idx=None is the dense warm-up stage: slot k is compressed block k
+    for every token (K = S/cr)."""
     B, S, H, D = Q.shape
     if idx is None:
         idx = np.broadcast_to(np.arange(S // cr, dtype=np.int32), (B, S, S // cr))
@@ -98,14 +101,17 @@ def distill_target(Q, pool, idx, wl, sink, doc_start, cr: int, scale: float, tok
     Q = _c(Q, np.uint16); pool = _c(pool, np.uint16); idx = _c(idx, np.int32)
     wl = _c(wl, np.float64); sink = _c(sink, np.float32); ds = _c(doc_start, np.int32)
     tk, n = _tokens(tokens, B, S)
+    assert not (per_branch and full_lse)
+    mode = 1 if per_branch else (2 if full_lse else 0)
     if per_branch:
         wl = None
-        sink = None
     else:
         assert wl.shape == (n, H)
+    if per_branch or full_lse:
+        sink = None
     p = np.empty((n, K), dtype=np.float64)
     bad = _load().orc_distill_target(_ptr(Q), _ptr(pool), _ptr(idx), _ptr(wl), _ptr(sink), _ptr(ds),
-                                     B, S, H, D, K, cr, float(scale), _ptr(tk), n, 1 if per_branch else 0,
+                                     B, S, H, D, K, cr, float(scale), _ptr(tk), n, mode,
                                      _ptr(p))
     return p, int(bad)
 

@@ -10,6 +10,8 @@
  *   [P1] "perf(deepseek-v4): fuse and enable the indexer distillation loss"
  *        (Primus pull request 992): commit messages, "Summary",
  *        "Why the target was wrong", "Test plan".
+ *   [P2] "Docker Build for DeepSeek-v4 (Don't Merge)" (Primus pull request
+ *        862): the gluon_v3 commit message, "Optimization Notes", "Forward".
  *   [P3] "Add Indexer Loss [Deepseek v4]" (MaxText pull request 5033):
  *        commit messages (causal block mask, packing), code review
  *        ("Teacher Distribution Semantic Mismatch", "Numerical & JAX
@@ -48,6 +50,10 @@ int orc_num_threads(void)
 
 #define ORC_FLT_MIN 1.1754943508222875e-38 /* float32 tiny, 2^-126 */
 #define ORC_OLD_FLOOR 1e-10                 /* the per-branch target's floor */
+/* how distill_target forms lse_full[h] */
+#define ORC_LSE_JOINT 0                     /* LSE(window, compressed, sink) */
+#define ORC_LSE_PER_BRANCH 1                /* the compressed LSE alone */
+#define ORC_LSE_GIVEN 2                     /* passed in by the caller */
 
 static double bf16_val(uint16_t bits)
 {
@@ -154,21 +160,30 @@ void orc_window_lse(const uint16_t *Q, const uint16_t *Kw, const int32_t *doc_st
  *   p[k]         = u[k] / max(m, FLT_MIN)  (0 on masked slots) [the floor is the
  *                  smallest normal float32, no longer 1e-10]
  *
- * per_branch != 0 selects the earlier per-branch target that the Primus page
+ * mode == ORC_LSE_PER_BRANCH selects the earlier per-branch target that the Primus page
  * keeps behind an A/B switch and the MaxText page prints [P1, second commit
  * message: PRIMUS_V4_DISTILL_NONCOMP_LSE=0 restores it; P3 commit messages]:
  * every head is normalised over the selected compressed entries alone,
  *   lse_full[h] = clse[h]   (window and sink ignored; wl and sink may be NULL)
  * and the floor is the old 1e-10: p[k] = u[k] / max(m, 1e-10).
  *
- * wl: [n, H] window log-mass rows aligned with the token list.
+ * mode == ORC_LSE_GIVEN takes lse_full[h] from the wl rows as given: the
+ * per-head log-normaliser of the whole attention row (window, selected
+ * compressed entries and sink), which a CSA attention forward that returns
+ * its LSE has already computed [P1, first commit message: the compressed
+ * share of a head is exp(compressed_lse - full_lse); P2, gluon_v3
+ * "Optimization Notes", "Forward": the CSA forward route returns its LSE].
+ * The sink is not read and the floor is FLT_MIN, as for the joint target.
+ *
+ * wl: [n, H] rows aligned with the token list: the window log-mass, or
+ * lse_full itself under ORC_LSE_GIVEN (unused under ORC_LSE_PER_BRANCH).
  * Returns the number of idx entries outside {-1} U [0, P) (data errors; those
  * slots are masked).
  */
 int64_t orc_distill_target(const uint16_t *Q, const uint16_t *pool, const int32_t *idx,
                            const double *wl, const float *sink, const int32_t *doc_start,
                            int64_t B, int64_t S, int64_t H, int64_t D, int64_t K, int64_t cr,
-                           double scale, const int64_t *tokens, int64_t n_tokens, int per_branch, double *p)
+                           double scale, const int64_t *tokens, int64_t n_tokens, int mode, double *p)
 {
     int64_t n = tokens ? n_tokens : B * S;
     int64_t P = S / cr;
@@ -193,8 +208,12 @@ int64_t orc_distill_target(const uint16_t *Q, const uint16_t *pool, const int32_
             for (int64_t k = 0; k < K; ++k)
                 z[h * K + k] = sel[k] ? scale * dot_bf16(q, pool + (b * P + row[k]) * D, D) : -INFINITY;
             double clse = lse_list(z + h * K, K);
-            if (per_branch) {
+            if (mode == ORC_LSE_PER_BRANCH) {
                 lse_full[h] = clse;
+                continue;
+            }
+            if (mode == ORC_LSE_GIVEN) {
+                lse_full[h] = wl[i * H + h];
                 continue;
             }
             double parts[3];
@@ -215,7 +234,7 @@ int64_t orc_distill_target(const uint16_t *Q, const uint16_t *pool, const int32_
             u[k] = acc;
             m += acc;
         }
-        const double floor_ = per_branch ? ORC_OLD_FLOOR : ORC_FLT_MIN;
+        const double floor_ = mode == ORC_LSE_PER_BRANCH ? ORC_OLD_FLOOR : ORC_FLT_MIN;
         double den = m > floor_ ? m : floor_;
         for (int64_t k = 0; k < K; ++k)
             u[k] = sel[k] ? u[k] / den : 0.0;

@@ -58,3 +58,45 @@ def target_long_way(Q, Kw, pool, idx, sink, doc_start, W, cr, scale, tokens=None
         row[np.nonzero(sel)[0]] = mass / max(m, FLT_MIN)
         out.append(row)
     return np.array(out).reshape(-1, K)
+
+
+def joint_lse_long_way(Q, Kw, pool, idx, sink, doc_start, W, cr, scale):
+    """[B*S, H]: log of the joint softmax's denominator per (token, head), i.e.
+    the log-normaliser a CSA attention forward over the window keys, the
+    selected compressed rows and the sink reports, from the same concatenated
+    logit vector as target_long_way."""
+    B, S, H, D = Q.shape
+    P = pool.shape[1]
+    Qf, Kf, Pf = _f64(Q), _f64(Kw), _f64(pool)
+    out = np.empty((B * S, H))
+    for g in range(B * S):
+        b, t = divmod(g, S)
+        d0 = 0 if doc_start is None else min(max(int(doc_start[b, t]), 0), t)
+        lo = max(d0, t - W + 1)
+        q = Qf[b, t]
+        sel = selected_mask(idx[b, t], t, cr, P, d0)
+        parts = [scale * (q @ Kf[b, lo:t + 1].T), scale * (q @ Pf[b, idx[b, t][sel].astype(np.int64)].T)]
+        if sink is not None:
+            parts.append(sink.astype(np.float64)[:, None])
+        logits = np.concatenate(parts, axis=1)
+        mx = logits.max(axis=1)
+        out[g] = mx + np.log(np.exp(logits - mx[:, None]).sum(axis=1))
+    return out
+
+
+def compressed_lse_long_way(Q, pool, idx, doc_start, cr, scale):
+    """[B*S, H]: log-sum-exp of each head's selected compressed logits (-inf
+    where a token selects nothing)."""
+    B, S, H, D = Q.shape
+    P = pool.shape[1]
+    Qf, Pf = _f64(Q), _f64(pool)
+    out = np.full((B * S, H), -np.inf)
+    for g in range(B * S):
+        b, t = divmod(g, S)
+        d0 = 0 if doc_start is None else min(max(int(doc_start[b, t]), 0), t)
+        sel = selected_mask(idx[b, t], t, cr, P, d0)
+        if sel.any():
+            z = scale * (Qf[b, t] @ Pf[b, idx[b, t][sel].astype(np.int64)].T)
+            mx = z.max(axis=1)
+            out[g] = mx + np.log(np.exp(z - mx[:, None]).sum(axis=1))
+    return out

@@ -17,7 +17,7 @@ from scipy.special import logsumexp
 
 import oracle
 import synth
-from tests.longway import FLT_MIN, target_long_way
+from tests.longway import FLT_MIN, compressed_lse_long_way, joint_lse_long_way, target_long_way
 
 GOLD = os.path.join(os.path.dirname(__file__), "golden")
 
@@ -295,6 +295,52 @@ def test_per_branch_mode_ignores_window_and_sink_and_sums_to_one():
     rows = p1.sum(axis=1)
     nonempty = rows > 0
     np.testing.assert_allclose(rows[nonempty], 1.0, rtol=1e-12)
+
+
+@pytest.mark.parametrize("seed,docs,sink,W", [(50, False, True, 5), (51, True, True, 3), (52, True, False, 7)])
+def test_full_lse_mode_with_joint_lse_is_joint_target(seed, docs, sink, W):
+    """Handing the target the joint softmax's own log-normaliser (the LSE a
+    CSA attention forward over window, selected rows and sink returns,
+    computed here the long way) reproduces the joint target written out term
+    by term; the sink is inside that LSE and must not be added again."""
+    Q, Kw, pool, idx, snk, ds = _rand_problem(seed, B=2, S=32, H=3, D=16, K=6, W=W, docs=docs, sink=sink)
+    scale = 1 / 4
+    lf = joint_lse_long_way(Q, Kw, pool, idx, snk, ds, W, 4, scale)
+    p, bad = oracle.distill_target(Q, pool, idx, lf, snk, ds, 4, scale, full_lse=True)
+    assert bad == 0
+    ref = target_long_way(Q, Kw, pool, idx, snk, ds, W, 4, scale)
+    np.testing.assert_allclose(p, ref, rtol=0, atol=1e-12)
+    p_nosink, _ = oracle.distill_target(Q, pool, idx, lf, None, ds, 4, scale, full_lse=True)
+    np.testing.assert_array_equal(p, p_nosink)
+
+
+def test_full_lse_mode_is_shift_invariant():
+    """A common offset c on every head's LSE scales every u_k by exp(-c), so
+    the L1-normalised p does not move (the floor stays idle here); an offset
+    on one head alone re-weights that head and does move p."""
+    Q, Kw, pool, idx, snk, ds = _rand_problem(53, B=1, S=32, H=3, D=16, K=6, docs=True)
+    scale = 0.3
+    lf = joint_lse_long_way(Q, Kw, pool, idx, snk, ds, 5, 4, scale)
+    p0, _ = oracle.distill_target(Q, pool, idx, lf, None, ds, 4, scale, full_lse=True)
+    p1, _ = oracle.distill_target(Q, pool, idx, lf + 3.7, None, ds, 4, scale, full_lse=True)
+    np.testing.assert_allclose(p1, p0, rtol=1e-12, atol=1e-15)
+    lf2 = lf.copy()
+    lf2[:, 1] += 3.0
+    p2, _ = oracle.distill_target(Q, pool, idx, lf2, None, ds, 4, scale, full_lse=True)
+    assert np.abs(p2 - p0).max() > 1e-3
+
+
+def test_full_lse_mode_with_compressed_lse_is_per_branch():
+    """With each head's own compressed LSE as the given normaliser every head
+    contributes a full distribution over its selected rows: the per-branch
+    target (its 1e-10 floor is idle, the row mass being H)."""
+    Q, Kw, pool, idx, snk, ds = _rand_problem(54, B=2, S=32, H=4, D=16, K=6, docs=True)
+    scale = 0.25
+    lc = compressed_lse_long_way(Q, pool, idx, ds, 4, scale)
+    lc = np.where(np.isfinite(lc), lc, 0.0)   # tokens with nothing selected: p is 0 regardless
+    p, _ = oracle.distill_target(Q, pool, idx, lc, None, ds, 4, scale, full_lse=True)
+    pb, _ = oracle.distill_target(Q, pool, idx, None, None, ds, 4, scale, per_branch=True)
+    np.testing.assert_allclose(p, pb, rtol=0, atol=1e-13)
 
 
 def test_target_invariants():
