@@ -127,8 +127,9 @@ sai_status sai_distill_target(const uint16_t *Q, const uint16_t *pool, const int
                               int B, int S, int H, int D, int K, int cr, float scale,
                               float *p, int32_t *d_err, void *stream);
 
-/* Flags of sai_distill_target_ex. */
+/* Flags of sai_distill_target_ex (at most one of the two). */
 #define SAI_TARGET_PER_BRANCH 1u
+#define SAI_TARGET_FULL_LSE 2u
 
 /*
  * sai_distill_target_ex -- sai_distill_target with a flags word.
@@ -144,8 +145,23 @@ sai_status sai_distill_target(const uint16_t *Q, const uint16_t *pool, const int
  *
  * i.e. p is the head mean of the per-head softmaxes over the selected slots.
  * window_lse and sink are not read in that mode and may be NULL.
- * Unknown flag bits return SAI_ERR_UNSUPPORTED; everything else (layouts,
- * sizes, errors, ownership) is as for sai_distill_target.
+ *
+ * SAI_TARGET_FULL_LSE: window_lse [B,S,H] fp32 holds lse_full itself, each
+ * head's natural-log normaliser over the whole attention row (window keys,
+ * selected compressed entries and sink), as a CSA attention forward that
+ * returns its LSE has computed it (Primus page "perf(deepseek-v4): fuse and
+ * enable the indexer distillation loss", first commit message: the
+ * compressed share of a head is exp(compressed_lse - full_lse); Primus page
+ * "Docker Build for DeepSeek-v4", gluon_v3 "Optimization Notes": the CSA
+ * forward route returns its LSE). Then
+ *
+ *   u[k] = sum_h exp(z[h,k] - window_lse[b,t,h]),  p[b,t,k] = u[k] / max(m, FLT_MIN),
+ *
+ * no window pass is needed, and sink is not read (it is inside the LSE).
+ *
+ * Unknown flag bits, or both flags at once, return SAI_ERR_UNSUPPORTED;
+ * everything else (layouts, sizes, errors, ownership) is as for
+ * sai_distill_target.
  */
 sai_status sai_distill_target_ex(const uint16_t *Q, const uint16_t *pool, const int32_t *idx,
                                  const float *window_lse, const float *sink, const int32_t *doc_start,

@@ -49,6 +49,7 @@ _lib.sai_distill_target_ex.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _
                                        _P, _P, _P]
 _lib.sai_distill_target_ex.restype = _I
 TARGET_PER_BRANCH = 1   # flag of sai_distill_target_ex: the earlier per-branch target
+TARGET_FULL_LSE = 2     # flag of sai_distill_target_ex: window_lse holds the full per-head LSE
 _lib.sai_distill_target_kl_workspace_bytes.argtypes = [_I, _I, _I]
 _lib.sai_distill_target_kl_workspace_bytes.restype = ctypes.c_size_t
 _lib.sai_distill_target_kl.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, ctypes.c_uint,
@@ -137,14 +138,9 @@ def window_lse(Q: torch.Tensor, Kw: torch.Tensor, W: int, scale: float,
     return out
 
 
-def distill_target(Q: torch.Tensor, pool: torch.Tensor, idx: Optional[torch.Tensor], wl: Optional[torch.Tensor], cr: int,
-                   scale: float, sink: Optional[torch.Tensor] = None, doc_start: Optional[torch.Tensor] = None,
-                   err: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
-                   per_branch: bool = False) -> torch.Tensor:
-    """p[B,S,K] through sai_distill_target_ex. per_branch=True selects the
-    earlier per-branch target; wl and sink are then not used (may be None).
-    idx=None is the dense warm-up stage: every compressed block is a slot
-    (K = S/cr, slot k = block k)."""
+def _target_inputs(Q, pool, idx, wl, cr, sink, doc_start, err, per_branch, full_lse):
+    """Checked arguments shared by the target entry points:
+    (Q bits, pool bits, K, wl, sink, flags)."""
     B, S, H, D = Q.shape
     K = idx.shape[-1] if idx is not None else S // cr
     Q = _bf16_bits(Q, "Q")
@@ -152,10 +148,14 @@ def distill_target(Q: torch.Tensor, pool: torch.Tensor, idx: Optional[torch.Tens
     if tuple(pool.shape) != (B, S // cr, D):
         raise ValueError("pool must be [B,S/cr,D]")
     _want(idx, "idx", torch.int32, (B, S, K))
+    if per_branch and full_lse:
+        raise ValueError("per_branch and full_lse exclude each other")
     if per_branch:
         wl, sink = None, None
     elif wl is None:
-        raise ValueError("window_lse is required unless per_branch")
+        raise ValueError("window_lse (the full LSE with full_lse=True) is required unless per_branch")
+    if full_lse:
+        sink = None   # already inside the given LSE
     _want(wl, "window_lse", torch.float32, (B, S, H))
     if sink is not None:
         # The Primus page: a sink must hold one value per head (else ValueError).
@@ -164,11 +164,27 @@ def distill_target(Q: torch.Tensor, pool: torch.Tensor, idx: Optional[torch.Tens
         _want(sink, "sink", torch.float32)
     _want(doc_start, "doc_start", torch.int32, (B, S))
     _want(err, "err", torch.int32)
+    flags = (TARGET_PER_BRANCH if per_branch else 0) | (TARGET_FULL_LSE if full_lse else 0)
+    return Q, pool, K, wl, sink, flags
+
+
+def distill_target(Q: torch.Tensor, pool: torch.Tensor, idx: Optional[torch.Tensor], wl: Optional[torch.Tensor], cr: int,
+                   scale: float, sink: Optional[torch.Tensor] = None, doc_start: Optional[torch.Tensor] = None,
+                   err: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
+                   per_branch: bool = False, full_lse: bool = False) -> torch.Tensor:
+    """p[B,S,K] through sai_distill_target_ex. per_branch=True selects the
+    earlier per-branch target; wl and sink are then not used (may be None).
+    full_lse=True says wl already holds lse_full, each head's log-normaliser
+    over the window, the selected entries and the sink, as a CSA attention
+    forward returns it; sink is then not used. idx=None is the dense warm-up
+    stage: every compressed block is a slot (K = S/cr, slot k = block k)."""
+    B, S, H, D = Q.shape
+    Q, pool, K, wl, sink, flags = _target_inputs(Q, pool, idx, wl, cr, sink, doc_start, err, per_branch, full_lse)
     if out is None:
         out = torch.empty((B, S, K), dtype=torch.float32, device=Q.device)
     _want(out, "out", torch.float32, (B, S, K))
     st = _lib.sai_distill_target_ex(_ptr(Q), _ptr(pool), _ptr(idx), _ptr(wl), _ptr(sink), _ptr(doc_start),
-                                    B, S, H, D, K, int(cr), float(scale), TARGET_PER_BRANCH if per_branch else 0,
+                                    B, S, H, D, K, int(cr), float(scale), flags,
                                     _ptr(out), _ptr(err), _stream(Q.device))
     _check(st, "sai_distill_target_ex")
     return out
@@ -183,30 +199,15 @@ def distill_target_kl(Q: torch.Tensor, pool: torch.Tensor, idx: Optional[torch.T
                       sink: Optional[torch.Tensor] = None, doc_start: Optional[torch.Tensor] = None,
                       err: Optional[torch.Tensor] = None, p: Optional[torch.Tensor] = None,
                       per_branch: bool = False, workspace: Optional[torch.Tensor] = None,
-                      loss: Optional[torch.Tensor] = None, dscores: Optional[torch.Tensor] = None
-                      ) -> Tuple[torch.Tensor, torch.Tensor]:
+                      loss: Optional[torch.Tensor] = None, dscores: Optional[torch.Tensor] = None,
+                      full_lse: bool = False) -> Tuple[torch.Tensor, torch.Tensor]:
     """(loss, dscores) through sai_distill_target_kl: the target and the KL
     stage in one call. p (optional [B,S,K] fp32 output) receives the target
     when given; without it the target never leaves the GPU's on-chip memory
-    where the fused route applies."""
+    where the fused route applies. per_branch and full_lse as for
+    distill_target."""
     B, S, H, D = Q.shape
-    K = idx.shape[-1] if idx is not None else S // cr
-    Q = _bf16_bits(Q, "Q")
-    pool = _bf16_bits(pool, "pool")
-    if tuple(pool.shape) != (B, S // cr, D):
-        raise ValueError("pool must be [B,S/cr,D]")
-    _want(idx, "idx", torch.int32, (B, S, K))
-    if per_branch:
-        wl, sink = None, None
-    elif wl is None:
-        raise ValueError("window_lse is required unless per_branch")
-    _want(wl, "window_lse", torch.float32, (B, S, H))
-    if sink is not None:
-        if sink.numel() != H:
-            raise ValueError(f"sink needs one logit per head: expected {H} values, found {sink.numel()}")
-        _want(sink, "sink", torch.float32)
-    _want(doc_start, "doc_start", torch.int32, (B, S))
-    _want(err, "err", torch.int32)
+    Q, pool, K, wl, sink, flags = _target_inputs(Q, pool, idx, wl, cr, sink, doc_start, err, per_branch, full_lse)
     _want(scores, "scores", torch.float32, (B, S, K))
     if valid.dtype == torch.bool:
         valid = valid.view(torch.uint8)
@@ -221,7 +222,7 @@ def distill_target_kl(Q: torch.Tensor, pool: torch.Tensor, idx: Optional[torch.T
         dscores = torch.empty((B, S, K), dtype=torch.float32, device=Q.device)
     _want(dscores, "dscores", torch.float32, (B, S, K))
     st = _lib.sai_distill_target_kl(_ptr(Q), _ptr(pool), _ptr(idx), _ptr(wl), _ptr(sink), _ptr(doc_start),
-                                    B, S, H, D, K, int(cr), float(scale), TARGET_PER_BRANCH if per_branch else 0,
+                                    B, S, H, D, K, int(cr), float(scale), flags,
                                     _ptr(scores), _ptr(valid), float(coeff), _ptr(p), _ptr(loss), _ptr(dscores),
                                     _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(err),
                                     _stream(Q.device))

@@ -84,7 +84,7 @@ __global__ void __launch_bounds__(kGenThreads)
     target_generic_kernel(const uint16_t *__restrict__ Q, const uint16_t *__restrict__ pool,
                           const int32_t *__restrict__ idx, const float *__restrict__ wl,
                           const float *__restrict__ sink, const int32_t *__restrict__ doc_start, int S, int H,
-                          int D, int K, int cr, float scale, int per_branch, float *__restrict__ p, int32_t *err)
+                          int D, int K, int cr, float scale, int lse_mode, float *__restrict__ p, int32_t *err)
 {
     extern __shared__ float gsm[];
     float *qs = gsm;                              // [H][D]
@@ -145,11 +145,15 @@ __global__ void __launch_bounds__(kGenThreads)
             se += expf(zs[j * H + h] - M);
         const float clse = M + logf(se);
         hM[h] = M;
-        if (per_branch) {
+        if (lse_mode == kLsePerBranch) {
             hA[h] = M - clse;                     // each head normalised over its selected entries
             continue;
         }
         const float w = wl[(size_t)g * H + h];
+        if (lse_mode == kLseGiven) {
+            hA[h] = M - w;                        // the whole row's normaliser, as given
+            continue;
+        }
         float mm = fmaxf(w, clse);
         if (sink)
             mm = fmaxf(mm, sink[h]);
@@ -171,7 +175,7 @@ __global__ void __launch_bounds__(kGenThreads)
         mpart += u;
     }
     const float mt = block_sum(mpart, scratch);
-    const float ln_floor = per_branch ? kLnOldFloorG : kLnFltMinG;
+    const float ln_floor = lse_mode == kLsePerBranch ? kLnOldFloorG : kLnFltMinG;
     const bool plain = logf(mt) + At >= ln_floor;
     const float f = plain ? 0.f : expf(At - ln_floor);
     for (int j = threadIdx.x; j < nsel; j += blockDim.x)
@@ -201,7 +205,7 @@ size_t target_simt_smem_bytes(int H, int D, int K)
 
 cudaError_t launch_target_simt(const uint16_t *Q, const uint16_t *pool, const int32_t *idx, const float *wl,
                                const float *sink, const int32_t *doc_start, int B, int S, int H, int D, int K,
-                               int cr, float scale, int per_branch, float *p, int32_t *err,
+                               int cr, float scale, int lse_mode, float *p, int32_t *err,
                                cudaStream_t stream)
 {
     const size_t smem = target_simt_smem_bytes(H, D, K);
@@ -210,7 +214,7 @@ cudaError_t launch_target_simt(const uint16_t *Q, const uint16_t *pool, const in
     if (e != cudaSuccess)
         return e;
     target_generic_kernel<<<B * S, kGenThreads, smem, stream>>>(Q, pool, idx, wl, sink, doc_start, S, H, D, K, cr,
-                                                                scale, per_branch, p, err);
+                                                                scale, lse_mode, p, err);
     return cudaGetLastError();
 }
 

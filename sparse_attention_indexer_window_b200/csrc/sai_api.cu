@@ -178,13 +178,16 @@ sai_status target_impl(const uint16_t *Q, const uint16_t *pool, const int32_t *i
                        const float *sink, const int32_t *doc_start, int B, int S, int H, int D, int K, int cr,
                        float scale, unsigned flags, float *p, int32_t *d_err, cudaStream_t st, const KlFuse *kf)
 {
-    if (flags & ~SAI_TARGET_PER_BRANCH)
+    if ((flags & ~(SAI_TARGET_PER_BRANCH | SAI_TARGET_FULL_LSE)) ||
+        (flags & (SAI_TARGET_PER_BRANCH | SAI_TARGET_FULL_LSE)) == (SAI_TARGET_PER_BRANCH | SAI_TARGET_FULL_LSE))
         return SAI_ERR_UNSUPPORTED;
     const bool per_branch = (flags & SAI_TARGET_PER_BRANCH) != 0;
-    if (per_branch) {
+    const int lse_mode = per_branch ? sai::kLsePerBranch
+                                    : ((flags & SAI_TARGET_FULL_LSE) ? sai::kLseGiven : sai::kLseJoint);
+    if (per_branch)
         window_lse = nullptr;   // not read in this mode
-        sink = nullptr;
-    }
+    if (lse_mode != sai::kLseJoint)
+        sink = nullptr;         // per-branch: no sink; given LSE: the sink is inside it
     // idx NULL: dense over all blocks; p may be NULL only when the KL is fused
     if (!Q || !pool || (!window_lse && !per_branch) || (!p && !kf))
         return SAI_ERR_NULL;
@@ -221,7 +224,7 @@ sai_status target_impl(const uint16_t *Q, const uint16_t *pool, const int32_t *i
         a.tiles_per_group = 256 / H;
         a.idx_bulk = (idx && (K % 4) == 0 && al16(idx)) ? 1 : 0;
         a.n_astages = n_astages;
-        a.per_branch = per_branch ? 1 : 0;
+        a.lse_mode = lse_mode;
         a.pool_box_rows = (int)std::min<int64_t>(128, (int64_t)B * P);
         a.scale = scale;
         a.pool = pool;
@@ -272,7 +275,7 @@ sai_status target_impl(const uint16_t *Q, const uint16_t *pool, const int32_t *i
             return e;
     } else if ((int)sai::target_simt_smem_bytes(H, D, K) <= smem_cap) {
         sai_status e = cuda_status(sai::launch_target_simt(Q, pool, idx, window_lse, sink, doc_start, B, S, H, D, K,
-                                                           cr, scale, per_branch ? 1 : 0, p, d_err, st));
+                                                           cr, scale, lse_mode, p, d_err, st));
         if (e != SAI_OK || !kf)
             return e;
     } else {

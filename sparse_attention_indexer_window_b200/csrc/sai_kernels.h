@@ -25,6 +25,12 @@ cudaError_t launch_window_lse_tc(const CUtensorMap &mapQ, const CUtensorMap &map
                                  int grid, cudaStream_t stream);
 
 // ------------------------------------------------------------ distill_target
+// How the target forms each head's log-normaliser lse_full.
+enum : int {
+    kLseJoint = 0,      // LSE(window log-mass, compressed LSE, sink); floor FLT_MIN
+    kLsePerBranch = 1,  // the compressed LSE alone; floor 1e-10; wl and sink unused
+    kLseGiven = 2,      // wl holds lse_full itself; floor FLT_MIN; sink unused
+};
 struct TgtTcArgs {
     int B, S, H, D, K, cr, P;
     int n_tok;            // B*S
@@ -32,7 +38,7 @@ struct TgtTcArgs {
     int idx_bulk;         // idx rows are 16-byte aligned (K % 4 == 0): stage them by bulk copy
     int n_astages;        // depth of the gathered-row stage ring
     int pool_box_rows;    // rows of the pool's TMA box (min(128, B*P))
-    int per_branch;       // 1: per-branch target (lse_full = clse, floor 1e-10); wl and sink unused
+    int lse_mode;         // how lse_full is formed: kLseJoint, kLsePerBranch or kLseGiven
     float scale;
     const uint16_t *pool;
     const int32_t *idx;
@@ -66,7 +72,7 @@ cudaError_t launch_window_lse_simt(const uint16_t *Q, const uint16_t *Kw, const 
 size_t target_simt_smem_bytes(int H, int D, int K);
 cudaError_t launch_target_simt(const uint16_t *Q, const uint16_t *pool, const int32_t *idx, const float *wl,
                                const float *sink, const int32_t *doc_start, int B, int S, int H, int D, int K,
-                               int cr, float scale, int per_branch, float *p, int32_t *err,
+                               int cr, float scale, int lse_mode, float *p, int32_t *err,
                                cudaStream_t stream);
 
 // ---------------------------------------------------------------- distill_kl

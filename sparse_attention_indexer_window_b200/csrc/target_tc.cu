@@ -747,9 +747,12 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
                             if (et < HH) {
                                 const float M = st.colM[et] * 0.69314718055994531f;  // natural log units
                                 const float clse = M + logf(st.colS[et]);
-                                if (a.per_branch) {
+                                if (a.lse_mode == kLsePerBranch) {
                                     // each head normalised over its selected entries alone
                                     st.head_a[et] = M - clse;
+                                } else if (a.lse_mode == kLseGiven) {
+                                    // the whole row's normaliser, as the attention forward gave it
+                                    st.head_a[et] = M - wl_h;
                                 } else {
                                     float mm = fmaxf(fmaxf(wl_h, clse), sink_h);
                                     float acc = expf(wl_h - mm) + expf(clse - mm);
@@ -841,7 +844,7 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
                 mtot += st.red_m[w];
             float f = 0.f;
             if (nsel > 0) {
-                const float ln_floor = a.per_branch ? kLnOldFloor : kLnFltMin;
+                const float ln_floor = a.lse_mode == kLsePerBranch ? kLnOldFloor : kLnFltMin;
                 const bool plain = logf(mtot) + At >= ln_floor;
                 f = plain ? 1.0f / mtot : expf(At - ln_floor);
             }

@@ -1,4 +1,4 @@
-"""The distillation target written out the long way (numpy, fp64).
+"""The distillation target computed term by term (numpy, fp64).
 
 The Primus page ("perf(deepseek-v4): fuse and enable the indexer distillation
 loss", second commit message and "Test plan") checks its fused target against

@@ -79,13 +79,16 @@ def test_distill_target_host_errors(sai):
 
 
 def test_distill_target_ex_host_errors(sai):
-    """The flags variant: unknown flag bits are refused; the joint target
-    (flags 0) needs window_lse. Only paths that return before any launch."""
+    """The flags variant: unknown flag bits and the two modes at once are
+    refused; the joint target (flags 0) and the given-LSE target need
+    window_lse. Only paths that return before any launch."""
     f = sai.lib().sai_distill_target_ex
     args = lambda wl, flags: (FAKE, FAKE, FAKE, wl, None, None, 1, 64, 4, 32, 8, 4, 0.1, flags, FAKE, None, None)
-    assert f(*args(FAKE, 2)) == 3                     # unknown flag bit
+    assert f(*args(FAKE, 4)) == 3                     # unknown flag bit
     assert f(*args(FAKE, 0x80000000)) == 3
+    assert f(*args(FAKE, 3)) == 3                     # per-branch and full LSE together
     assert f(*args(None, 0)) == 1                     # joint target without window_lse
+    assert f(*args(None, 2)) == 1                     # full-LSE target without its LSE
     assert f(*args(FAKE, 1)[:6], 1, 64, 4, 32, 8, 3, 0.1, 1, FAKE, None, None) == 2   # S % cr, per-branch
 
 

@@ -183,7 +183,7 @@ def test_target_long_way_on_tiny_workload():
 @pytest.mark.parametrize("docs", [False, True])
 def test_dense_mode_is_every_causal_block(docs):
     """Dense warm-up (idx omitted): slot k is compressed block k. The target
-    equals the joint softmax written out the long way over the explicit
+    equals the joint softmax computed term by term over the explicit
     index row 0..P-1, puts exactly zero on blocks a token cannot see (the
     MaxText page's rule: with t=4, cr=4 block 0 visible, block 1 masked), and
     with every block visible equals the sparse target that selects them all."""
