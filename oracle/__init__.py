@@ -46,6 +46,8 @@ def _load():
         lib.orc_count_valid_rows.restype = I
         lib.orc_distill_kl.argtypes = [P, P, P, I, I, Dd, I, P, P, P]
         lib.orc_distill_kl.restype = None
+        lib.orc_indexer_topk.argtypes = [P, P, I, I, I, I, P, I, P, P, P]
+        lib.orc_indexer_topk.restype = None
         lib.orc_num_threads.argtypes = []
         lib.orc_num_threads.restype = ctypes.c_int
         _lib = lib
@@ -152,3 +154,18 @@ def run_all(w, tokens=None):
         _, ds, _ = distill_kl(p, w.scores.reshape(-1, K)[tokens], w.valid.reshape(-1, K)[tokens],
                               w.coeff, n_norm=n_all)
     return wl, p, loss, ds, bad
+
+
+def indexer_topk(scores, doc_start, cr: int, K: int, tokens=None):
+    """(idx [n, K] int32, sel [n, K] fp32, valid [n, K] uint8): the top-K
+    candidate blocks of each token by indexer score, in ascending block
+    order with a -1 tail; ``scores`` is [B, S, S/cr] fp32."""
+    B, S, P = scores.shape
+    assert P * cr == S and 1 <= K <= P
+    sc = _c(scores, np.float32); ds = _c(doc_start, np.int32)
+    tk, n = _tokens(tokens, B, S)
+    idx = np.empty((n, K), dtype=np.int32)
+    sel = np.empty((n, K), dtype=np.float32)
+    valid = np.empty((n, K), dtype=np.uint8)
+    _load().orc_indexer_topk(_ptr(sc), _ptr(ds), B, S, cr, K, _ptr(tk), n, _ptr(idx), _ptr(sel), _ptr(valid))
+    return idx, sel, valid

@@ -328,3 +328,78 @@ void orc_distill_kl(const double *p, const float *scores, const uint8_t *valid,
     if (loss)
         *loss = coeff * total / den;
 }
+
+/*
+ * Top-K selection of compressed blocks per token, from given indexer scores
+ * [P3, the indexer's selection: top-k block indices, with -1 wherever the
+ * selection is invalid, returned together with the index scores; P3 commit
+ * messages: causal block mask and packing mask]. The score formula of the
+ * indexer itself is not on the pages; its output is this function's input.
+ *
+ *   block j of token (b,t) is a candidate iff (j+1)*cr - 1 <= t, j*cr >= d0,
+ *   and its score is neither NaN nor -inf (a masked or invalid entry);
+ *   the K candidates with the largest scores are selected, an equal score
+ *   going to the lower block index (+0 and -0 are equal);
+ *   slot k holds the k-th selected block in ascending block order; the
+ *   slots past the number selected hold -1.
+ *
+ * scores: [B*S, P] fp32 with P = S/cr. Outputs for the flat token ids in
+ * tokens (all when NULL): idx [n, K]; sel [n, K] = the score of the block in
+ * each slot (0 on -1 slots); valid [n, K] = 1 on selected slots.
+ */
+typedef struct {
+    float s;
+    int64_t j;
+} orc_cand;
+
+static int orc_cand_by_score(const void *pa, const void *pb)
+{
+    const orc_cand *a = (const orc_cand *)pa, *b = (const orc_cand *)pb;
+    if (a->s > b->s)
+        return -1;
+    if (a->s < b->s)
+        return 1;
+    return (a->j > b->j) - (a->j < b->j);
+}
+
+static int orc_cand_by_block(const void *pa, const void *pb)
+{
+    const orc_cand *a = (const orc_cand *)pa, *b = (const orc_cand *)pb;
+    return (a->j > b->j) - (a->j < b->j);
+}
+
+void orc_indexer_topk(const float *scores, const int32_t *doc_start, int64_t B, int64_t S, int64_t cr, int64_t K,
+                      const int64_t *tokens, int64_t n_tokens, int32_t *idx, float *sel, uint8_t *valid)
+{
+    int64_t n = tokens ? n_tokens : B * S;
+    int64_t P = S / cr;
+#pragma omp parallel for schedule(dynamic, 16)
+    for (int64_t i = 0; i < n; ++i) {
+        int64_t g = tokens ? tokens[i] : i;
+        int64_t t = g % S;
+        int64_t d0 = doc_begin(doc_start, g, t);
+        const float *row = scores + g * P;
+        orc_cand *c = (orc_cand *)malloc(sizeof(orc_cand) * (size_t)(P > 0 ? P : 1));
+        int64_t m = 0;
+        for (int64_t j = 0; j < P; ++j) {
+            float s = row[j];
+            if ((j + 1) * cr - 1 <= t && j * cr >= d0 && !isnan(s) && !(isinf(s) && s < 0)) {
+                c[m].s = s;
+                c[m].j = j;
+                ++m;
+            }
+        }
+        qsort(c, (size_t)m, sizeof(orc_cand), orc_cand_by_score);
+        int64_t take = m < K ? m : K;
+        qsort(c, (size_t)take, sizeof(orc_cand), orc_cand_by_block);
+        for (int64_t k = 0; k < K; ++k) {
+            const int inr = k < take;
+            idx[i * K + k] = inr ? (int32_t)c[k].j : -1;
+            if (sel)
+                sel[i * K + k] = inr ? c[k].s : 0.0f;
+            if (valid)
+                valid[i * K + k] = (uint8_t)(inr ? 1 : 0);
+        }
+        free(c);
+    }
+}

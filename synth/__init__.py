@@ -238,6 +238,14 @@ def make(name: str, *, seed: Optional[int] = None, with_sink: bool = True,
                     scores=scores, valid=valid)
 
 
+def index_scores(B: int, S: int, cr: int, seed: int) -> np.ndarray:
+    """[B, S, S/cr] fp32 indexer scores over every compressed block, N(0,1)
+    (the flash workload's random causal score; which blocks a token may
+    select is left to the selection)."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    return rng.standard_normal((B, S, S // cr), dtype=np.float32)
+
+
 def sample_tokens(B: int, S: int, n: int, seed: int = 7) -> np.ndarray:
     """A sorted, seeded sample of flat token ids b*S+t that always includes the
     first and last token of every row (the lightest and heaviest)."""

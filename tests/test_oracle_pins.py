@@ -343,6 +343,85 @@ def test_full_lse_mode_with_compressed_lse_is_per_branch():
     np.testing.assert_allclose(p, pb, rtol=0, atol=1e-13)
 
 
+def _topk_golden_inputs():
+    g = _gold("indexer_topk_small.json")
+    B, S, cr, K = g["B"], g["S"], g["cr"], g["K"]
+    sc = np.zeros((B, S, S // cr), dtype=np.float32)
+    sc[:] = -np.inf                                    # blocks a row does not list
+    for r in g["rows"]:
+        v = [float(x) for x in r["scores"]]
+        sc[r["b"], r["t"], :len(v)] = np.array(v, dtype=np.float32)
+    ds = np.zeros((B, S), dtype=np.int32)
+    ds[1, g["doc_start_batch1_from_t8"]:] = g["doc_start_batch1_from_t8"]
+    return g, sc, ds
+
+
+def test_topk_golden_hand_rows():
+    """Rows worked by hand from the selection rules: the largest scores, a
+    boundary tie to the lower block, +0 == -0, NaN and -inf never selected,
+    the causal block rule and the document rule, -1 padding."""
+    g, sc, ds = _topk_golden_inputs()
+    assert np.signbit(sc[0, 29, 0]) and not np.signbit(sc[0, 29, 2])
+    toks = [r["b"] * g["S"] + r["t"] for r in g["rows"]]
+    idx, sel, valid = oracle.indexer_topk(sc, ds, g["cr"], g["K"], tokens=toks)
+    for i, r in enumerate(g["rows"]):
+        assert idx[i].tolist() == r["idx"], (r["note"], idx[i].tolist())
+        for k, j in enumerate(r["idx"]):
+            assert valid[i, k] == (1 if j >= 0 else 0)
+            want = sc[r["b"], r["t"], j] if j >= 0 else 0.0
+            assert sel[i, k] == want or (np.isinf(want) and sel[i, k] == want)
+
+
+@pytest.mark.parametrize("seed,docs,K,step", [(60, False, 5, 0.5), (61, True, 3, 0.25), (62, True, 8, 0.0)])
+def test_topk_selection_properties(seed, docs, K, step):
+    """On random scores (rounded to a coarse grid so that ties are common),
+    every row satisfies the definition: min(K, candidates) slots filled in
+    ascending block order then -1; no unselected candidate scores above a
+    selected one; on the boundary score the lowest blocks are taken."""
+    rng = np.random.default_rng(seed)
+    B, S, cr = 2, 64, 4
+    P = S // cr
+    sc = rng.standard_normal((B, S, P)).astype(np.float32)
+    if step:
+        sc = (np.round(sc / step) * step).astype(np.float32)
+    sc[rng.random((B, S, P)) < 0.05] = -np.inf
+    ds = None
+    if docs:
+        ds = np.zeros((B, S), dtype=np.int32)
+        for b in range(B):
+            s0 = int(rng.integers(1, S))
+            ds[b, s0:] = s0
+    idx, sel, valid = oracle.indexer_topk(sc, ds, cr, K)
+    idx = idx.reshape(B, S, K)
+    for b in range(B):
+        for t in range(S):
+            d0 = 0 if ds is None else min(int(ds[b, t]), t)
+            j = np.arange(P)
+            cand = ((j + 1) * cr - 1 <= t) & (j * cr >= d0) & ~np.isnan(sc[b, t]) & (sc[b, t] != -np.inf)
+            n = min(K, int(cand.sum()))
+            row = idx[b, t]
+            assert np.all(row[n:] == -1) and np.all(row[:n] >= 0)
+            chosen = row[:n]
+            assert np.all(np.diff(chosen) > 0)
+            assert np.all(cand[chosen])
+            if n == 0:
+                continue
+            rest = cand.copy()
+            rest[chosen] = False
+            lo = sc[b, t, chosen].min()
+            if rest.any():
+                assert sc[b, t][rest].max() <= lo
+                tied_rest = np.nonzero(rest & (sc[b, t] == lo))[0]
+                tied_in = chosen[sc[b, t, chosen] == lo]
+                if tied_rest.size:
+                    assert tied_in.max() < tied_rest.min()
+    flat = idx.reshape(-1, K)
+    assert np.array_equal(valid, (flat >= 0).astype(np.uint8))
+    rows = np.arange(B * S)[:, None]
+    want = np.where(flat >= 0, sc.reshape(B * S, P)[rows, np.maximum(flat, 0)], 0.0).astype(np.float32)
+    assert np.array_equal(sel, want)
+
+
 def test_target_invariants():
     Q, Kw, pool, idx, snk, ds = _rand_problem(30, B=2, S=32, H=4, D=16, K=8, docs=True)
     scale = 0.25
