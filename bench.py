@@ -62,6 +62,19 @@ def workload_config(w, n):
     }
 
 
+def candidate_blocks(w):
+    """Blocks every token may select (causal and inside its document): the
+    score entries the selection kernel reads."""
+    t = np.arange(w.S)
+    hi = (t + 1) // w.cr
+    n = 0
+    for b in range(w.B):
+        d0 = np.zeros(w.S, dtype=np.int64) if w.doc_start is None else np.clip(w.doc_start[b], 0, t)
+        lo = (d0 + w.cr - 1) // w.cr
+        n += int(np.maximum(hi - lo, 0).sum())
+    return n
+
+
 def algorithmic_counts(w):
     """Valid selected slots and window keys: the units behind the flop and byte
     counts (2*H*D flops per slot or key)."""
@@ -346,6 +359,26 @@ def main():
     e2e_ms = shard.max_over_ranks(e0.elapsed_time(e1), device=dev)
     e2e_value = B * S * world * args.e2e_steps / (e2e_ms / 1e3)
 
+    # ------------------------------------------- block selection (side line)
+    # sai_indexer_topk feeds idx, scores and valid to the step above; it is
+    # timed on its own, on this workload's shape, and is not part of `value`.
+    isc = torch.from_numpy(synth.index_scores(B, S, w.cr, seed=shard.rank_seed(7001, rank))).to(dev)
+    t_idx = torch.empty((B, S, K), dtype=torch.int32, device=dev)
+    t_sel = torch.empty((B, S, K), dtype=torch.float32, device=dev)
+    t_val = torch.empty((B, S, K), dtype=torch.uint8, device=dev)
+    sel_steps = max(3, min(nsteps, 200))
+    sel_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(sel_steps)]
+    for i in range(3 + sel_steps):
+        flush_l2(i)
+        if i >= 3:
+            sel_ev[i - 3][0].record(stream)
+        sai.indexer_topk(isc, w.cr, K, doc_start=t["doc_start"], idx=t_idx, sel_scores=t_sel, valid=t_val)
+        if i >= 3:
+            sel_ev[i - 3][1].record(stream)
+    torch.cuda.synchronize(dev)
+    sel_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in sel_ev)
+    del isc
+
     # batch-wide loss over all ranks, for the record (not part of the timed path)
     n_rows = int(t["valid"].reshape(-1, K).any(dim=1).sum().item())
     loss_all, _ = shard.global_mean_loss(float(loss.item()), n_rows, device=dev)
@@ -363,6 +396,8 @@ def main():
         # algorithmic bytes of the two HBM-bound kernels
         win_bytes = B * S * H * D * 2 + B * S * D * 2 + B * S * H * 4
         kl_bytes = B * S * K * (4 + 4 + 1 + 4)
+        cand = candidate_blocks(w)
+        sel_bytes = 4 * cand + B * S * K * (4 + 4 + 1)
         line = {
             "metric": METRIC,
             "value": value,
@@ -397,6 +432,14 @@ def main():
                                "traffic": traffic_record("window_lse_tc.cu")},
                 "distill_kl": {"bound": "hbm", "achieved_gbs": kl_bytes / (kl_ms / 1e3) / 1e9,
                                "peak_gbs": hbm_gbs, "frac": kl_bytes / (kl_ms / 1e3) / 1e9 / hbm_gbs},
+            },
+            "selection": {
+                "kernel": "indexer_topk_kernel (sai_indexer_topk), not part of the step",
+                "ms": sel_ms, "bound": "hbm", "achieved_gbs": sel_bytes / (sel_ms / 1e3) / 1e9,
+                "peak_gbs": hbm_gbs, "frac": sel_bytes / (sel_ms / 1e3) / 1e9 / hbm_gbs,
+                "algorithmic": f"4 B per candidate score read ({cand} candidates) + 9 B per slot written "
+                               f"({B * S * K} slots) = {sel_bytes} B/launch",
+                "launches": sel_steps, "input": "index scores N(0,1) over every block, seed per rank",
             },
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "steps": args.e2e_steps},

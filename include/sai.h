@@ -259,6 +259,43 @@ sai_status sai_distill_kl_noalloc(const float *p, const float *scores, const uin
                                   int B, int S, int K, float coeff,
                                   float *loss, float *dscores, void *stream);
 
+/*
+ * sai_indexer_topk -- which compressed blocks each token selects, from the
+ * lightning indexer's scores.
+ *
+ * Source: MaxText page "Add Indexer Loss [Deepseek v4]": the indexer keeps its
+ * top-k block indices, writes -1 wherever the choice is invalid, and returns
+ * the index scores with them; its commit messages give the causal block mask
+ * and the packing mask. The indexer's own score formula is not on the pages:
+ * index_scores is the caller's. Rule, per token (b,t) with document start d0
+ * (clamped to [0, t]):
+ *
+ *   block j (0 <= j < P = S/cr) is a candidate iff (j+1)*cr - 1 <= t,
+ *   j*cr >= d0, and index_scores[b,t,j] is neither NaN nor -inf;
+ *   the K candidates with the largest scores are selected, an equal score
+ *   going to the lower block (+0 and -0 are equal);
+ *   idx[b,t,k] = the k-th selected block in ascending block order, and -1
+ *   for k >= the number selected (fewer than K candidates).
+ *
+ * The outputs are the inputs the loss calls take: idx for
+ * sai_distill_target, and sel_scores / valid for sai_distill_kl.
+ *
+ *   index_scores [B,S,P] fp32 device, 4-byte aligned (entries of blocks that
+ *                are not candidates are not read)
+ *   doc_start    [B,S] int32 or NULL (one document per sequence)
+ *   idx          [B,S,K] int32, written
+ *   sel_scores   [B,S,K] fp32 or NULL: index_scores[b,t,idx] on selected
+ *                slots, 0 on -1 slots
+ *   valid        [B,S,K] uint8 or NULL: 1 on selected slots, 0 elsewhere
+ *
+ * Sizes: S % cr == 0, 1 <= K <= P, P <= 32768. All buffers caller-owned; no
+ * allocation, no synchronisation; deterministic. Errors: SAI_ERR_NULL,
+ * SAI_ERR_SHAPE, SAI_ERR_ALIGN, SAI_ERR_UNSUPPORTED (P too large),
+ * SAI_ERR_CUDA.
+ */
+sai_status sai_indexer_topk(const float *index_scores, const int32_t *doc_start, int B, int S, int cr, int K,
+                            int32_t *idx, float *sel_scores, uint8_t *valid, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -65,6 +65,8 @@ _lib.sai_distill_kl_noalloc_max_scratch_bytes.argtypes = []
 _lib.sai_distill_kl_noalloc_max_scratch_bytes.restype = ctypes.c_size_t
 _lib.sai_status_string.argtypes = [_I]
 _lib.sai_status_string.restype = ctypes.c_char_p
+_lib.sai_indexer_topk.argtypes = [_P, _P, _I, _I, _I, _I, _P, _P, _P, _P]
+_lib.sai_indexer_topk.restype = _I
 _lib.sai_version.argtypes = []
 _lib.sai_version.restype = _I
 
@@ -288,3 +290,30 @@ def distill_loss(Q, Kw, pool, idx, scores, valid, *, W: int, cr: int, scale: flo
     p = distill_target(Q, pool, idx, wl, cr, scale, sink=sink, doc_start=doc_start, err=err)
     loss, ds = distill_kl(p, scores, valid, coeff, workspace=workspace)
     return loss, ds, p, wl
+
+
+def indexer_topk(index_scores: torch.Tensor, cr: int, K: int, doc_start: Optional[torch.Tensor] = None,
+                 idx: Optional[torch.Tensor] = None, sel_scores: Optional[torch.Tensor] = None,
+                 valid: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+    """(idx, sel_scores, valid) through sai_indexer_topk: each token's K
+    candidate blocks with the largest indexer scores, in ascending block
+    order with a -1 tail, the scores of those blocks and the valid flags."""
+    B, S, P = index_scores.shape
+    if P * cr != S:
+        raise ValueError("index_scores must be [B,S,S/cr]")
+    _want(index_scores, "index_scores", torch.float32, (B, S, P))
+    _want(doc_start, "doc_start", torch.int32, (B, S))
+    dev = index_scores.device
+    if idx is None:
+        idx = torch.empty((B, S, K), dtype=torch.int32, device=dev)
+    if sel_scores is None:
+        sel_scores = torch.empty((B, S, K), dtype=torch.float32, device=dev)
+    if valid is None:
+        valid = torch.empty((B, S, K), dtype=torch.uint8, device=dev)
+    _want(idx, "idx", torch.int32, (B, S, K))
+    _want(sel_scores, "sel_scores", torch.float32, (B, S, K))
+    _want(valid, "valid", torch.uint8, (B, S, K))
+    st = _lib.sai_indexer_topk(_ptr(index_scores), _ptr(doc_start), B, S, int(cr), int(K), _ptr(idx),
+                               _ptr(sel_scores), _ptr(valid), _stream(dev))
+    _check(st, "sai_indexer_topk")
+    return idx, sel_scores, valid

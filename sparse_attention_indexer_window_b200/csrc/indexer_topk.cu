@@ -1,0 +1,212 @@
+// Top-K compressed-block selection per token from given indexer scores
+// (MaxText page "Add Indexer Loss [Deepseek v4]": the indexer keeps its
+// top-k block indices, writes -1 wherever the choice is invalid and returns
+// the scores alongside; its commit messages give the causal block mask and
+// the packing mask). The indexer's own score formula is not on the pages;
+// its output is this kernel's input.
+//
+// Rule: block j of token (b,t) is a candidate iff (j+1)*cr - 1 <= t,
+// j*cr >= d0 (the token's document start) and its score is neither NaN nor
+// -inf. The K candidates with the largest scores are selected, an equal
+// score going to the lower block (+0 and -0 are equal). Slot k holds the
+// k-th selected block in ascending block order; the slots past the number
+// selected hold -1.
+//
+// One CTA per token row. HBM-bound: a row's candidate scores are read once
+// (about half the row on average, since later blocks are in the future),
+// kept in shared memory as order-preserving 32-bit keys, and selected with
+// an 8-bit radix select (four histogram passes) for the K-th largest key.
+// A block-wide scan then compacts the selected blocks in block order, which
+// gives the ascending slot order without a sort.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "indexer_topk.h"
+
+namespace sai {
+namespace {
+
+constexpr int kTkThreads = 256;
+constexpr int kTkWarps = kTkThreads / 32;
+
+// Order-preserving key of a score: a larger score gives a larger key, +0 and
+// -0 give the same key, and 0 marks an entry that cannot be selected (NaN or
+// -inf). Every selectable key is at least the key of -FLT_MAX, 0x00800000.
+__device__ __forceinline__ uint32_t order_key(float x)
+{
+    uint32_t u = __float_as_uint(x);
+    if ((u & 0x7fffffffu) > 0x7f800000u || u == 0xff800000u)   // NaN, -inf
+        return 0u;
+    if ((u << 1) == 0u)                                         // -0 -> +0
+        u = 0u;
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Exclusive prefix sum of v over the block (thread order), and the total.
+__device__ __forceinline__ int block_excl_scan(int v, int *warp_buf, int &total)
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o)
+            incl += y;
+    }
+    if (lane == 31)
+        warp_buf[warp] = incl;
+    __syncthreads();
+    int before = 0, tot = 0;
+#pragma unroll
+    for (int w = 0; w < kTkWarps; ++w) {
+        const int x = warp_buf[w];
+        before += (w < warp) ? x : 0;
+        tot += x;
+    }
+    __syncthreads();   // warp_buf is free again for the next scan
+    total = tot;
+    return before + incl - v;
+}
+
+__global__ void __launch_bounds__(kTkThreads)
+    indexer_topk_kernel(const float *__restrict__ scores, const int32_t *__restrict__ doc_start, int S, int cr,
+                        int P, int K, int32_t *__restrict__ idx, float *__restrict__ sel,
+                        uint8_t *__restrict__ valid)
+{
+    extern __shared__ uint32_t keys[];   // [P]
+    __shared__ int hist[256];
+    __shared__ int warp_buf[kTkWarps];
+    __shared__ uint32_t s_prefix;
+    __shared__ int s_rem;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int g = blockIdx.x;
+    const int t = g % S;
+    int d0 = 0;
+    if (doc_start) {
+        d0 = doc_start[g];
+        d0 = d0 < 0 ? 0 : (d0 > t ? t : d0);
+    }
+    // candidates are the blocks j in [jlo, jhi): (j+1)*cr - 1 <= t and j*cr >= d0
+    const int jhi = min(P, (t + 1) / cr);
+    const int jlo = (d0 + cr - 1) / cr;
+    const float *row = scores + (size_t)g * P;
+
+    int cnt = 0;
+    for (int j = tid; j < P; j += kTkThreads) {
+        const uint32_t k = (j >= jlo && j < jhi) ? order_key(__ldg(row + j)) : 0u;
+        keys[j] = k;
+        cnt += k != 0u;
+    }
+    int n_cand = 0;
+    block_excl_scan(cnt, warp_buf, n_cand);   // also orders the key writes before the reads below
+
+    // Threshold key T and the number `rem` of entries equal to T to take.
+    // With no more candidates than K, every candidate is taken (T = 0).
+    uint32_t T = 0u;
+    int rem = 0;
+    if (n_cand > K) {
+        uint32_t prefix = 0u, mask = 0u;
+        rem = K;
+        for (int shift = 24; shift >= 0; shift -= 8) {
+            for (int i = tid; i < 256; i += kTkThreads)
+                hist[i] = 0;
+            __syncthreads();
+            for (int j = tid; j < P; j += kTkThreads) {
+                const uint32_t k = keys[j];
+                if (k != 0u && (k & mask) == prefix)
+                    atomicAdd(&hist[(k >> shift) & 255u], 1);
+            }
+            __syncthreads();
+            if (warp == 0) {
+                // lane l holds bins 255-8l, 254-8l, ..., 248-8l (high to low)
+                int c[8], sum = 0;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    c[e] = hist[255 - 8 * lane - e];
+                    sum += c[e];
+                }
+                int incl = sum;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+                    if (lane >= o)
+                        incl += y;
+                }
+                const int excl = incl - sum;
+                // the keys matching the prefix number at least rem, so exactly
+                // one lane holds the bin where the count from the top reaches rem
+                const unsigned here = __ballot_sync(0xffffffffu, excl < rem && rem <= incl);
+                if (lane == __ffs(here) - 1) {
+                    int acc = excl, e = 0;
+                    while (e < 7 && acc + c[e] < rem)
+                        acc += c[e++];
+                    s_prefix = prefix | ((uint32_t)(255 - 8 * lane - e) << shift);
+                    s_rem = rem - acc;
+                }
+            }
+            __syncthreads();
+            prefix = s_prefix;
+            rem = s_rem;
+            mask |= 255u << shift;
+        }
+        T = prefix;
+    }
+
+    // Compaction in block order: thread i owns blocks [i*E, (i+1)*E).
+    const int E = (P + kTkThreads - 1) / kTkThreads;
+    const int j0 = min(P, tid * E), j1 = min(P, j0 + E);
+    int cgt = 0, ceq = 0;
+    for (int j = j0; j < j1; ++j) {
+        const uint32_t k = keys[j];
+        cgt += k > T;
+        ceq += (k != 0u && k == T);
+    }
+    int n_eq = 0;
+    const int eq_before = block_excl_scan(ceq, warp_buf, n_eq);
+    const int take_eq = max(0, min(ceq, rem - eq_before));
+    int n_out = 0;
+    int slot = block_excl_scan(cgt + take_eq, warp_buf, n_out);
+    int32_t *irow = idx + (size_t)g * K;
+    float *srow = sel ? sel + (size_t)g * K : nullptr;
+    uint8_t *vrow = valid ? valid + (size_t)g * K : nullptr;
+    int eq_seen = eq_before;
+    for (int j = j0; j < j1; ++j) {
+        const uint32_t k = keys[j];
+        bool take = k > T;
+        if (!take && k != 0u && k == T)
+            take = eq_seen++ < rem;
+        if (take) {
+            irow[slot] = j;
+            if (srow)
+                srow[slot] = __ldg(row + j);
+            if (vrow)
+                vrow[slot] = 1;
+            ++slot;
+        }
+    }
+    for (int k = n_out + tid; k < K; k += kTkThreads) {
+        irow[k] = -1;
+        if (srow)
+            srow[k] = 0.f;
+        if (vrow)
+            vrow[k] = 0;
+    }
+}
+
+}  // namespace
+
+size_t indexer_topk_smem_bytes(int P) { return (size_t)P * 4; }
+
+cudaError_t launch_indexer_topk(const float *scores, const int32_t *doc_start, int B, int S, int cr, int K,
+                                int32_t *idx, float *sel, uint8_t *valid, cudaStream_t stream)
+{
+    const int P = S / cr;
+    const size_t smem = indexer_topk_smem_bytes(P);
+    cudaError_t e = cudaFuncSetAttribute(indexer_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess)
+        return e;
+    indexer_topk_kernel<<<B * S, kTkThreads, smem, stream>>>(scores, doc_start, S, cr, P, K, idx, sel, valid);
+    return cudaGetLastError();
+}
+
+}  // namespace sai

@@ -10,6 +10,7 @@
 #include <string.h>
 
 #include "sai.h"
+#include "indexer_topk.h"
 #include "sai_kernels.h"
 
 namespace {
@@ -94,7 +95,7 @@ const char *sai_status_string(int status)
     }
 }
 
-int sai_version(void) { return 100; }
+int sai_version(void) { return 200; }
 
 sai_status sai_window_lse(const uint16_t *Q, const uint16_t *Kw, const int32_t *doc_start, int B, int S, int H,
                           int D, int W, float scale, float *window_lse, void *stream)
@@ -351,6 +352,24 @@ sai_status sai_distill_kl(const float *p, const float *scores, const uint8_t *va
         return SAI_ERR_WORKSPACE;
     return cuda_status(sai::launch_distill_kl(pl, p, scores, valid, coeff, loss, dscores, workspace,
                                               reinterpret_cast<cudaStream_t>(stream)));
+}
+
+sai_status sai_indexer_topk(const float *index_scores, const int32_t *doc_start, int B, int S, int cr, int K,
+                            int32_t *idx, float *sel_scores, uint8_t *valid, void *stream)
+{
+    if (!index_scores || !idx)
+        return SAI_ERR_NULL;
+    if (B < 1 || S < 1 || cr < 1 || K < 1 || (S % cr) != 0)
+        return SAI_ERR_SHAPE;
+    const int P = S / cr;
+    if (K > P || (int64_t)B * S * P > INT32_MAX || (int64_t)B * S * K > INT32_MAX)
+        return SAI_ERR_SHAPE;
+    if (P > sai::kTopkMaxP || (int)sai::indexer_topk_smem_bytes(P) > max_smem_optin())
+        return SAI_ERR_UNSUPPORTED;
+    if (!al4(index_scores) || !al4(idx) || (sel_scores && !al4(sel_scores)) || (doc_start && !al4(doc_start)))
+        return SAI_ERR_ALIGN;
+    return cuda_status(sai::launch_indexer_topk(index_scores, doc_start, B, S, cr, K, idx, sel_scores, valid,
+                                                reinterpret_cast<cudaStream_t>(stream)));
 }
 
 }  // extern "C"

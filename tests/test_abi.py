@@ -126,3 +126,15 @@ def test_python_sink_length_check(sai):
     with pytest.raises((ValueError, TypeError)):
         sai.distill_target(Q, torch.zeros((1, 2, 8), dtype=torch.bfloat16), torch.zeros((1, 8, 2), dtype=torch.int32),
                            torch.zeros((1, 8, 4)), 4, 0.1, sink=torch.zeros(3))
+
+
+def test_indexer_topk_host_errors(sai):
+    """Refusals that return before any launch: missing pointers, S % cr,
+    K outside [1, P], too many blocks per row."""
+    f = sai.lib().sai_indexer_topk
+    assert f(None, None, 1, 64, 4, 8, FAKE, None, None, None) == 1     # no scores
+    assert f(FAKE, None, 1, 64, 4, 8, None, None, None, None) == 1     # no idx
+    assert f(FAKE, None, 1, 66, 4, 8, FAKE, None, None, None) == 2     # S % cr
+    assert f(FAKE, None, 1, 64, 4, 17, FAKE, None, None, None) == 2    # K > P
+    assert f(FAKE, None, 1, 64, 4, 0, FAKE, None, None, None) == 2     # K < 1
+    assert f(FAKE, None, 1, 40000, 1, 8, FAKE, None, None, None) == 3  # P > 32768
