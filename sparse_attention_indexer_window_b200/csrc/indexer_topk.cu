@@ -13,9 +13,10 @@
 // selected hold -1.
 //
 // One CTA per token row. HBM-bound: a row's candidate scores are read once
-// (about half the row on average, since later blocks are in the future),
-// kept in shared memory as order-preserving 32-bit keys, and selected with
-// an 8-bit radix select (four histogram passes) for the K-th largest key.
+// (about half the row on average, since later blocks are in the future; only
+// the candidate range is read and walked), kept in shared memory as
+// order-preserving 32-bit keys, and selected with an 8-bit radix select
+// (four histogram passes) for the K-th largest key.
 // A block-wide scan then compacts the selected blocks in block order, which
 // gives the ascending slot order without a sort.
 #include <cuda_runtime.h>
@@ -73,7 +74,7 @@ __global__ void __launch_bounds__(kTkThreads)
                         int P, int K, int32_t *__restrict__ idx, float *__restrict__ sel,
                         uint8_t *__restrict__ valid)
 {
-    extern __shared__ uint32_t keys[];   // [P]
+    extern __shared__ uint32_t keys[];   // [jhi - jlo] (at most P)
     __shared__ int hist[256];
     __shared__ int warp_buf[kTkWarps];
     __shared__ uint32_t s_prefix;
@@ -88,13 +89,14 @@ __global__ void __launch_bounds__(kTkThreads)
     }
     // candidates are the blocks j in [jlo, jhi): (j+1)*cr - 1 <= t and j*cr >= d0
     const int jhi = min(P, (t + 1) / cr);
-    const int jlo = (d0 + cr - 1) / cr;
-    const float *row = scores + (size_t)g * P;
+    const int jlo = min(jhi, (d0 + cr - 1) / cr);
+    const int L = jhi - jlo;                          // keys[i] is block jlo + i
+    const float *row = scores + (size_t)g * P + jlo;
 
     int cnt = 0;
-    for (int j = tid; j < P; j += kTkThreads) {
-        const uint32_t k = (j >= jlo && j < jhi) ? order_key(__ldg(row + j)) : 0u;
-        keys[j] = k;
+    for (int i = tid; i < L; i += kTkThreads) {
+        const uint32_t k = order_key(__ldg(row + i));
+        keys[i] = k;
         cnt += k != 0u;
     }
     int n_cand = 0;
@@ -111,8 +113,8 @@ __global__ void __launch_bounds__(kTkThreads)
             for (int i = tid; i < 256; i += kTkThreads)
                 hist[i] = 0;
             __syncthreads();
-            for (int j = tid; j < P; j += kTkThreads) {
-                const uint32_t k = keys[j];
+            for (int i = tid; i < L; i += kTkThreads) {
+                const uint32_t k = keys[i];
                 if (k != 0u && (k & mask) == prefix)
                     atomicAdd(&hist[(k >> shift) & 255u], 1);
             }
@@ -152,12 +154,12 @@ __global__ void __launch_bounds__(kTkThreads)
         T = prefix;
     }
 
-    // Compaction in block order: thread i owns blocks [i*E, (i+1)*E).
-    const int E = (P + kTkThreads - 1) / kTkThreads;
-    const int j0 = min(P, tid * E), j1 = min(P, j0 + E);
+    // Compaction in block order: thread n owns candidates [n*E, (n+1)*E).
+    const int E = (L + kTkThreads - 1) / kTkThreads;
+    const int i0 = min(L, tid * E), i1 = min(L, i0 + E);
     int cgt = 0, ceq = 0;
-    for (int j = j0; j < j1; ++j) {
-        const uint32_t k = keys[j];
+    for (int i = i0; i < i1; ++i) {
+        const uint32_t k = keys[i];
         cgt += k > T;
         ceq += (k != 0u && k == T);
     }
@@ -170,15 +172,15 @@ __global__ void __launch_bounds__(kTkThreads)
     float *srow = sel ? sel + (size_t)g * K : nullptr;
     uint8_t *vrow = valid ? valid + (size_t)g * K : nullptr;
     int eq_seen = eq_before;
-    for (int j = j0; j < j1; ++j) {
-        const uint32_t k = keys[j];
+    for (int i = i0; i < i1; ++i) {
+        const uint32_t k = keys[i];
         bool take = k > T;
         if (!take && k != 0u && k == T)
             take = eq_seen++ < rem;
         if (take) {
-            irow[slot] = j;
+            irow[slot] = jlo + i;
             if (srow)
-                srow[slot] = __ldg(row + j);
+                srow[slot] = __ldg(row + i);
             if (vrow)
                 vrow[slot] = 1;
             ++slot;
