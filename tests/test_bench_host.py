@@ -70,3 +70,17 @@ def test_traffic_record_is_dropped_when_sources_change(tmp_path, monkeypatch):
     (csrc / "k.cu").write_text("kernel v2")
     assert bench.traffic_record("k.cu") is None
     assert bench.traffic_record("other.cu") is None
+
+
+@pytest.mark.parametrize("name,kw", [("tiny", {}), ("small", {}), ("packed", {"B": 2, "S": 256, "K": 16})])
+def test_candidate_blocks_match_a_direct_count(name, kw):
+    """The selection line's read bytes count every (token, block) pair with
+    the block wholly at or before the token and inside its document."""
+    w = synth.make(name, **kw)
+    P = w.S // w.cr
+    n = 0
+    for b in range(w.B):
+        for t in range(w.S):
+            d0 = 0 if w.doc_start is None else min(max(int(w.doc_start[b, t]), 0), t)
+            n += sum(1 for j in range(P) if (j + 1) * w.cr - 1 <= t and j * w.cr >= d0)
+    assert bench.candidate_blocks(w) == n
