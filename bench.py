@@ -24,6 +24,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -139,7 +140,7 @@ class Clocks:
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_bench_{os.getpid()}.csv")
+        self.path = os.path.join(tempfile.gettempdir(), f"sai_clocks_{os.getpid()}_{gpu_index}.csv")
 
     def start(self):
         try:
@@ -161,7 +162,12 @@ class Clocks:
             self.proc.kill()
         self.f.close()
         with open(self.path) as f:
-            return self.parse(f)
+            summary = self.parse(f)
+        try:
+            os.remove(self.path)
+        except OSError:
+            pass
+        return summary
 
     @staticmethod
     def parse(lines):
