@@ -3,7 +3,6 @@ the workload description for one and several ranks, the algorithmic counts
 behind the roofline numbers, and the rule that a recorded DRAM traffic figure
 is dropped once the kernel's sources change."""
 import json
-import os
 
 import numpy as np
 import pytest
