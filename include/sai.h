@@ -10,6 +10,12 @@
  *   sai_distill_target  Q, pool, idx, window_lse, sink -> p [B,S,K]
  *   sai_distill_kl      p, scores, valid -> loss (device scalar), dscores [B,S,K]
  *
+ * Around them: sai_distill_target_ex (the per-branch target, or the target
+ * from the attention forward's own LSE), sai_distill_target_kl (target and
+ * KL in one call), sai_distill_kl_noalloc (no workspace argument), and
+ * sai_indexer_topk, the block selection that produces idx, scores and valid
+ * from the indexer's scores.
+ *
  * Conventions for every call
  *   - Tensor arguments are DEVICE pointers to dense row-major (C-contiguous)
  *     arrays, owned by the caller. The library never allocates device memory
@@ -44,7 +50,8 @@ typedef enum sai_status {
     SAI_ERR_CUDA = 4,        /* a CUDA runtime/driver call or a launch failed        */
     SAI_ERR_INDEX = 5,       /* device error word: an idx entry outside {-1}U[0,P)   */
     SAI_ERR_WORKSPACE = 6,   /* workspace NULL, too small or not 16-byte aligned     */
-    SAI_ERR_ALIGN = 7,       /* a tensor pointer is not 16-byte aligned              */
+    SAI_ERR_ALIGN = 7,       /* a tensor pointer is misaligned for its call (16 B for
+                                bf16 matrices and 16-byte-vector arrays, else 4 B)   */
     SAI_ERR_TIMEOUT = 8      /* device error word: a kernel gave up a bounded wait   */
 } sai_status;
 
@@ -73,7 +80,7 @@ int sai_version(void);
  *   Kw         [B,S,D]   bf16, 16-byte aligned
  *   doc_start  [B,S] int32 or NULL (one document per row)
  *   scale      logit scale > 0, e.g. 1/sqrt(D)
- *   window_lse [B,S,H] fp32, written
+ *   window_lse [B,S,H] fp32, written, 4-byte aligned
  *
  * Sizes: B,S,H,D,W >= 1 and D % 8 == 0. Errors: SAI_ERR_NULL, SAI_ERR_SHAPE,
  * SAI_ERR_ALIGN, SAI_ERR_UNSUPPORTED, SAI_ERR_CUDA.
@@ -90,9 +97,10 @@ sai_status sai_window_lse(const uint16_t *Q, const uint16_t *Kw, const int32_t *
  * keeps the softmax and the sum over heads on chip) and second commit message
  * / "Why the target was wrong" (each head normalises jointly over window keys,
  * chosen pool rows and its sink; the pool rows' share of head h is
- * exp(clse - lse_full); the L1 floor is the smallest normal float32). Causal block rule: MaxText page "Add Indexer Loss
- * [Deepseek v4]", commit messages (block j is visible to token t iff
- * (j+1)*cr - 1 <= t; cross-document blocks masked).
+ * exp(clse - lse_full); the L1 floor is the smallest normal float32).
+ * Causal block rule: MaxText page "Add Indexer Loss [Deepseek v4]", commit
+ * messages (block j is visible to token t iff (j+1)*cr - 1 <= t;
+ * cross-document blocks masked).
  *
  *   slot k selected iff 0 <= idx[b,t,k] < P (P = S/cr), (idx+1)*cr - 1 <= t
  *                       and idx*cr >= d0 (d0 as in sai_window_lse)
@@ -117,6 +125,8 @@ sai_status sai_window_lse(const uint16_t *Q, const uint16_t *Kw, const int32_t *
  *   d_err      device int32 or NULL. Data errors found on the device (an idx
  *              entry outside {-1} U [0,P)) mask the slot and store
  *              SAI_ERR_INDEX here; the caller zeroes it and reads it back.
+ *   The 32-bit arrays (idx, window_lse, sink, doc_start, p, d_err) must be
+ *   4-byte aligned.
  *
  * Sizes: S % cr == 0, 1 <= K <= S/cr (the MaxText page's topk <= length/4
  * check), D % 8 == 0, scale > 0. Errors: SAI_ERR_NULL, SAI_ERR_SHAPE, SAI_ERR_ALIGN,
@@ -219,9 +229,9 @@ size_t sai_distill_kl_workspace_bytes(int B, int S, int K);
  *   dscores[k]= coeff / max(N,1) * (q[k] * sum_{valid} p - p[k]) on valid
  *               slots of valid rows, 0 elsewhere
  *
- *   p, scores  [B,S,K] fp32; valid [B,S,K] uint8
- *   loss       device fp32 scalar, written
- *   dscores    [B,S,K] fp32, written; NULL = forward only
+ *   p, scores  [B,S,K] fp32; valid [B,S,K] uint8; all 16-byte aligned
+ *   loss       device fp32 scalar, written (4-byte aligned)
+ *   dscores    [B,S,K] fp32, written, 16-byte aligned; NULL = forward only
  *   workspace  device scratch of ws_bytes >= sai_distill_kl_workspace_bytes(),
  *              16-byte aligned; no initialisation needed; must not be shared
  *              by calls that overlap on the device.
