@@ -34,6 +34,7 @@ import numpy as np  # noqa: E402
 WORKLOAD = "flash"
 METRIC = "distill-loss tokens/s (fwd+bwd), S=4096 H=64 K=512 D=512; % bf16 TC peak"
 UNIT = "tokens/s"
+CLOCK_WINDOW_S = 1.5
 
 
 def parse():
@@ -130,11 +131,15 @@ def traffic_record(kernel_src: str):
 
 
 class Clocks:
-    """nvidia-smi sampling of SM clocks and throttle reasons while running."""
+    """nvidia-smi sampling of SM clocks and throttle reasons while running.
 
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    Samples carry nvidia-smi's own timestamps, so the summary can say how many
+    of them fall inside a given wall-clock window (the timed region)."""
+
+    Q = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    INTERVAL_MS = 50
 
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
@@ -146,14 +151,17 @@ class Clocks:
             os.makedirs(os.path.dirname(self.path), exist_ok=True)
             self.f = open(self.path, "w")
             self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.Q}",
-                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                          "--format=csv,noheader,nounits", "-lms", str(self.INTERVAL_MS)],
                                          stdout=self.f, stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
 
-    def stop(self):
+    def stop(self, window=None, timed=None):
+        """Summary over the samples inside `window` (wall-clock (t0, t1)),
+        with the count of those inside `timed` as well."""
         if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0,
+                    "samples_in_timed_region": 0}
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
@@ -161,7 +169,7 @@ class Clocks:
             self.proc.kill()
         self.f.close()
         with open(self.path) as f:
-            summary = self.parse(f)
+            summary = self.parse(f, window, timed)
         try:
             os.remove(self.path)
         except OSError:
@@ -169,26 +177,43 @@ class Clocks:
         return summary
 
     @staticmethod
-    def parse(lines):
+    def _stamp(s):
+        import datetime
+        for fmt in ("%Y/%m/%d %H:%M:%S.%f", "%Y/%m/%d %H:%M:%S"):
+            try:
+                return datetime.datetime.strptime(s, fmt).timestamp()
+            except ValueError:
+                pass
+        return None
+
+    @classmethod
+    def parse(cls, lines, window=None, timed=None):
         """Summary of nvidia-smi rows in the order of Q: median SM clock, max
-        clock, and every slowdown reason seen active in any sample."""
-        sm, mx, reasons, n = [], None, set(), 0
+        clock, and every slowdown reason seen active in any sample, over the
+        rows whose timestamp lies in `window` (all rows when None)."""
+        sm, mx, reasons, n, n_timed = [], None, set(), 0, 0
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for line in lines:
             parts = [x.strip() for x in line.split(",")]
-            if len(parts) < 9:
+            if len(parts) < 10:
+                continue
+            ts = cls._stamp(parts[0])
+            if window is not None and (ts is None or not window[0] <= ts <= window[1]):
                 continue
             try:
-                sm.append(float(parts[1]))
-                mx = float(parts[2])
+                sm.append(float(parts[2]))
+                mx = float(parts[3])
             except ValueError:
                 continue
             n += 1
-            for nm, v in zip(names, parts[5:9]):
+            if timed is not None and ts is not None and timed[0] <= ts <= timed[1]:
+                n_timed += 1
+            for nm, v in zip(names, parts[6:10]):
                 if v.lower() == "active":
                     reasons.add(nm)
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
-                "reasons": sorted(reasons), "samples": n}
+                "reasons": sorted(reasons), "samples": n, "samples_in_timed_region": n_timed,
+                "interval_ms": cls.INTERVAL_MS}
 
 
 def cpu_baseline(w, seconds: float):
@@ -301,10 +326,12 @@ def main():
     nsteps = args.steps
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(nsteps)]
     clocks = Clocks(local)
+    clocks.start()
+    time.sleep(0.2)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
-    clocks.start()
+    wall0 = time.time()
     for i in range(nsteps):
         flush_l2(i)
         e = ev[i]
@@ -317,9 +344,23 @@ def main():
         sai.distill_kl(p, t["scores"], t["valid"], w.coeff, workspace=ws, loss=loss, dscores=ds)
         e[3].record(stream)
     torch.cuda.synchronize(dev)
+    wall1 = time.time()
+    # A short timed region holds few clock samples: keep the same steps running
+    # (untimed) until the clock window spans at least CLOCK_WINDOW_S, so the
+    # record shows the clocks this work runs at. Every rank runs the same count.
+    soak = 0
+    if wall1 - wall0 < CLOCK_WINDOW_S:
+        per = max((wall1 - wall0) / nsteps, 1e-5)
+        soak = int(min(200000, (CLOCK_WINDOW_S - (wall1 - wall0)) / per)) + 1
+        for i in range(soak):
+            flush_l2(i)
+            step()
+        torch.cuda.synchronize(dev)
+    wall2 = time.time()
     if world > 1:
         dist.barrier()
-    clk = clocks.stop()
+    clk = clocks.stop(window=(wall0, wall2), timed=(wall0, wall1))
+    clk["window"] = f"timed region ({wall1 - wall0:.3f} s) plus {soak} more steps of the same work"
     k_win = [e[0].elapsed_time(e[1]) for e in ev]
     k_tgt = [e[1].elapsed_time(e[2]) for e in ev]
     k_kl = [e[2].elapsed_time(e[3]) for e in ev]

@@ -101,6 +101,15 @@ def _check(st: int, where: str):
         raise SaiError(st, where)
 
 
+def _call(fn, dev: torch.device, *args) -> int:
+    """Run one C entry point with the tensors' device current: the library
+    takes its device (SM count, TMA encoding, the allocation-free call's
+    scratch array) from the current device, and the stream passed is that
+    device's current stream."""
+    with torch.cuda.device(dev):
+        return fn(*args, _stream(dev))
+
+
 def _bf16_bits(t: torch.Tensor, name: str) -> torch.Tensor:
     if t.dtype in (torch.bfloat16, torch.int16, torch.uint16):
         if not t.is_contiguous():
@@ -134,8 +143,8 @@ def window_lse(Q: torch.Tensor, Kw: torch.Tensor, W: int, scale: float,
     if out is None:
         out = torch.empty((B, S, H), dtype=torch.float32, device=Q.device)
     _want(out, "out", torch.float32, (B, S, H))
-    st = _lib.sai_window_lse(_ptr(Q), _ptr(Kw), _ptr(doc_start), B, S, H, D, int(W), float(scale),
-                             _ptr(out), _stream(Q.device))
+    st = _call(_lib.sai_window_lse, Q.device, _ptr(Q), _ptr(Kw), _ptr(doc_start), B, S, H, D, int(W),
+               float(scale), _ptr(out))
     _check(st, "sai_window_lse")
     return out
 
@@ -185,9 +194,8 @@ def distill_target(Q: torch.Tensor, pool: torch.Tensor, idx: Optional[torch.Tens
     if out is None:
         out = torch.empty((B, S, K), dtype=torch.float32, device=Q.device)
     _want(out, "out", torch.float32, (B, S, K))
-    st = _lib.sai_distill_target_ex(_ptr(Q), _ptr(pool), _ptr(idx), _ptr(wl), _ptr(sink), _ptr(doc_start),
-                                    B, S, H, D, K, int(cr), float(scale), flags,
-                                    _ptr(out), _ptr(err), _stream(Q.device))
+    st = _call(_lib.sai_distill_target_ex, Q.device, _ptr(Q), _ptr(pool), _ptr(idx), _ptr(wl), _ptr(sink),
+               _ptr(doc_start), B, S, H, D, K, int(cr), float(scale), flags, _ptr(out), _ptr(err))
     _check(st, "sai_distill_target_ex")
     return out
 
@@ -223,11 +231,10 @@ def distill_target_kl(Q: torch.Tensor, pool: torch.Tensor, idx: Optional[torch.T
     if dscores is None:
         dscores = torch.empty((B, S, K), dtype=torch.float32, device=Q.device)
     _want(dscores, "dscores", torch.float32, (B, S, K))
-    st = _lib.sai_distill_target_kl(_ptr(Q), _ptr(pool), _ptr(idx), _ptr(wl), _ptr(sink), _ptr(doc_start),
-                                    B, S, H, D, K, int(cr), float(scale), flags,
-                                    _ptr(scores), _ptr(valid), float(coeff), _ptr(p), _ptr(loss), _ptr(dscores),
-                                    _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(err),
-                                    _stream(Q.device))
+    st = _call(_lib.sai_distill_target_kl, Q.device, _ptr(Q), _ptr(pool), _ptr(idx), _ptr(wl), _ptr(sink),
+               _ptr(doc_start), B, S, H, D, K, int(cr), float(scale), flags,
+               _ptr(scores), _ptr(valid), float(coeff), _ptr(p), _ptr(loss), _ptr(dscores),
+               _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(err))
     _check(st, "sai_distill_target_kl")
     return loss, dscores
 
@@ -255,9 +262,8 @@ def distill_kl(p: torch.Tensor, scores: torch.Tensor, valid: torch.Tensor, coeff
         dscores = torch.empty((B, S, K), dtype=torch.float32, device=scores.device)
     if not want_grad:
         dscores = None
-    st = _lib.sai_distill_kl(_ptr(p), _ptr(scores), _ptr(valid), B, S, K, float(coeff), _ptr(loss),
-                             _ptr(dscores), _ptr(workspace), workspace.numel() * workspace.element_size(),
-                             _stream(scores.device))
+    st = _call(_lib.sai_distill_kl, scores.device, _ptr(p), _ptr(scores), _ptr(valid), B, S, K, float(coeff),
+               _ptr(loss), _ptr(dscores), _ptr(workspace), workspace.numel() * workspace.element_size())
     _check(st, "sai_distill_kl")
     return loss, dscores
 
@@ -277,8 +283,8 @@ def distill_kl_noalloc(p: torch.Tensor, scores: torch.Tensor, valid: torch.Tenso
     _want(valid, "valid", torch.uint8, (B, S, K))
     _want(loss, "loss", torch.float32)
     _want(dscores, "dscores", torch.float32, (B, S, K))
-    st = _lib.sai_distill_kl_noalloc(_ptr(p), _ptr(scores), _ptr(valid), B, S, K, float(coeff), _ptr(loss),
-                                     _ptr(dscores), _stream(scores.device))
+    st = _call(_lib.sai_distill_kl_noalloc, scores.device, _ptr(p), _ptr(scores), _ptr(valid), B, S, K,
+               float(coeff), _ptr(loss), _ptr(dscores))
     _check(st, "sai_distill_kl_noalloc")
 
 
@@ -313,7 +319,7 @@ def indexer_topk(index_scores: torch.Tensor, cr: int, K: int, doc_start: Optiona
     _want(idx, "idx", torch.int32, (B, S, K))
     _want(sel_scores, "sel_scores", torch.float32, (B, S, K))
     _want(valid, "valid", torch.uint8, (B, S, K))
-    st = _lib.sai_indexer_topk(_ptr(index_scores), _ptr(doc_start), B, S, int(cr), int(K), _ptr(idx),
-                               _ptr(sel_scores), _ptr(valid), _stream(dev))
+    st = _call(_lib.sai_indexer_topk, dev, _ptr(index_scores), _ptr(doc_start), B, S, int(cr), int(K),
+               _ptr(idx), _ptr(sel_scores), _ptr(valid))
     _check(st, "sai_indexer_topk")
     return idx, sel_scores, valid

@@ -13,17 +13,28 @@ import synth
 
 def test_clock_summary_reports_median_and_reasons():
     rows = [
-        "0, 1965, 1965, 650.0, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active",
-        "0, 1965, 1965, 700.0, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active",
-        "0, 1800, 1965, 990.0, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
+        "2026/12/03 05:40:00.100, 0, 1965, 1965, 650.0, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active",
+        "2026/12/03 05:40:00.150, 0, 1965, 1965, 700.0, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active",
+        "2026/12/03 05:40:00.200, 0, 1800, 1965, 990.0, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
         "garbage line",
-        "0, [N/A], 1965, 1.0, x, Not Active, Not Active, Not Active, Not Active",
+        "2026/12/03 05:40:00.250, 0, [N/A], 1965, 1.0, x, Not Active, Not Active, Not Active, Not Active",
     ]
     r = bench.Clocks.parse(rows)
     assert r["samples"] == 3
     assert r["sm_mhz"] == 1965.0 and r["sm_max_mhz"] == 1965.0
     assert r["reasons"] == ["sw_power_cap"]
     assert bench.Clocks.parse([])["sm_mhz"] is None
+
+
+def test_clock_summary_windows_by_timestamp():
+    """Only samples inside the clock window count; those inside the timed
+    region are counted apart."""
+    rows = [f"2026/12/03 05:40:0{i}.000, 0, {1900 + i}, 1965, 700.0, 0x0, Not Active, Not Active, "
+            f"Not Active, Not Active" for i in range(6)]
+    t = [bench.Clocks._stamp(f"2026/12/03 05:40:0{i}.000") for i in range(6)]
+    r = bench.Clocks.parse(rows, window=(t[1], t[4]), timed=(t[1], t[2]))
+    assert r["samples"] == 4 and r["samples_in_timed_region"] == 2
+    assert r["sm_mhz"] == 1902.5
 
 
 def test_workload_config_single_and_multi_rank():
