@@ -46,6 +46,8 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--long-steps", type=int, default=30,
+                    help="timed steps of the long-context side line (0: skip it)")
     return ap.parse_args()
 
 
@@ -425,8 +427,56 @@ def main():
     sel_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in sel_ev)
     del isc
 
+    # ------------------------------------------- long context (side line)
+    # The same three calls on the long-context workload (S=16384, K=2048: up
+    # to 2048 selected blocks per token), timed like the step above; not part
+    # of `value`.
+    long_line = None
+    if args.long_steps > 0:
+        del t
+        torch.cuda.empty_cache()
+        wL = synth.make("long", seed=shard.rank_seed(synth.CONFIGS["long"].seed, rank))
+        tL = to_dev(wL, dev)
+        wlL = torch.empty((wL.B, wL.S, wL.H), device=dev)
+        pL = torch.empty((wL.B, wL.S, wL.K), device=dev)
+        dsL = torch.empty((wL.B, wL.S, wL.K), device=dev)
+        lossL = torch.empty(1, device=dev)
+        wsL = torch.empty(sai.kl_workspace_bytes(wL.B, wL.S, wL.K), dtype=torch.uint8, device=dev)
+        evL = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.long_steps)]
+        for i in range(3 + args.long_steps):
+            flush_l2(i)
+            if i >= 3:
+                evL[i - 3][0].record(stream)
+            sai.window_lse(tL["Q"], tL["Kw"], wL.W, wL.scale, tL["doc_start"], out=wlL)
+            if i >= 3:
+                evL[i - 3][1].record(stream)
+            sai.distill_target(tL["Q"], tL["pool"], tL["idx"], wlL, wL.cr, wL.scale, sink=tL["sink"],
+                               doc_start=tL["doc_start"], err=err, out=pL)
+            if i >= 3:
+                evL[i - 3][2].record(stream)
+            sai.distill_kl(pL, tL["scores"], tL["valid"], wL.coeff, workspace=wsL, loss=lossL, dscores=dsL)
+            if i >= 3:
+                evL[i - 3][3].record(stream)
+        torch.cuda.synchronize(dev)
+        assert int(err.item()) == 0
+        selL, winL = algorithmic_counts(wL)
+        msL = statistics.mean(e[0].elapsed_time(e[3]) for e in evL)
+        tgtL = statistics.mean(e[1].elapsed_time(e[2]) for e in evL)
+        long_line = {
+            "workload": f"long: B={wL.B} S={wL.S} H={wL.H} D={wL.D} cr={wL.cr} K={wL.K} W={wL.W}, random "
+                        f"distinct causal blocks, -1 tail; same value distributions",
+            "steps": args.long_steps, "ms_per_step": msL, "tokens_per_s": wL.B * wL.S / (msL / 1e3),
+            "kernels_ms": {"window_lse": statistics.mean(e[0].elapsed_time(e[1]) for e in evL),
+                           "distill_target": tgtL,
+                           "distill_kl": statistics.mean(e[2].elapsed_time(e[3]) for e in evL)},
+            "selected_slots": selL, "window_keys": winL,
+            "distill_target_tflops": 2.0 * wL.H * wL.D * selL / (tgtL / 1e3) / 1e12,
+            "step_tflops": 2.0 * wL.H * wL.D * (selL + winL) / (msL / 1e3) / 1e12,
+        }
+        del tL
+
     # batch-wide loss over all ranks, for the record (not part of the timed path)
-    n_rows = int(t["valid"].reshape(-1, K).any(dim=1).sum().item())
+    n_rows = int((w.valid.reshape(-1, K) != 0).any(axis=1).sum())
     loss_all, _ = shard.global_mean_loss(float(loss.item()), n_rows, device=dev)
 
     if rank == 0:
@@ -489,10 +539,14 @@ def main():
             },
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "steps": args.e2e_steps},
+            "long": long_line,
             "gpu_launches": 4 * nsteps * world,   # window, target, KL count, KL rows; every rank
             "clocks": clk,
             "loss": loss_all,
         }
+        if long_line is not None:
+            long_line["distill_target_frac"] = long_line["distill_target_tflops"] / peak_tf
+            long_line["step_frac"] = long_line["step_tflops"] / peak_tf
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
         print(json.dumps(line), flush=True)

@@ -12,9 +12,11 @@
  *
  * Around them: sai_distill_target_ex (the per-branch target, or the target
  * from the attention forward's own LSE), sai_distill_target_kl (target and
- * KL in one call), sai_distill_kl_noalloc (no workspace argument), and
+ * KL in one call), sai_distill_kl_noalloc (no workspace argument),
  * sai_indexer_topk, the block selection that produces idx, scores and valid
- * from the indexer's scores.
+ * from the indexer's scores, and the calls for splitting sequences across
+ * GPUs by token range: sai_window_lse_range, sai_distill_target_range,
+ * sai_count_valid_rows and sai_distill_kl_ex (a batch-wide N).
  *
  * Conventions for every call
  *   - Tensor arguments are DEVICE pointers to dense row-major (C-contiguous)
@@ -88,6 +90,31 @@ int sai_version(void);
 sai_status sai_window_lse(const uint16_t *Q, const uint16_t *Kw, const int32_t *doc_start,
                           int B, int S, int H, int D, int W, float scale,
                           float *window_lse, void *stream);
+
+/*
+ * sai_window_lse_range -- sai_window_lse over a token range of longer sequences.
+ *
+ * For splitting each sequence across GPUs by token range (the MaxText page
+ * "Add Indexer Loss [Deepseek v4]" speaks of context parallelism only in its
+ * configuration checks; the arithmetic is exactly sai_window_lse's). The call
+ * covers sequence positions t_begin .. t_begin+S-1 of every sequence:
+ *
+ *   window_lse[b,i,h] = log sum_{s=lo}^{t} exp(scale * <Q[b,i,h,:], Kw[b, s - t_begin + kw_lead, :]>)
+ *   t = t_begin + i,  lo = max(d0, t - W + 1),  d0 = clamp(doc_start[b,i], 0, t)
+ *
+ *   Q          [B,S,H,D] bf16: the range's own query rows
+ *   Kw         [B,S+kw_lead,D] bf16: the keys of positions
+ *              t_begin-kw_lead .. t_begin+S-1 (the range plus its halo)
+ *   doc_start  [B,S] int32 sequence positions, or NULL
+ *   t_begin    >= 0; kw_lead in [min(W-1, t_begin), t_begin] (the halo must
+ *              hold every key the range's first window reaches)
+ *
+ * sai_window_lse is this call with t_begin = kw_lead = 0. Errors as for
+ * sai_window_lse (SAI_ERR_SHAPE for a short halo).
+ */
+sai_status sai_window_lse_range(const uint16_t *Q, const uint16_t *Kw, const int32_t *doc_start,
+                                int B, int S, int H, int D, int W, int t_begin, int kw_lead, float scale,
+                                float *window_lse, void *stream);
 
 /*
  * sai_distill_target -- the indexer's teacher target p[b,t,:].
@@ -178,6 +205,30 @@ sai_status sai_distill_target_ex(const uint16_t *Q, const uint16_t *pool, const 
                                  int B, int S, int H, int D, int K, int cr, float scale, unsigned flags,
                                  float *p, int32_t *d_err, void *stream);
 
+/*
+ * sai_distill_target_range -- sai_distill_target_ex over a token range.
+ *
+ * The S tokens of each sequence passed here are positions t_begin ..
+ * t_begin+S-1 of sequences of S_seq tokens (for splitting a sequence across
+ * GPUs, as sai_window_lse_range). Positions, not row numbers, decide the
+ * causal and document rules, and the pool is the whole sequence's:
+ *
+ *   Q          [B,S,H,D] bf16: the range's own query rows
+ *   pool       [B,S_seq/cr,D] bf16: every compressed entry of the sequence
+ *   idx, window_lse, doc_start, p: [B,S,...] rows of the range; idx holds
+ *              pool row numbers, doc_start sequence positions
+ *   slot k of local token i selected iff 0 <= idx < S_seq/cr,
+ *              (idx+1)*cr - 1 <= t_begin + i and idx*cr >= d0
+ *
+ * Sizes: S_seq % cr == 0, 0 <= t_begin, t_begin + S <= S_seq,
+ * 1 <= K <= S_seq/cr. sai_distill_target_ex is this call with S_seq = S and
+ * t_begin = 0. Flags, errors and ownership as for sai_distill_target_ex.
+ */
+sai_status sai_distill_target_range(const uint16_t *Q, const uint16_t *pool, const int32_t *idx,
+                                    const float *window_lse, const float *sink, const int32_t *doc_start,
+                                    int B, int S, int S_seq, int t_begin, int H, int D, int K, int cr,
+                                    float scale, unsigned flags, float *p, int32_t *d_err, void *stream);
+
 /* Bytes of device workspace sai_distill_target_kl needs for these sizes. */
 size_t sai_distill_target_kl_workspace_bytes(int B, int S, int K);
 
@@ -243,6 +294,40 @@ sai_status sai_distill_kl(const float *p, const float *scores, const uint8_t *va
                           int B, int S, int K, float coeff,
                           float *loss, float *dscores, void *workspace, size_t ws_bytes,
                           void *stream);
+
+/*
+ * sai_count_valid_rows -- N, the rows of `valid` that hold a valid slot.
+ *
+ *   valid    [B,S,K] uint8 device, 16-byte aligned
+ *   n_rows   device int32, written (zeroed, then counted, on the stream)
+ *
+ * The count sai_distill_kl normalises by. A caller that splits the batch
+ * across GPUs sums the ranks' counts (an all-reduce of one integer) and hands
+ * the sum to sai_distill_kl_ex, so every rank's dscores carry the batch-wide
+ * 1/N and the ranks' losses add up to the batch loss. Errors: SAI_ERR_NULL,
+ * SAI_ERR_SHAPE, SAI_ERR_ALIGN, SAI_ERR_CUDA.
+ */
+sai_status sai_count_valid_rows(const uint8_t *valid, int B, int S, int K, int32_t *n_rows, void *stream);
+
+/*
+ * sai_distill_kl_ex -- sai_distill_kl with a caller-given N.
+ *
+ * n_rows NULL: exactly sai_distill_kl. Otherwise a device int32 (4-byte
+ * aligned) holding N, read by the kernels when they run (so it may be written
+ * earlier on the same stream, e.g. by an all-reduce of the ranks'
+ * sai_count_valid_rows). Then
+ *
+ *   *loss      = coeff * sum_{rows here} KL_t / max(N, 1)
+ *   dscores[k] = coeff / max(N, 1) * (q[k] * sum_{valid} p - p[k])
+ *
+ * i.e. this call's share of the batch-wide loss (summing the shares over
+ * ranks gives the batch loss) and the batch-wide gradient. Everything else as
+ * for sai_distill_kl.
+ */
+sai_status sai_distill_kl_ex(const float *p, const float *scores, const uint8_t *valid,
+                             int B, int S, int K, float coeff, const int32_t *n_rows,
+                             float *loss, float *dscores, void *workspace, size_t ws_bytes,
+                             void *stream);
 
 /*
  * sai_distill_kl_noalloc -- sai_distill_kl for callers that cannot allocate.

@@ -6,7 +6,11 @@ fallback here: if ``libsai.so`` is missing the import fails.
 
     window_lse(Q, Kw, W, scale, doc_start=None)                -> [B,S,H] fp32
     distill_target(Q, pool, idx, wl, cr, scale, sink=None, doc_start=None, err=None) -> [B,S,K] fp32
-    distill_kl(p, scores, valid, coeff, want_grad=True, workspace=None) -> (loss[1], dscores)
+    distill_kl(p, scores, valid, coeff, want_grad=True, workspace=None, n_rows=None) -> (loss[1], dscores)
+
+The token-range calls (window_lse_range, distill_target_range,
+count_valid_rows) serve a batch split across GPUs by sequence position; see
+shard.py for the call sequence.
 
 bf16 tensors may be passed as torch.bfloat16 or as int16/uint16 bit patterns.
 """
@@ -59,6 +63,15 @@ _lib.sai_distill_kl_workspace_bytes.argtypes = [_I, _I, _I]
 _lib.sai_distill_kl_workspace_bytes.restype = ctypes.c_size_t
 _lib.sai_distill_kl.argtypes = [_P, _P, _P, _I, _I, _I, _F, _P, _P, _P, ctypes.c_size_t, _P]
 _lib.sai_distill_kl.restype = _I
+_lib.sai_window_lse_range.argtypes = [_P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P, _P]
+_lib.sai_window_lse_range.restype = _I
+_lib.sai_distill_target_range.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F,
+                                          ctypes.c_uint, _P, _P, _P]
+_lib.sai_distill_target_range.restype = _I
+_lib.sai_count_valid_rows.argtypes = [_P, _I, _I, _I, _P, _P]
+_lib.sai_count_valid_rows.restype = _I
+_lib.sai_distill_kl_ex.argtypes = [_P, _P, _P, _I, _I, _I, _F, _P, _P, _P, _P, ctypes.c_size_t, _P]
+_lib.sai_distill_kl_ex.restype = _I
 _lib.sai_distill_kl_noalloc.argtypes = [_P, _P, _P, _I, _I, _I, _F, _P, _P, _P]
 _lib.sai_distill_kl_noalloc.restype = _I
 _lib.sai_distill_kl_noalloc_max_scratch_bytes.argtypes = []
@@ -149,15 +162,36 @@ def window_lse(Q: torch.Tensor, Kw: torch.Tensor, W: int, scale: float,
     return out
 
 
-def _target_inputs(Q, pool, idx, wl, cr, sink, doc_start, err, per_branch, full_lse):
+def window_lse_range(Q: torch.Tensor, Kw: torch.Tensor, W: int, scale: float, t_begin: int, kw_lead: int,
+                     doc_start: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """window_lse for sequence positions t_begin .. t_begin+S-1, through
+    sai_window_lse_range. Q is the range's [B,S,H,D]; Kw [B,S+kw_lead,D] holds
+    the keys from position t_begin-kw_lead on (the range and its halo)."""
+    B, S, H, D = Q.shape
+    Q = _bf16_bits(Q, "Q")
+    Kw = _bf16_bits(Kw, "Kw")
+    if tuple(Kw.shape) != (B, S + kw_lead, D):
+        raise ValueError(f"Kw must be [B,S+kw_lead,D] = {(B, S + kw_lead, D)}, got {tuple(Kw.shape)}")
+    _want(doc_start, "doc_start", torch.int32, (B, S))
+    if out is None:
+        out = torch.empty((B, S, H), dtype=torch.float32, device=Q.device)
+    _want(out, "out", torch.float32, (B, S, H))
+    st = _call(_lib.sai_window_lse_range, Q.device, _ptr(Q), _ptr(Kw), _ptr(doc_start), B, S, H, D, int(W),
+               int(t_begin), int(kw_lead), float(scale), _ptr(out))
+    _check(st, "sai_window_lse_range")
+    return out
+
+
+def _target_inputs(Q, pool, idx, wl, cr, sink, doc_start, err, per_branch, full_lse, S_seq=None):
     """Checked arguments shared by the target entry points:
     (Q bits, pool bits, K, wl, sink, flags)."""
     B, S, H, D = Q.shape
-    K = idx.shape[-1] if idx is not None else S // cr
+    S_seq = S if S_seq is None else S_seq
+    K = idx.shape[-1] if idx is not None else S_seq // cr
     Q = _bf16_bits(Q, "Q")
     pool = _bf16_bits(pool, "pool")
-    if tuple(pool.shape) != (B, S // cr, D):
-        raise ValueError("pool must be [B,S/cr,D]")
+    if tuple(pool.shape) != (B, S_seq // cr, D):
+        raise ValueError("pool must be [B,S_seq/cr,D]")
     _want(idx, "idx", torch.int32, (B, S, K))
     if per_branch and full_lse:
         raise ValueError("per_branch and full_lse exclude each other")
@@ -197,6 +231,42 @@ def distill_target(Q: torch.Tensor, pool: torch.Tensor, idx: Optional[torch.Tens
     st = _call(_lib.sai_distill_target_ex, Q.device, _ptr(Q), _ptr(pool), _ptr(idx), _ptr(wl), _ptr(sink),
                _ptr(doc_start), B, S, H, D, K, int(cr), float(scale), flags, _ptr(out), _ptr(err))
     _check(st, "sai_distill_target_ex")
+    return out
+
+
+def distill_target_range(Q: torch.Tensor, pool: torch.Tensor, idx: Optional[torch.Tensor],
+                         wl: Optional[torch.Tensor], cr: int, scale: float, S_seq: int, t_begin: int,
+                         sink: Optional[torch.Tensor] = None, doc_start: Optional[torch.Tensor] = None,
+                         err: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
+                         per_branch: bool = False, full_lse: bool = False) -> torch.Tensor:
+    """p for sequence positions t_begin .. t_begin+S-1 of sequences of S_seq
+    tokens, through sai_distill_target_range: Q, idx, wl and doc_start are the
+    range's rows, pool is the whole sequence's [B,S_seq/cr,D]."""
+    B, S, H, D = Q.shape
+    Q, pool, K, wl, sink, flags = _target_inputs(Q, pool, idx, wl, cr, sink, doc_start, err, per_branch,
+                                                 full_lse, S_seq=S_seq)
+    if out is None:
+        out = torch.empty((B, S, K), dtype=torch.float32, device=Q.device)
+    _want(out, "out", torch.float32, (B, S, K))
+    st = _call(_lib.sai_distill_target_range, Q.device, _ptr(Q), _ptr(pool), _ptr(idx), _ptr(wl), _ptr(sink),
+               _ptr(doc_start), B, S, int(S_seq), int(t_begin), H, D, K, int(cr), float(scale), flags,
+               _ptr(out), _ptr(err))
+    _check(st, "sai_distill_target_range")
+    return out
+
+
+def count_valid_rows(valid: torch.Tensor, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """N, the rows of valid [B,S,K] with a valid slot, as a device int32 [1]
+    (sai_count_valid_rows); nothing is read back to the host."""
+    B, S, K = valid.shape
+    if valid.dtype == torch.bool:
+        valid = valid.view(torch.uint8)
+    _want(valid, "valid", torch.uint8, (B, S, K))
+    if out is None:
+        out = torch.empty(1, dtype=torch.int32, device=valid.device)
+    _want(out, "out", torch.int32, (1,))
+    st = _call(_lib.sai_count_valid_rows, valid.device, _ptr(valid), B, S, K, _ptr(out))
+    _check(st, "sai_count_valid_rows")
     return out
 
 
@@ -245,9 +315,13 @@ def kl_workspace_bytes(B: int, S: int, K: int) -> int:
 
 def distill_kl(p: torch.Tensor, scores: torch.Tensor, valid: torch.Tensor, coeff: float,
                want_grad: bool = True, workspace: Optional[torch.Tensor] = None,
-               loss: Optional[torch.Tensor] = None, dscores: Optional[torch.Tensor] = None
-               ) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+               loss: Optional[torch.Tensor] = None, dscores: Optional[torch.Tensor] = None,
+               n_rows: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """(loss[1], dscores) through sai_distill_kl_ex. n_rows (device int32 [1],
+    optional) is the batch-wide N when the batch is split across GPUs; the
+    loss is then this call's share of the batch loss."""
     B, S, K = scores.shape
+    _want(n_rows, "n_rows", torch.int32, (1,))
     _want(p, "p", torch.float32, (B, S, K))
     _want(scores, "scores", torch.float32, (B, S, K))
     if valid.dtype == torch.bool:
@@ -262,9 +336,10 @@ def distill_kl(p: torch.Tensor, scores: torch.Tensor, valid: torch.Tensor, coeff
         dscores = torch.empty((B, S, K), dtype=torch.float32, device=scores.device)
     if not want_grad:
         dscores = None
-    st = _call(_lib.sai_distill_kl, scores.device, _ptr(p), _ptr(scores), _ptr(valid), B, S, K, float(coeff),
-               _ptr(loss), _ptr(dscores), _ptr(workspace), workspace.numel() * workspace.element_size())
-    _check(st, "sai_distill_kl")
+    st = _call(_lib.sai_distill_kl_ex, scores.device, _ptr(p), _ptr(scores), _ptr(valid), B, S, K, float(coeff),
+               _ptr(n_rows), _ptr(loss), _ptr(dscores), _ptr(workspace),
+               workspace.numel() * workspace.element_size())
+    _check(st, "sai_distill_kl_ex")
     return loss, dscores
 
 

@@ -84,6 +84,40 @@ __global__ void __launch_bounds__(kKlThreads)
     }
 }
 
+// Rows with a valid slot, added into *n (zeroed by the caller's stream first).
+__global__ void __launch_bounds__(kKlThreads)
+    count_rows_kernel(const uint8_t *__restrict__ valid, int rows, int K, int32_t *n)
+{
+    __shared__ int wcount[kKlWarps];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    int c = 0;
+    const bool vec = (K & 15) == 0;
+    for (int r = blockIdx.x * kKlWarps + warp; r < rows; r += gridDim.x * kKlWarps) {
+        const uint8_t *vr = valid + (size_t)r * K;
+        bool any = false;
+        if (vec) {
+            for (int k = lane * 16; k < K; k += 32 * 16) {
+                const uint4 x = __ldg(reinterpret_cast<const uint4 *>(vr + k));
+                any |= (x.x | x.y | x.z | x.w) != 0;
+            }
+        } else {
+            for (int k = lane; k < K; k += 32)
+                any |= vr[k] != 0;
+        }
+        c += __any_sync(0xffffffffu, any) ? 1 : 0;
+    }
+    if (lane == 0)
+        wcount[warp] = c;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int s = 0;
+        for (int i = 0; i < kKlWarps; ++i)
+            s += wcount[i];
+        if (s)
+            atomicAdd(n, s);
+    }
+}
+
 __device__ __forceinline__ float warp_max(float v)
 {
     for (int o = 16; o >= 1; o >>= 1)
@@ -224,7 +258,8 @@ __device__ __forceinline__ float kl_row_any(const float *__restrict__ pr, const 
 template <int NV>
 __global__ void __launch_bounds__(kKlThreads, 4)
     kl_rows_kernel(const float *__restrict__ p, const float *__restrict__ scores, const uint8_t *__restrict__ valid,
-                   int rows, int K, float coeff, float *loss, float *dscores, void *ws, int count_blocks)
+                   int rows, int K, float coeff, float *loss, float *dscores, void *ws, int count_blocks,
+                   const int32_t *n_given)
 {
     KlWs w = ws_layout(ws, count_blocks);
     __shared__ double wkl[kKlWarps];
@@ -232,16 +267,18 @@ __global__ void __launch_bounds__(kKlThreads, 4)
     __shared__ bool last;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-    // N = number of valid rows, from the count kernel's partials.
+    // N = number of valid rows: the caller's (e.g. summed over ranks), else
+    // from the count kernel's partials.
     int n = 0;
-    for (int i = threadIdx.x; i < count_blocks; i += blockDim.x)
-        n += w.count_part[i];
+    if (!n_given)
+        for (int i = threadIdx.x; i < count_blocks; i += blockDim.x)
+            n += w.count_part[i];
     for (int o = 16; o >= 1; o >>= 1)
         n += __shfl_xor_sync(0xffffffffu, n, o);
     if (threadIdx.x == 0)
-        nshare = 0;
+        nshare = n_given ? *n_given : 0;
     __syncthreads();
-    if (lane == 0)
+    if (lane == 0 && !n_given)
         atomicAdd(&nshare, n);
     __syncthreads();
     const int N = nshare;
@@ -314,26 +351,44 @@ cudaError_t launch_kl_count(const KlPlan &pl, const uint8_t *valid, void *ws, cu
     return cudaGetLastError();
 }
 
-cudaError_t launch_distill_kl(const KlPlan &pl, const float *p, const float *scores, const uint8_t *valid,
-                              float coeff, float *loss, float *dscores, void *ws, cudaStream_t stream)
+cudaError_t launch_count_rows(const uint8_t *valid, int rows, int K, int32_t *n, cudaStream_t stream)
 {
-    kl_count_kernel<<<pl.count_blocks, kKlThreads, 0, stream>>>(valid, pl.rows, pl.K, ws, pl.count_blocks);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = cudaMemsetAsync(n, 0, sizeof(int32_t), stream);
+    if (e != cudaSuccess)
+        return e;
+    const int need = (rows + kKlWarps - 1) / kKlWarps;
+    const int blocks = need < kKlMaxBlocks ? (need > 0 ? need : 1) : kKlMaxBlocks;
+    count_rows_kernel<<<blocks, kKlThreads, 0, stream>>>(valid, rows, K, n);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_distill_kl(const KlPlan &pl, const float *p, const float *scores, const uint8_t *valid,
+                              float coeff, float *loss, float *dscores, void *ws, cudaStream_t stream,
+                              const int32_t *n_given)
+{
+    cudaError_t e;
+    if (n_given) {
+        // N is the caller's: only the completion counter needs resetting
+        e = cudaMemsetAsync(ws, 0, 16, stream);
+    } else {
+        kl_count_kernel<<<pl.count_blocks, kKlThreads, 0, stream>>>(valid, pl.rows, pl.K, ws, pl.count_blocks);
+        e = cudaGetLastError();
+    }
     if (e != cudaSuccess)
         return e;
     const int K = pl.K;
     if ((K & 3) == 0 && K <= 128)
         kl_rows_kernel<1><<<pl.row_blocks, kKlThreads, 0, stream>>>(p, scores, valid, pl.rows, K, coeff, loss,
-                                                                     dscores, ws, pl.count_blocks);
+                                                                     dscores, ws, pl.count_blocks, n_given);
     else if ((K & 3) == 0 && K <= 256)
         kl_rows_kernel<2><<<pl.row_blocks, kKlThreads, 0, stream>>>(p, scores, valid, pl.rows, K, coeff, loss,
-                                                                     dscores, ws, pl.count_blocks);
+                                                                     dscores, ws, pl.count_blocks, n_given);
     else if ((K & 3) == 0 && K <= 512)
         kl_rows_kernel<4><<<pl.row_blocks, kKlThreads, 0, stream>>>(p, scores, valid, pl.rows, K, coeff, loss,
-                                                                     dscores, ws, pl.count_blocks);
+                                                                     dscores, ws, pl.count_blocks, n_given);
     else
         kl_rows_kernel<0><<<pl.row_blocks, kKlThreads, 0, stream>>>(p, scores, valid, pl.rows, K, coeff, loss,
-                                                                     dscores, ws, pl.count_blocks);
+                                                                     dscores, ws, pl.count_blocks, n_given);
     return cudaGetLastError();
 }
 

@@ -36,27 +36,29 @@ __device__ __forceinline__ float block_sum(float v, float *scratch)
 
 __global__ void __launch_bounds__(kGenThreads)
     window_lse_generic_kernel(const uint16_t *__restrict__ Q, const uint16_t *__restrict__ Kw,
-                              const int32_t *__restrict__ doc_start, int S, int H, int D, int W, float scale,
-                              float *__restrict__ out)
+                              const int32_t *__restrict__ doc_start, int S, int H, int D, int W, int t_begin,
+                              int kw_lead, float scale, float *__restrict__ out)
 {
     extern __shared__ float gsm[];
     float *qs = gsm;               // [H][D]
     float *zs = qs + H * D;        // [H][W]
     const int g = blockIdx.x;
-    const int b = g / S, t = g - b * S;
+    const int b = g / S;
+    const int t = g - b * S + t_begin;   // sequence position
     int d0 = 0;
     if (doc_start) {
         d0 = doc_start[g];
         d0 = d0 < 0 ? 0 : (d0 > t ? t : d0);
     }
-    const int lo = max(d0, t - W + 1);
+    const int lo = max(max(d0, t - W + 1), t_begin - kw_lead);
     const int nw = t - lo + 1;
     for (int i = threadIdx.x; i < H * D; i += blockDim.x)
         qs[i] = bf16f(Q[(size_t)g * H * D + i]);
     __syncthreads();
     for (int pr = threadIdx.x; pr < H * nw; pr += blockDim.x) {
         const int h = pr / nw, s = lo + pr % nw;
-        const uint16_t *k = Kw + ((size_t)b * S + s) * D;
+        // Kw is [B, S + kw_lead, D]; position s is row s - t_begin + kw_lead
+        const uint16_t *k = Kw + ((size_t)b * (S + kw_lead) + (s - t_begin + kw_lead)) * D;
         float acc = 0.f;
         for (int d = 0; d < D; ++d)
             acc = fmaf(qs[h * D + d], bf16f(k[d]), acc);
@@ -83,8 +85,9 @@ __global__ void __launch_bounds__(kGenThreads)
 __global__ void __launch_bounds__(kGenThreads)
     target_generic_kernel(const uint16_t *__restrict__ Q, const uint16_t *__restrict__ pool,
                           const int32_t *__restrict__ idx, const float *__restrict__ wl,
-                          const float *__restrict__ sink, const int32_t *__restrict__ doc_start, int S, int H,
-                          int D, int K, int cr, float scale, int lse_mode, float *__restrict__ p, int32_t *err)
+                          const float *__restrict__ sink, const int32_t *__restrict__ doc_start, int S, int P,
+                          int t_begin, int H, int D, int K, int cr, float scale, int lse_mode,
+                          float *__restrict__ p, int32_t *err)
 {
     extern __shared__ float gsm[];
     float *qs = gsm;                              // [H][D]
@@ -97,8 +100,8 @@ __global__ void __launch_bounds__(kGenThreads)
     int *slots = rows + K;                        // [K]
     int *cnt = slots + K;                         // [1]
     const int g = blockIdx.x;
-    const int b = g / S, t = g - b * S;
-    const int P = S / cr;
+    const int b = g / S;
+    const int t = g - b * S + t_begin;   // sequence position
     int d0 = 0;
     if (doc_start) {
         d0 = doc_start[g];
@@ -187,14 +190,16 @@ __global__ void __launch_bounds__(kGenThreads)
 size_t window_simt_smem_bytes(int H, int D, int W) { return (size_t)(H * D + H * W) * 4; }
 
 cudaError_t launch_window_lse_simt(const uint16_t *Q, const uint16_t *Kw, const int32_t *doc_start, int B, int S,
-                                   int H, int D, int W, float scale, float *out, cudaStream_t stream)
+                                   int H, int D, int W, int t_begin, int kw_lead, float scale, float *out,
+                                   cudaStream_t stream)
 {
     const size_t smem = window_simt_smem_bytes(H, D, W);
     cudaError_t e = cudaFuncSetAttribute(window_lse_generic_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess)
         return e;
-    window_lse_generic_kernel<<<B * S, kGenThreads, smem, stream>>>(Q, Kw, doc_start, S, H, D, W, scale, out);
+    window_lse_generic_kernel<<<B * S, kGenThreads, smem, stream>>>(Q, Kw, doc_start, S, H, D, W, t_begin, kw_lead,
+                                                                    scale, out);
     return cudaGetLastError();
 }
 
@@ -204,8 +209,8 @@ size_t target_simt_smem_bytes(int H, int D, int K)
 }
 
 cudaError_t launch_target_simt(const uint16_t *Q, const uint16_t *pool, const int32_t *idx, const float *wl,
-                               const float *sink, const int32_t *doc_start, int B, int S, int H, int D, int K,
-                               int cr, float scale, int lse_mode, float *p, int32_t *err,
+                               const float *sink, const int32_t *doc_start, int B, int S, int P, int t_begin,
+                               int H, int D, int K, int cr, float scale, int lse_mode, float *p, int32_t *err,
                                cudaStream_t stream)
 {
     const size_t smem = target_simt_smem_bytes(H, D, K);
@@ -213,8 +218,8 @@ cudaError_t launch_target_simt(const uint16_t *Q, const uint16_t *pool, const in
         cudaFuncSetAttribute(target_generic_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess)
         return e;
-    target_generic_kernel<<<B * S, kGenThreads, smem, stream>>>(Q, pool, idx, wl, sink, doc_start, S, H, D, K, cr,
-                                                                scale, lse_mode, p, err);
+    target_generic_kernel<<<B * S, kGenThreads, smem, stream>>>(Q, pool, idx, wl, sink, doc_start, S, P, t_begin, H,
+                                                                D, K, cr, scale, lse_mode, p, err);
     return cudaGetLastError();
 }
 

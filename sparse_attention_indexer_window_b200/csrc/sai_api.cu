@@ -97,18 +97,23 @@ const char *sai_status_string(int status)
 
 int sai_version(void) { return 200; }
 
-sai_status sai_window_lse(const uint16_t *Q, const uint16_t *Kw, const int32_t *doc_start, int B, int S, int H,
-                          int D, int W, float scale, float *window_lse, void *stream)
+namespace {
+
+sai_status window_impl(const uint16_t *Q, const uint16_t *Kw, const int32_t *doc_start, int B, int S, int H, int D,
+                       int W, int t_begin, int kw_lead, float scale, float *window_lse, cudaStream_t st)
 {
     if (!Q || !Kw || !window_lse)
         return SAI_ERR_NULL;
     if (B < 1 || S < 1 || H < 1 || D < 1 || W < 1 || (D % 8) != 0 || !isfinite(scale) || scale <= 0.f)
         return SAI_ERR_SHAPE;
-    if ((int64_t)B * S * H * D > INT32_MAX || (int64_t)B * S * H > INT32_MAX)
+    // a range needs every key its first token's window can reach
+    if (t_begin < 0 || kw_lead < 0 || kw_lead > t_begin || kw_lead < std::min(W - 1, t_begin))
+        return SAI_ERR_SHAPE;
+    if ((int64_t)B * S * H * D > INT32_MAX || (int64_t)B * S * H > INT32_MAX ||
+        (int64_t)t_begin + S > INT32_MAX || (int64_t)B * (S + kw_lead) * D > INT32_MAX)
         return SAI_ERR_SHAPE;
     if (!al16(Q) || !al16(Kw) || !al4(window_lse) || (doc_start && !al4(doc_start)))
         return SAI_ERR_ALIGN;
-    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const int smem_cap = max_smem_optin();
 
     if (tc_heads(H) && (D % 64) == 0 && S % (128 / H) == 0 && W + 128 / H - 1 <= 256) {
@@ -118,6 +123,8 @@ sai_status sai_window_lse(const uint16_t *Q, const uint16_t *Kw, const int32_t *
         a.H = H;
         a.D = D;
         a.W = W;
+        a.t_begin = t_begin;
+        a.kw_lead = kw_lead;
         a.TQ = 128 / H;
         a.NB = ((W + a.TQ - 1) + 15) / 16 * 16;
         a.n_tiles = B * S / a.TQ;
@@ -129,7 +136,7 @@ sai_status sai_window_lse(const uint16_t *Q, const uint16_t *Kw, const int32_t *
             return SAI_ERR_UNSUPPORTED;
         CUtensorMap mq, mk;
         if (!make_map_bf16(&mq, Q, (uint64_t)B * S * H, D, 128) ||
-            !make_map_bf16(&mk, Kw, (uint64_t)B * S, D, (uint32_t)a.NB))
+            !make_map_bf16(&mk, Kw, (uint64_t)B * (S + kw_lead), D, (uint32_t)a.NB))
             return SAI_ERR_CUDA;
         int grid = sm_count();
         if (grid <= 0)
@@ -139,8 +146,26 @@ sai_status sai_window_lse(const uint16_t *Q, const uint16_t *Kw, const int32_t *
         return cuda_status(sai::launch_window_lse_tc(mq, mk, a, grid, st));
     }
     if ((int)sai::window_simt_smem_bytes(H, D, W) <= smem_cap)
-        return cuda_status(sai::launch_window_lse_simt(Q, Kw, doc_start, B, S, H, D, W, scale, window_lse, st));
+        return cuda_status(sai::launch_window_lse_simt(Q, Kw, doc_start, B, S, H, D, W, t_begin, kw_lead, scale,
+                                                       window_lse, st));
     return SAI_ERR_UNSUPPORTED;
+}
+
+}  // namespace
+
+sai_status sai_window_lse(const uint16_t *Q, const uint16_t *Kw, const int32_t *doc_start, int B, int S, int H,
+                          int D, int W, float scale, float *window_lse, void *stream)
+{
+    return window_impl(Q, Kw, doc_start, B, S, H, D, W, 0, 0, scale, window_lse,
+                       reinterpret_cast<cudaStream_t>(stream));
+}
+
+sai_status sai_window_lse_range(const uint16_t *Q, const uint16_t *Kw, const int32_t *doc_start, int B, int S,
+                                int H, int D, int W, int t_begin, int kw_lead, float scale, float *window_lse,
+                                void *stream)
+{
+    return window_impl(Q, Kw, doc_start, B, S, H, D, W, t_begin, kw_lead, scale, window_lse,
+                       reinterpret_cast<cudaStream_t>(stream));
 }
 
 sai_status sai_distill_target(const uint16_t *Q, const uint16_t *pool, const int32_t *idx, const float *window_lse,
@@ -175,9 +200,12 @@ size_t fused_ws_bytes(const sai::KlPlan &pl)
     return a + parts;
 }
 
+// S local tokens per sequence starting at position t_begin of sequences of
+// S_seq tokens (the whole sequence: S_seq == S, t_begin == 0).
 sai_status target_impl(const uint16_t *Q, const uint16_t *pool, const int32_t *idx, const float *window_lse,
-                       const float *sink, const int32_t *doc_start, int B, int S, int H, int D, int K, int cr,
-                       float scale, unsigned flags, float *p, int32_t *d_err, cudaStream_t st, const KlFuse *kf)
+                       const float *sink, const int32_t *doc_start, int B, int S, int S_seq, int t_begin, int H,
+                       int D, int K, int cr, float scale, unsigned flags, float *p, int32_t *d_err,
+                       cudaStream_t st, const KlFuse *kf)
 {
     if ((flags & ~(SAI_TARGET_PER_BRANCH | SAI_TARGET_FULL_LSE)) ||
         (flags & (SAI_TARGET_PER_BRANCH | SAI_TARGET_FULL_LSE)) == (SAI_TARGET_PER_BRANCH | SAI_TARGET_FULL_LSE))
@@ -192,10 +220,12 @@ sai_status target_impl(const uint16_t *Q, const uint16_t *pool, const int32_t *i
     // idx NULL: dense over all blocks; p may be NULL only when the KL is fused
     if (!Q || !pool || (!window_lse && !per_branch) || (!p && !kf))
         return SAI_ERR_NULL;
-    if (B < 1 || S < 1 || H < 1 || D < 1 || K < 1 || cr < 1 || (D % 8) != 0 || (S % cr) != 0 ||
+    if (B < 1 || S < 1 || H < 1 || D < 1 || K < 1 || cr < 1 || (D % 8) != 0 || S_seq < 1 || (S_seq % cr) != 0 ||
         !isfinite(scale) || scale <= 0.f)
         return SAI_ERR_SHAPE;
-    const int P = S / cr;
+    if (t_begin < 0 || (int64_t)t_begin + S > S_seq)
+        return SAI_ERR_SHAPE;
+    const int P = S_seq / cr;
     if (K > P)
         return SAI_ERR_SHAPE;
     if ((int64_t)B * S * H * D > INT32_MAX || (int64_t)B * S * K > INT32_MAX)
@@ -221,6 +251,7 @@ sai_status target_impl(const uint16_t *Q, const uint16_t *pool, const int32_t *i
         a.K = K;
         a.cr = cr;
         a.P = P;
+        a.t_begin = t_begin;
         a.n_tok = B * S;
         a.tiles_per_group = 256 / H;
         a.idx_bulk = (idx && (K % 4) == 0 && al16(idx)) ? 1 : 0;
@@ -275,8 +306,8 @@ sai_status target_impl(const uint16_t *Q, const uint16_t *pool, const int32_t *i
         if (e != SAI_OK || fuse_here || !kf)
             return e;
     } else if ((int)sai::target_simt_smem_bytes(H, D, K) <= smem_cap) {
-        sai_status e = cuda_status(sai::launch_target_simt(Q, pool, idx, window_lse, sink, doc_start, B, S, H, D, K,
-                                                           cr, scale, lse_mode, p, d_err, st));
+        sai_status e = cuda_status(sai::launch_target_simt(Q, pool, idx, window_lse, sink, doc_start, B, S, P,
+                                                           t_begin, H, D, K, cr, scale, lse_mode, p, d_err, st));
         if (e != SAI_OK || !kf)
             return e;
     } else {
@@ -294,8 +325,17 @@ sai_status sai_distill_target_ex(const uint16_t *Q, const uint16_t *pool, const 
                                  int H, int D, int K, int cr, float scale, unsigned flags, float *p, int32_t *d_err,
                                  void *stream)
 {
-    return target_impl(Q, pool, idx, window_lse, sink, doc_start, B, S, H, D, K, cr, scale, flags, p, d_err,
+    return target_impl(Q, pool, idx, window_lse, sink, doc_start, B, S, S, 0, H, D, K, cr, scale, flags, p, d_err,
                        reinterpret_cast<cudaStream_t>(stream), nullptr);
+}
+
+sai_status sai_distill_target_range(const uint16_t *Q, const uint16_t *pool, const int32_t *idx,
+                                    const float *window_lse, const float *sink, const int32_t *doc_start, int B,
+                                    int S, int S_seq, int t_begin, int H, int D, int K, int cr, float scale,
+                                    unsigned flags, float *p, int32_t *d_err, void *stream)
+{
+    return target_impl(Q, pool, idx, window_lse, sink, doc_start, B, S, S_seq, t_begin, H, D, K, cr, scale, flags,
+                       p, d_err, reinterpret_cast<cudaStream_t>(stream), nullptr);
 }
 
 size_t sai_distill_target_kl_workspace_bytes(int B, int S, int K)
@@ -327,7 +367,7 @@ sai_status sai_distill_target_kl(const uint16_t *Q, const uint16_t *pool, const 
     kf.plan = sai::kl_plan(B, S, K);
     if (!workspace || !al16(workspace) || ws_bytes < fused_ws_bytes(kf.plan))
         return SAI_ERR_WORKSPACE;
-    return target_impl(Q, pool, idx, window_lse, sink, doc_start, B, S, H, D, K, cr, scale, flags, p, d_err,
+    return target_impl(Q, pool, idx, window_lse, sink, doc_start, B, S, S, 0, H, D, K, cr, scale, flags, p, d_err,
                        reinterpret_cast<cudaStream_t>(stream), &kf);
 }
 size_t sai_distill_kl_workspace_bytes(int B, int S, int K)
@@ -341,6 +381,26 @@ sai_status sai_distill_kl(const float *p, const float *scores, const uint8_t *va
                           float coeff, float *loss, float *dscores, void *workspace, size_t ws_bytes,
                           void *stream)
 {
+    return sai_distill_kl_ex(p, scores, valid, B, S, K, coeff, nullptr, loss, dscores, workspace, ws_bytes, stream);
+}
+
+sai_status sai_count_valid_rows(const uint8_t *valid, int B, int S, int K, int32_t *n_rows, void *stream)
+{
+    if (!valid || !n_rows)
+        return SAI_ERR_NULL;
+    if (B < 1 || S < 1 || K < 1 || (int64_t)B * S * K > INT32_MAX)
+        return SAI_ERR_SHAPE;
+    if (!al16(valid) || !al4(n_rows))
+        return SAI_ERR_ALIGN;
+    return cuda_status(sai::launch_count_rows(valid, B * S, K, n_rows, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+sai_status sai_distill_kl_ex(const float *p, const float *scores, const uint8_t *valid, int B, int S, int K,
+                             float coeff, const int32_t *n_rows, float *loss, float *dscores, void *workspace,
+                             size_t ws_bytes, void *stream)
+{
+    if (n_rows && !al4(n_rows))
+        return SAI_ERR_ALIGN;
     if (!p || !scores || !valid || !loss)
         return SAI_ERR_NULL;
     if (B < 1 || S < 1 || K < 1 || !isfinite(coeff) || (int64_t)B * S * K > INT32_MAX)
@@ -351,7 +411,7 @@ sai_status sai_distill_kl(const float *p, const float *scores, const uint8_t *va
     if (!workspace || !al16(workspace) || ws_bytes < pl.ws_bytes)
         return SAI_ERR_WORKSPACE;
     return cuda_status(sai::launch_distill_kl(pl, p, scores, valid, coeff, loss, dscores, workspace,
-                                              reinterpret_cast<cudaStream_t>(stream)));
+                                              reinterpret_cast<cudaStream_t>(stream), n_rows));
 }
 
 sai_status sai_indexer_topk(const float *index_scores, const int32_t *doc_start, int B, int S, int cr, int K,

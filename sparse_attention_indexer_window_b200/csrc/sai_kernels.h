@@ -12,6 +12,8 @@ namespace sai {
 // ---------------------------------------------------------------- window_lse
 struct WinTcArgs {
     int B, S, H, D, W;
+    int t_begin;          // sequence position of local token 0 (token-range calls; else 0)
+    int kw_lead;          // Kw rows per sequence before local token 0 (Kw holds S + kw_lead rows)
     int TQ;               // tokens per 128-row tile (128 / H)
     int NB;               // band rows = roundup16(W + TQ - 1), <= 256
     int n_tiles;          // B*S / TQ
@@ -32,7 +34,8 @@ enum : int {
     kLseGiven = 2,      // wl holds lse_full itself; floor FLT_MIN; sink unused
 };
 struct TgtTcArgs {
-    int B, S, H, D, K, cr, P;
+    int B, S, H, D, K, cr, P;   // P = pool rows per sequence (sequence length / cr)
+    int t_begin;          // sequence position of local token 0 (token-range calls; else 0)
     int n_tok;            // B*S
     int tiles_per_group;  // 128-slot tiles per TMEM accumulator (256 / H)
     int idx_bulk;         // idx rows are 16-byte aligned (K % 4 == 0): stage them by bulk copy
@@ -68,11 +71,12 @@ cudaError_t launch_target_tc(const CUtensorMap &mapQ, const CUtensorMap &mapP, c
 // For shapes the tensor-core kernels do not take (small H or D).
 size_t window_simt_smem_bytes(int H, int D, int W);
 cudaError_t launch_window_lse_simt(const uint16_t *Q, const uint16_t *Kw, const int32_t *doc_start, int B, int S,
-                                   int H, int D, int W, float scale, float *out, cudaStream_t stream);
+                                   int H, int D, int W, int t_begin, int kw_lead, float scale, float *out,
+                                   cudaStream_t stream);
 size_t target_simt_smem_bytes(int H, int D, int K);
 cudaError_t launch_target_simt(const uint16_t *Q, const uint16_t *pool, const int32_t *idx, const float *wl,
-                               const float *sink, const int32_t *doc_start, int B, int S, int H, int D, int K,
-                               int cr, float scale, int lse_mode, float *p, int32_t *err,
+                               const float *sink, const int32_t *doc_start, int B, int S, int P, int t_begin,
+                               int H, int D, int K, int cr, float scale, int lse_mode, float *p, int32_t *err,
                                cudaStream_t stream);
 
 // ---------------------------------------------------------------- distill_kl
@@ -86,7 +90,12 @@ KlPlan kl_plan(int B, int S, int K);
 // Per-block counts of rows with a valid slot into the KL workspace (its
 // layout: completion counter at byte 0, which this resets, counts at byte 16).
 cudaError_t launch_kl_count(const KlPlan &pl, const uint8_t *valid, void *ws, cudaStream_t stream);
+// n_given: device int32 holding N (rows with a valid slot over the whole
+// batch, e.g. summed over ranks); NULL: counted here from `valid`.
 cudaError_t launch_distill_kl(const KlPlan &pl, const float *p, const float *scores, const uint8_t *valid,
-                              float coeff, float *loss, float *dscores, void *ws, cudaStream_t stream);
+                              float coeff, float *loss, float *dscores, void *ws, cudaStream_t stream,
+                              const int32_t *n_given = nullptr);
+// *n = rows of `valid` [rows, K] with a valid slot (the stream zeroes *n first).
+cudaError_t launch_count_rows(const uint8_t *valid, int rows, int K, int32_t *n, cudaStream_t stream);
 
 }  // namespace sai

@@ -230,7 +230,7 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
         for (int gt = blockIdx.x; gt < a.n_tok && ok; gt += gridDim.x, ++it) {
             const int g = a.n_tok - 1 - gt;
             const int b = g / a.S;
-            const int t = g - b * a.S;
+            const int t = g - b * a.S + a.t_begin;   // sequence position
             const int m3 = it % kMeta;
             int32_t *ib = idxs + (it % 3) * Kp;
             stage_idx(gt + 2 * (int)gridDim.x, (it + 2) % 3);

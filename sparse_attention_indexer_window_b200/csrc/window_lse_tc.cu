@@ -1,7 +1,9 @@
 // Banded sliding-window log-mass on tcgen05 tensor cores (sm_100a).
 //
 // Computes window_lse[b,t,h] = log sum_{s=lo}^{t} exp(scale <Q[b,t,h],Kw[b,s]>),
-// lo = max(d0, t-W+1): the log mass of the sliding-window keys that the joint
+// lo = max(d0, t-W+1) (t, s and d0 are sequence positions; a token-range call
+// covers positions t_begin .. t_begin+S-1 with Kw holding kw_lead keys before
+// them): the log mass of the sliding-window keys that the joint
 // softmax of a CSA layer carries in its denominator (Primus page "perf(
 // deepseek-v4): fuse and enable the indexer distillation loss", second commit
 // message: computing the window mass eagerly materialises per-head window
@@ -100,7 +102,8 @@ __global__ void __launch_bounds__(kWinThreads, 1)
                 const int b = g0 / a.S;
                 const int t0 = g0 - b * a.S;
                 const int rowQ = g0 * a.H;
-                const int rowK = b * a.S + t0 - a.W + 1;
+                // Kw is [B, S + kw_lead, D]: local token t sits at Kw row t + kw_lead
+                const int rowK = b * (a.S + a.kw_lead) + t0 + a.kw_lead - a.W + 1;
                 for (int c = 0; c < n_chunks; c += cps) {
                     if (!mbar_wait(&sm->empty[stage], phase ^ 1u, abort_flag, nullptr)) {
                         ok = false;
@@ -194,13 +197,14 @@ __global__ void __launch_bounds__(kWinThreads, 1)
             const int g0 = tile * a.TQ;
             const int g = g0 + rt;
             const int b = g0 / a.S;
-            const int t = g - b * a.S;
-            const int t0 = g0 - b * a.S;
+            const int t = g - b * a.S + a.t_begin;       // sequence positions
+            const int t0 = g0 - b * a.S + a.t_begin;
             int d0 = 0;
             if (a.doc_start) {
                 d0 = a.doc_start[g];
                 d0 = d0 < 0 ? 0 : (d0 > t ? t : d0);
             }
+            d0 = max(d0, a.t_begin - a.kw_lead);         // the first key the caller passed
             if (!mbar_wait(&sm->acc_full[wg], uses & 1, abort_flag, nullptr)) {
                 a.out[(size_t)g * a.H + h] = __int_as_float(0x7fc00000);
                 break;

@@ -1,24 +1,31 @@
 """Host-side plumbing for running the loss data-parallel, one process per GPU.
 
 Every token's target and KL row depend only on that token's own inputs (its
-Q rows, the window keys before it, its idx row) and on its sequence's pool,
-so ranks split the batch by whole sequences and run the three calls on their
-share with nothing exchanged on the data path. What remains for the host:
+Q rows, the W-1 window keys before it, its idx row) and on its sequence's
+pool. So ranks can split a batch two ways:
 
-* which sequences (or, for synthetic runs, which seed) a rank owns;
-* the max over ranks of a device-timed duration (the slowest rank decides);
-* turning per-rank losses, each a mean over that rank's valid rows, into the
-  mean over the whole batch, and the factor that rescales a rank's dscores to
-  match (both are linear in 1/N).
+* by whole sequences (``split_sequences``): each rank runs the three calls on
+  its share, nothing is exchanged on the data path, and per-rank losses are
+  combined afterwards (``global_mean_loss``);
+* by token range within every sequence (``token_ranges``), for batches with
+  fewer sequences than ranks (one long sequence): a rank holds its positions'
+  Q, idx, scores, valid and doc_start rows, the W-1 window keys before its
+  first position (the halo) and the whole pool, and runs the range calls.
+  The one exchange step is N, the batch's count of rows with a valid slot,
+  which every rank's dscores are normalised by: each rank counts its rows on
+  the device, one all-reduce of that integer gives N, and the KL call reads it
+  from device memory (``sharded_distill_loss``).
 
-The collectives here act on a handful of host scalars after the path has run;
-they work with any torch.distributed backend (nccl on GPUs, gloo on CPU).
+Also here: per-rank seeds for synthetic runs and the max over ranks of a
+device-timed duration. The collectives work with any torch.distributed
+backend (nccl on GPUs, gloo on CPU).
 """
 from __future__ import annotations
 
-from typing import Tuple
+from typing import Sequence, Tuple
 
-__all__ = ["rank_seed", "split_sequences", "max_over_ranks", "global_mean_loss"]
+__all__ = ["rank_seed", "split_sequences", "max_over_ranks", "global_mean_loss", "token_cost",
+           "token_ranges", "halo_rows", "range_views", "sharded_distill_loss"]
 
 
 def rank_seed(base_seed: int, rank: int) -> int:
@@ -81,3 +88,91 @@ def global_mean_loss(local_loss: float, local_rows: int, device=None) -> Tuple[f
         kl_sum, rows = float(t[0].item()), int(round(float(t[1].item())))
     n = max(rows, 1)
     return kl_sum / n, n_r / n
+
+
+def token_cost(S: int, cr: int, K: int, W: int):
+    """Relative work of each position t of a sequence: its window keys plus
+    the compressed blocks it can select, min(W, t+1) + min(K, (t+1)//cr)
+    (each costs 2*H*D flops; a sparse selection can leave fewer, never more)."""
+    import numpy as np
+    t = np.arange(S, dtype=np.int64)
+    return np.minimum(W, t + 1) + np.minimum(K, (t + 1) // cr)
+
+
+def token_ranges(S: int, world: int, cost=None) -> Sequence[Tuple[int, int]]:
+    """[t_begin, t_end) for every rank: contiguous, covering 0..S-1, each
+    non-empty when S >= world. With ``cost`` (per position, e.g. token_cost)
+    the cut points split the cumulative cost evenly, so the later positions,
+    which select more blocks, are spread over more ranks; else equal
+    lengths."""
+    if world < 1 or S < 1:
+        raise ValueError(f"need world >= 1 and S >= 1, got world={world} S={S}")
+    import numpy as np
+    if cost is None:
+        cuts = [(S * r) // world for r in range(world + 1)]
+    else:
+        c = np.cumsum(np.asarray(cost, dtype=np.float64))
+        if c.shape != (S,):
+            raise ValueError("cost must hold one value per position")
+        cuts = [0]
+        for r in range(1, world):
+            t = int(np.searchsorted(c, c[-1] * r / world, side="left")) + 1
+            # keep every range non-empty
+            t = max(t, cuts[-1] + 1)
+            t = min(t, S - (world - r))
+            cuts.append(t)
+        cuts.append(S)
+    return [(cuts[r], cuts[r + 1]) for r in range(world)]
+
+
+def halo_rows(t_begin: int, W: int) -> int:
+    """Window keys a range starting at t_begin needs before it."""
+    return min(max(W - 1, 0), t_begin)
+
+
+def range_views(t_begin: int, t_end: int, W: int, Q, Kw, idx, scores, valid, doc_start=None):
+    """The slices of whole-sequence [B,S,...] arrays (numpy or torch) that a
+    rank owning positions [t_begin, t_end) holds: its own rows of Q, idx,
+    scores, valid and doc_start, and Kw from t_begin - halo on. The pool is
+    not sliced: every rank holds the whole pool. Returns a dict with kw_lead."""
+    h = halo_rows(t_begin, W)
+    return {
+        "Q": Q[:, t_begin:t_end],
+        "Kw": Kw[:, t_begin - h:t_end],
+        "idx": None if idx is None else idx[:, t_begin:t_end],
+        "scores": scores[:, t_begin:t_end],
+        "valid": valid[:, t_begin:t_end],
+        "doc_start": None if doc_start is None else doc_start[:, t_begin:t_end],
+        "kw_lead": h,
+        "t_begin": t_begin,
+    }
+
+
+def sharded_distill_loss(calls, view, pool, *, S_seq: int, W: int, cr: int, scale: float, coeff: float,
+                         sink=None, err=None):
+    """One rank's share of the loss over a batch split by token range.
+
+    ``calls`` provides window_lse_range, distill_target_range,
+    count_valid_rows and distill_kl (the package itself on GPUs). ``view`` is
+    this rank's range_views() dict with contiguous tensors. The sequence:
+
+      window_lse_range -> distill_target_range   (this rank's positions)
+      count_valid_rows -> all-reduce(sum)        (N over the whole batch)
+      distill_kl(n_rows=N)                       (dscores with the batch-wide 1/N)
+      all-reduce(sum) of the loss shares         (the batch loss on every rank)
+
+    Returns (loss [1], dscores, p, window_lse) with dscores, p and window_lse
+    for this rank's positions. Every rank must call it (two collectives)."""
+    t_begin = view["t_begin"]
+    wl = calls.window_lse_range(view["Q"], view["Kw"], W, scale, t_begin, view["kw_lead"],
+                                doc_start=view["doc_start"])
+    p = calls.distill_target_range(view["Q"], pool, view["idx"], wl, cr, scale, S_seq, t_begin, sink=sink,
+                                   doc_start=view["doc_start"], err=err)
+    n = calls.count_valid_rows(view["valid"])
+    dist = _dist()
+    if dist is not None and dist.get_world_size() > 1:
+        dist.all_reduce(n, op=dist.ReduceOp.SUM)
+    loss, ds = calls.distill_kl(p, view["scores"], view["valid"], coeff, n_rows=n)
+    if dist is not None and dist.get_world_size() > 1:
+        dist.all_reduce(loss, op=dist.ReduceOp.SUM)
+    return loss, ds, p, wl
