@@ -343,7 +343,10 @@ sai_status sai_distill_kl_ex(const float *p, const float *scores, const uint8_t 
  *
  *   - The first call on each device looks up the array's device address
  *     (cudaGetSymbolAddress) with that device current; make that first call
- *     before any stream capture begins.
+ *     before any stream capture begins. The address is kept for the life of
+ *     the process: after cudaDeviceReset (or anything else that tears down
+ *     and re-creates the device's primary context) it is stale, so do not
+ *     call this entry point again after such a reset.
  *   - Every call on a device shares the one array: calls that overlap on the
  *     GPU (other streams, other host threads) race and can corrupt each
  *     other's loss. Nothing needs clearing between calls.

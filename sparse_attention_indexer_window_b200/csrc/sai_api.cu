@@ -237,7 +237,14 @@ sai_status target_impl(const uint16_t *Q, const uint16_t *pool, const int32_t *i
 
     // the tensor-core kernel addresses pool rows with 32-bit byte offsets
     const bool pool_fits = (uint64_t)B * P * D * 2 < 0xffffffffull;
-    const int n_astages = tc_heads(H) && (D % 64) == 0 && pool_fits ? sai::target_tc_stages(H, K, smem_cap) : 0;
+    // two 64-column chunks of D per pipeline stage where D and shared memory
+    // allow it (half the per-stage synchronisation), else one
+    int cps = (D % 128) == 0 ? 2 : 1;
+    int n_astages = tc_heads(H) && (D % 64) == 0 && pool_fits ? sai::target_tc_stages(H, K, cps, smem_cap) : 0;
+    if (n_astages == 0 && cps == 2) {
+        cps = 1;
+        n_astages = tc_heads(H) && (D % 64) == 0 && pool_fits ? sai::target_tc_stages(H, K, cps, smem_cap) : 0;
+    }
     // the epilogue computes the KL from two slots per thread (K <= 512)
     const bool fuse_here = kf && n_astages > 0 && K <= 512;
     if (kf && !fuse_here && !p)
@@ -256,6 +263,7 @@ sai_status target_impl(const uint16_t *Q, const uint16_t *pool, const int32_t *i
         a.tiles_per_group = 256 / H;
         a.idx_bulk = (idx && (K % 4) == 0 && al16(idx)) ? 1 : 0;
         a.n_astages = n_astages;
+        a.cps = cps;
         a.lse_mode = lse_mode;
         a.pool_box_rows = (int)std::min<int64_t>(128, (int64_t)B * P);
         a.scale = scale;

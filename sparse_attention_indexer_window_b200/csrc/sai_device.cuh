@@ -105,6 +105,18 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
     }
 }
 
+// mbar_wait by a whole warp: every lane runs the same wait, so the warp never
+// splits (a wait taken by one lane and broadcast leaves the warp running as
+// two groups on this part until something reconverges it, and every
+// instruction after it then issues twice). The vote makes the outcome
+// uniform and leaves the warp converged.
+__device__ __forceinline__ bool warp_mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
+                                               int32_t *err)
+{
+    const bool ok = mbar_wait(bar, parity, abort_flag, err);
+    return __all_sync(0xffffffffu, ok);
+}
+
 // Bounded wait used only while unwinding after an abort (short limit, no
 // error reporting): lets in-flight copies land before the CTA exits.
 __device__ __forceinline__ void mbar_drain(uint64_t *bar, uint32_t parity)
@@ -291,6 +303,14 @@ __device__ __forceinline__ float warp_colreduce16(float (&v)[16], Op op)
     }
     const float other = __shfl_xor_sync(0xffffffffu, v[0], 16);
     return op(v[0], other);
+}
+
+// Maximum of v over the 32 lanes of a warp, in every lane (one instruction).
+__device__ __forceinline__ float warp_max_f32(float v)
+{
+    float r;
+    asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(v));
+    return r;
 }
 
 struct OpMax {

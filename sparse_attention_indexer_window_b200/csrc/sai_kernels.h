@@ -39,7 +39,8 @@ struct TgtTcArgs {
     int n_tok;            // B*S
     int tiles_per_group;  // 128-slot tiles per TMEM accumulator (256 / H)
     int idx_bulk;         // idx rows are 16-byte aligned (K % 4 == 0): stage them by bulk copy
-    int n_astages;        // depth of the gathered-row stage ring
+    int n_astages;        // depth of the gathered-row stage ring (divides 8)
+    int cps;              // 64-column chunks of D per stage (1 or 2; D/64 % cps == 0)
     int pool_box_rows;    // rows of the pool's TMA box (min(128, B*P))
     int lse_mode;         // how lse_full is formed: kLseJoint, kLsePerBranch or kLseGiven
     float scale;
@@ -62,8 +63,9 @@ struct TgtTcArgs {
     double *kl_part;            // [grid] per-CTA KL sums
     uint32_t *kl_done;          // completion counter, zeroed by kl_count_kernel
 };
-// Deepest gathered-row stage ring that fits `smem_limit` bytes (0: none).
-int target_tc_stages(int H, int K, int smem_limit);
+// Deepest gathered-row stage ring of `cps`-chunk stages that fits
+// `smem_limit` bytes (0: none).
+int target_tc_stages(int H, int K, int cps, int smem_limit);
 cudaError_t launch_target_tc(const CUtensorMap &mapQ, const CUtensorMap &mapP, const TgtTcArgs &a, int grid,
                              cudaStream_t stream);
 

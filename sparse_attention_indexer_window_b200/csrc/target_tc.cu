@@ -20,19 +20,17 @@
 // Gather. A dedicated warp compacts each token's idx row (selected slots
 // first, masked slots last), up to two tokens ahead; the idx rows arrive by
 // its own cp.async copies, and the compaction turns pool rows into byte
-// offsets. Eight gather warps each own one 16 KB slot of the A ring and fill
-// every stage
-// that lands in it: 128 selected rows x one 128-byte chunk of D, copied into
-// the swizzled K-major operand layout with 16-byte cp.async (eight lanes per
-// row, four rows per instruction, every 128-byte row segment one coalesced
-// request), then wait for their own copies and publish the stage with a
-// single mbarrier arrival. Per-stage synchronisation is thus one wait and one
-// arrival per stage, not per warp and stage; with many warps each sharing
-// every stage that bookkeeping, not the copies, set the pace. A separate warp
-// loads the Q[t] chunks (contiguous) by TMA several chunks ahead. A tile
-// whose selected rows are consecutive pool rows (every tile of an early token
-// under a sorted top-k, whose selection is all causal blocks) is one TMA box
-// instead. Masked slots are never loaded.
+// offsets. A pipeline stage is 128 selected rows x CPS 128-byte chunks of D
+// (CPS = 2 where D allows: 32 KB); the A ring holds NA stages (4 at the
+// V4-Flash shape) and 8 / NA gather warps fill each stage, each its share of
+// the rows, copied into the swizzled K-major operand layout with 16-byte
+// cp.async (eight lanes per row, four rows per instruction, every 128-byte
+// row segment one coalesced request). Each warp waits for its own copies and
+// arrives once on the stage's barrier. A separate warp loads the Q[t] chunks
+// (contiguous) by TMA, CPS chunks per ring entry, several entries ahead. A
+// tile whose selected rows are consecutive pool rows (every tile of an early
+// token under a sorted top-k, whose selection is all causal blocks) is one
+// TMA box per chunk instead. Masked slots are never loaded.
 //
 // The epilogue needs the per-head log-sum-exp over ALL selected slots before
 // it can form u, so a token's scores stay in TMEM until it is done: up to
@@ -64,6 +62,8 @@
 // (heaviest) to the first. All mbarrier waits are bounded; a timeout is
 // reported through err and the CTA unwinds. Named barriers are only used
 // where every participating thread is guaranteed to arrive.
+#include <climits>
+
 #include "sai_device.cuh"
 #include "sai_kernels.h"
 
@@ -87,12 +87,13 @@ constexpr int kLaunchRegs = 96;
 constexpr int kLowRegs = 56;
 constexpr int kHighRegs = 152;
 static_assert(384 * kLowRegs + 256 * kHighRegs <= kTgtThreads * kLaunchRegs, "register split");
-constexpr int kMaxAStages = kGatherWarps;          // one A ring slot per gather warp
+constexpr int kMaxAStages = kGatherWarps;          // at most one A ring slot per gather warp
 constexpr int kQStagesMax = 6;
-// Q[t] chunk ring depth: the Q warp runs this many 64-column chunks ahead
-template <int HH>
-constexpr int q_stages() { return HH <= 64 ? 6 : 3; }
-constexpr int kMeta = 3;                            // compaction runs up to two tokens ahead
+// Q[t] ring: the Q warp runs this many 64-column chunks ahead, in entries of
+// CPS chunks (the chunks one stage's MMAs read); at least two entries.
+template <int HH, int CPS>
+constexpr int q_entries() { return (HH <= 64 ? 6 : 3) / CPS >= 2 ? (HH <= 64 ? 6 : 3) / CPS : 2; }
+constexpr int kMeta = 4;                            // compaction runs up to three tokens ahead
 constexpr uint32_t kATile = 128 * 128;              // 128 rows x 128 bytes
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLnFltMin = -87.33654475055310898657f;  // log(2^-126)
@@ -121,11 +122,13 @@ struct TgtSmem {
     uint32_t tmem_base;
     int abort_flag;
     int nsel[kMeta];
+    int ident[kMeta];     // 1: the selected slots are slots 0..nsel-1 (slot list not written)
+    uint32_t contig[kMeta];  // bit i: tile i's rows are consecutive pool rows (one TMA box per chunk)
     EpiState<HH> epi[1];
 };
 
 // Bytes of dynamic smem other than the A-stage ring.
-template <int HH>
+template <int HH, int CPS>
 __host__ __device__ inline size_t fixed_smem_bytes(int K);
 
 __device__ __forceinline__ int n_groups(int nsel, int TB)
@@ -142,43 +145,52 @@ __device__ __forceinline__ bool selected(int j, int t, int d0, int P, int cr)
 
 // FUSE_KL: the epilogue also computes the KL stage (sai_distill_target_kl);
 // a separate instantiation, so the plain target kernel carries none of it.
-template <int HH, bool FUSE_KL>
+// CPS: 64-column chunks of D per pipeline stage. One stage is CPS x 4 MMAs
+// behind one barrier wait, one fence and one commit; on this part a commit
+// every 4 MMAs leaves the tensor pipe idle about half the time, so CPS = 2
+// whenever D allows it.
+template <int HH, bool FUSE_KL, int CPS>
 __global__ void __launch_bounds__(kTgtThreads, 1)
     target_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapP,
                      const TgtTcArgs a)
 {
     constexpr int TB = 256 / HH;                 // tiles per accumulator
-    constexpr uint32_t kQTile = HH * 128;        // H rows x 128 bytes
+    constexpr uint32_t kQTile = HH * 128;        // one chunk of Q[t]: H rows x 128 bytes
+    constexpr uint32_t kQEntry = CPS * kQTile;   // one Q ring entry
+    constexpr uint32_t kAStage = CPS * kATile;   // one A ring stage: 128 rows x CPS chunks
     constexpr int NC16 = HH / 16;
 
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int K = a.K;
     const int Kp = (K + 3) & ~3;
-    const int NA = a.n_astages;              // A-stage ring depth (sized on the host)
-    uint8_t *a_buf = base;                                                   // NA x 16 KB
-    constexpr int QS = q_stages<HH>();
-    uint8_t *q_buf = a_buf + NA * kATile;                                    // QS x H*128
+    const int NA = a.n_astages;              // A-stage ring depth (sized on the host; divides 8)
+    uint8_t *a_buf = base;                                                   // NA x kAStage
+    constexpr int QS = q_entries<HH, CPS>();
+    uint8_t *q_buf = a_buf + NA * kAStage;                                   // QS x kQEntry
     // byte offset in pool of every selected slot's row, compacted per token
-    uint32_t *rowoff = reinterpret_cast<uint32_t *>(q_buf + QS * kQTile);    // [kMeta][Kp]
+    uint32_t *rowoff = reinterpret_cast<uint32_t *>(q_buf + QS * kQEntry);   // [kMeta][Kp]
     int32_t *slot = reinterpret_cast<int32_t *>(rowoff + kMeta * Kp);        // [kMeta][Kp]
     int32_t *idxs = slot + kMeta * Kp;                                       // [3][Kp] staged idx rows
     float *ubuf = reinterpret_cast<float *>(idxs + 3 * Kp);                  // [Kp] u' of a token
-    TgtSmem<HH> *sm = reinterpret_cast<TgtSmem<HH> *>(ubuf + Kp);
+    // then [2][TB*128] partial u of the two epilogue warpgroups (H >= 32)
+    TgtSmem<HH> *sm = reinterpret_cast<TgtSmem<HH> *>(ubuf + Kp + (HH >= 32 ? 2 * TB * 128 : 0));
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int n_chunks = a.D / 64;
+    const int n_cp = n_chunks / CPS;             // stages per tile (D / 64 is a multiple of CPS)
+    const int WPS = kGatherWarps / NA;           // gather warps filling each A slot
     const bool idx_bulk = a.idx_bulk != 0;       // idx rows staged by bulk copy
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < NA; ++s) {
-            mbar_init(&sm->a_full[s], 1);        // the owning gather warp's lane 0
-            mbar_init(&sm->a_empty[s], 1);
+            mbar_init(&sm->a_full[s], WPS);      // lane 0 of each warp filling the slot
+            mbar_init(&sm->a_empty[s], 2);       // the consumer's commit + the other MMA thread's arrival
         }
         for (int s = 0; s < QS; ++s) {
             mbar_init(&sm->q_full[s], 1);
-            mbar_init(&sm->q_empty[s], 2);      // both MMA threads release a Q chunk
+            mbar_init(&sm->q_empty[s], 2);      // both MMA threads release a Q entry
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&sm->acc_full[b], 2);     // both MMA threads commit a group
@@ -236,9 +248,7 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
             stage_idx(gt + 2 * (int)gridDim.x, (it + 2) % 3);
             cp_async_wait<2>();                  // this token's row has landed
             __syncwarp();
-            if (lane == 0)
-                ok = mbar_wait(&sm->meta_empty[m3], ((it / kMeta) & 1) ^ 1u, abort_flag, a.err);
-            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+            ok = warp_mbar_wait(&sm->meta_empty[m3], ((it / kMeta) & 1) ^ 1u, abort_flag, a.err);
             if (!ok)
                 break;
             int d0 = 0;
@@ -246,13 +256,80 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
                 d0 = a.doc_start[g];
                 d0 = d0 < 0 ? 0 : (d0 > t ? t : d0);
             }
-            // selected slots in order at the front, masked slots from the back;
-            // lane L takes 4 consecutive slots
             uint32_t *rw = rowoff + m3 * Kp;
             int32_t *sl = slot + m3 * Kp;
             const int32_t *grow = a.idx ? a.idx + (size_t)g * K : nullptr;   // NULL: slot k is block k
             int nsel = 0, nmask = 0;
             bool bad = false;
+            // Fast path. When the selected slots are exactly slots 0..n-1 (the
+            // usual layout: valid entries first, -1 or masked entries after),
+            // the compaction is the identity and only the row offsets are
+            // written. Lane L takes 4 consecutive slots per 128-slot tile; a
+            // slot j is selected when lo <= j < hi (the causal and document
+            // bounds of the selection rule, turned into a block interval once
+            // per token). The layout is the identity when the highest
+            // selected slot is nsel - 1. A tile's rows are consecutive pool
+            // rows when idx[k] - k is the same for all its selected slots.
+            const uint32_t rbyte = (uint32_t)a.D * 2u;
+            const uint32_t rbase = (uint32_t)(b * a.P);
+            const int lo = (d0 + a.cr - 1) / a.cr;
+            const int hi = min(a.P, (t + 1) / a.cr);
+            const uint32_t span = hi > lo ? (uint32_t)(hi - lo) : 0u;
+            int cnt = 0, kmax = -1;
+            uint32_t contig = 0;                 // bit i: tile i holds consecutive blocks
+            for (int k0 = 0; k0 < K; k0 += 128) {
+                const int k = k0 + 4 * lane;
+                int j[4];
+                if (idx_bulk) {
+                    int4 v = make_int4(-1, -1, -1, -1);
+                    if (k < K)
+                        v = *reinterpret_cast<const int4 *>(ib + k);
+                    j[0] = v.x;
+                    j[1] = v.y;
+                    j[2] = v.z;
+                    j[3] = v.w;
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        j[e] = (k + e < K) ? (grow ? __ldg(grow + k + e) : k + e) : -1;
+                }
+                int dmin = INT_MAX, dmax = INT_MIN;
+                uint4 ro;
+                uint32_t *rop = &ro.x;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const bool in = k + e < K;
+                    const bool sv = (uint32_t)j[e] - (uint32_t)lo < span;
+                    bad |= in && j[e] != -1 && (uint32_t)j[e] >= (uint32_t)a.P;
+                    cnt += sv ? 1 : 0;
+                    kmax = sv ? k + e : kmax;
+                    const int dd = j[e] - (k + e);
+                    dmin = sv ? min(dmin, dd) : dmin;
+                    dmax = sv ? max(dmax, dd) : dmax;
+                    rop[e] = (rbase + (uint32_t)j[e]) * rbyte;
+                }
+                if (k < K)
+                    *reinterpret_cast<uint4 *>(rw + k) = ro;
+                const int tmin = __reduce_min_sync(0xffffffffu, dmin);
+                const int tmax = __reduce_max_sync(0xffffffffu, dmax);
+                if (tmin == tmax || tmax == INT_MIN)    // one offset, or no selected slot
+                    contig |= 1u << (k0 >> 7);
+            }
+            nsel = __reduce_add_sync(0xffffffffu, cnt);
+            const bool prefix = __reduce_max_sync(0xffffffffu, kmax) + 1 == nsel;
+            if (prefix) {
+                if (lane == 0) {
+                    sm->ident[m3] = 1;
+                    sm->contig[m3] = contig;
+                }
+            } else {
+            nsel = 0;
+            if (lane == 0) {
+                sm->ident[m3] = 0;
+                sm->contig[m3] = 0u;             // general layout: every tile by cp.async
+            }
+            // general case: selected slots in order at the front, masked slots
+            // from the back; lane L takes 4 consecutive slots
             for (int k0 = 0; k0 < K; k0 += 128) {
                 const int k = k0 + 4 * lane;
                 int j[4];
@@ -303,6 +380,7 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
                 nsel += tot & 0xffff;
                 nmask += tot >> 16;
             }
+            }
             if (__any_sync(0xffffffffu, bad) && lane == 0 && a.err)
                 atomicExch(a.err, kErrIndex);
             if (lane == 0)
@@ -310,13 +388,14 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
             __syncwarp();
             if (lane == 0)
                 mbar_arrive(&sm->meta_full[m3]);
+            __syncwarp();
         }
         cp_async_wait<0>();
         __syncwarp();
     } else if (warp == kQWarp) {
         // ============================================================ Q[t] chunks
-        // Every (pass, group, chunk) of a token uses the chunk's H x 64 slice
-        // of Q[t]; this warp loads them by TMA, QS chunks ahead of the MMA.
+        // Every (pass, group, chunk pair) of a token uses CPS H x 64 slices
+        // of Q[t]; this warp loads them by TMA, QS entries ahead of the MMA.
         int qs = 0;
         uint32_t qph = 0;
         uint32_t q_issued = 0, q_last = 0;
@@ -327,26 +406,27 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
         for (int gt = blockIdx.x; gt < a.n_tok && ok; gt += gridDim.x, ++it) {
             const int g = a.n_tok - 1 - gt;
             const int m3 = it % kMeta;
-            if (lane == 0)
-                ok = mbar_wait(&sm->meta_full[m3], (it / kMeta) & 1, abort_flag, a.err);
-            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+            ok = warp_mbar_wait(&sm->meta_full[m3], (it / kMeta) & 1, abort_flag, a.err);
             if (!ok)
                 break;
             const int nsel = sm->nsel[m3];
             const int G = n_groups(nsel, TB);
-            const int nq = (G > 1 ? 2 : 1) * G * n_chunks;
+            const int nq = (G > 1 ? 2 : 1) * G * n_cp;
             for (int qi = 0; qi < nq && ok; ++qi) {
-                const int c = qi % n_chunks;
-                if (lane == 0) {
-                    ok = mbar_wait(&sm->q_empty[qs], qph ^ 1u, abort_flag, a.err);
-                    if (ok) {
-                        mbar_arrive_expect_tx(&sm->q_full[qs], kQTile);
-                        tma_load_2d(q_buf + qs * kQTile, &mapQ, &sm->q_full[qs], c * 64, g * HH);
-                        q_issued |= 1u << qs;
-                        q_last = (q_last & ~(1u << qs)) | (qph << qs);
+                const int c0 = (qi % n_cp) * CPS;
+                ok = warp_mbar_wait(&sm->q_empty[qs], qph ^ 1u, abort_flag, a.err);
+                if (ok) {
+                    if (lane == 0) {
+                        mbar_arrive_expect_tx(&sm->q_full[qs], kQEntry);
+#pragma unroll
+                        for (int cc = 0; cc < CPS; ++cc)
+                            tma_load_2d(q_buf + qs * kQEntry + cc * kQTile, &mapQ, &sm->q_full[qs], (c0 + cc) * 64,
+                                        g * HH);
                     }
+                    __syncwarp();
+                    q_issued |= 1u << qs;
+                    q_last = (q_last & ~(1u << qs)) | (qph << qs);
                 }
-                ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
                 if (++qs == QS) {
                     qs = 0;
                     qph ^= 1u;
@@ -361,16 +441,22 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
         __syncwarp();
     } else if (warp != kMmaWarp && warp != kMmaWarp2 && warp < kEpiWarp0) {
         // ============================================================ gathers
-        // Gather warp gw owns A ring slot gw: it fills every stage that lands
-        // there (stages gw, gw + NA, gw + 2 NA, ... of the MMA's sequence),
-        // waits for its own copies and publishes the stage with one arrival.
-        // Each slot has a single producer, so its phases are seen in order.
+        // Stage k of the MMA sequence lands in slot k % NA of the A ring. The
+        // eight gather warps share the NA slots: warp gw fills part gw / NA
+        // (128 / WPS consecutive rows, all CPS chunks) of every stage that
+        // lands in slot gw % NA, waits for its own copies and arrives once;
+        // the slot's barrier completes when all WPS parts have arrived. Every
+        // producer of a slot waits for the slot's release before refilling it.
         const int gw = warp < kMmaWarp ? warp - 1 : warp - 2;   // 0..7
-        if (gw < NA) {
+        const int aslot = gw % NA;
+        const int part = gw / NA;
+        const int rows_per = 128 / WPS;
+        const int r_lo = part * rows_per;
+        {
             const char *pool_bytes = reinterpret_cast<const char *>(a.pool);
             const int seg = lane & 7;            // 16-byte segment of a 128-byte row chunk
             const int r_in = lane >> 3;          // row within a 4-row group
-            const uint32_t dst0 = smem_u32(a_buf + gw * kATile);
+            const uint32_t dst0 = smem_u32(a_buf + aslot * kAStage);
             const uint32_t row_bytes = (uint32_t)a.D * 2u;
             if (lane == 0)
                 tma_prefetch_desc(&mapP);
@@ -380,12 +466,11 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
             int it = 0;
             for (int gt = blockIdx.x; gt < a.n_tok && ok; gt += gridDim.x, ++it) {
                 const int m3 = it % kMeta;
-                if (lane == 0)
-                    ok = mbar_wait(&sm->meta_full[m3], (it / kMeta) & 1, abort_flag, a.err);
-                ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+                ok = warp_mbar_wait(&sm->meta_full[m3], (it / kMeta) & 1, abort_flag, a.err);
                 if (!ok)
                     break;
                 const int nsel = sm->nsel[m3];
+                const uint32_t tcontig = sm->contig[m3];
                 const uint32_t *rw = rowoff + m3 * Kp;
                 const int nt = (nsel + 127) / 128;
                 const int G = n_groups(nsel, TB);
@@ -394,47 +479,59 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
                     for (int grp = 0; grp < G && ok; ++grp) {
                         const int i0 = grp * TB;
                         const int ntg = min(nt, i0 + TB) - i0;
-                        for (int c = 0; c < n_chunks && ok; ++c) {
+                        for (int cp = 0; cp < n_cp && ok; ++cp) {
                             for (int i = 0; i < ntg; ++i) {
-                                const bool mine = (s == gw);
+                                const bool mine = (s == aslot);
                                 if (++s == NA)
                                     s = 0;
                                 if (!mine)
                                     continue;
-                                if (lane == 0)
-                                    ok = mbar_wait(&sm->a_empty[gw], ph ^ 1u, abort_flag, a.err);
-                                ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+                                ok = warp_mbar_wait(&sm->a_empty[aslot], ph ^ 1u, abort_flag, a.err);
                                 if (!ok)
                                     break;
                                 const int tile_row0 = (i0 + i) * 128;
                                 const int rows = min(128, nsel - tile_row0);
                                 const uint32_t *ro = rw + tile_row0;
-                                // a tile whose rows are consecutive pool rows is one TMA box
-                                const uint32_t ro0 = ro[0];
-                                bool run = true;
-                                for (int q = lane; q < rows; q += 32)
-                                    run = run && ro[q] == ro0 + (uint32_t)q * row_bytes;
-                                if (__all_sync(0xffffffffu, run)) {
+                                // a tile whose rows are consecutive pool rows (the compaction
+                                // warp marks it) is one TMA box per chunk
+                                if ((tcontig >> (i0 + i)) & 1u) {
+                                    const uint32_t ro0 = ro[0];
                                     if (lane == 0) {
-                                        mbar_arrive_expect_tx(&sm->a_full[gw], (uint32_t)a.pool_box_rows * 128u);
-                                        tma_load_2d(a_buf + gw * kATile, &mapP, &sm->a_full[gw], c * 64,
-                                                    (int32_t)(ro0 / row_bytes));
+                                        if (part == 0) {
+                                            mbar_arrive_expect_tx(&sm->a_full[aslot],
+                                                                  (uint32_t)(CPS * a.pool_box_rows) * 128u);
+#pragma unroll
+                                            for (int cc = 0; cc < CPS; ++cc)
+                                                tma_load_2d(a_buf + aslot * kAStage + cc * kATile, &mapP,
+                                                            &sm->a_full[aslot], (cp * CPS + cc) * 64,
+                                                            (int32_t)(ro0 / row_bytes));
+                                        } else {
+                                            mbar_arrive(&sm->a_full[aslot]);
+                                        }
                                     }
                                     __syncwarp();
                                 } else {
-                                    const char *src0 = pool_bytes + c * 128 + seg * 16;
-#pragma unroll 8
-                                    for (int j = 0; j < 32; ++j) {
-                                        const int r = 4 * j + r_in;
-                                        if (r < rows)
-                                            cp_async16(dst0 + r * 128 + ((seg ^ (r & 7)) << 4), src0 + ro[r]);
+                                    // one row-offset load and address computation per row, reused
+                                    // for each of the stage's CPS chunks
+                                    const char *src0 = pool_bytes + cp * CPS * 128 + seg * 16;
+#pragma unroll 4
+                                    for (int j = 0; j < rows_per / 4; ++j) {
+                                        const int r = r_lo + 4 * j + r_in;
+                                        if (r < rows) {
+                                            const char *src = src0 + ro[r];
+                                            const uint32_t d = dst0 + r * 128 + ((seg ^ (r & 7)) << 4);
+#pragma unroll
+                                            for (int cc = 0; cc < CPS; ++cc)
+                                                cp_async16(d + cc * kATile, src + cc * 128);
+                                        }
                                     }
                                     cp_async_commit();
                                     cp_async_wait<0>();
                                     fence_proxy_async_smem();
                                     __syncwarp();
                                     if (lane == 0)
-                                        mbar_arrive(&sm->a_full[gw]);
+                                        mbar_arrive(&sm->a_full[aslot]);
+                                    __syncwarp();
                                 }
                                 ph ^= 1u;
                             }
@@ -446,13 +543,19 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
         __syncwarp();
     } else if (warp == kMmaWarp || warp == kMmaWarp2) {
         // ============================================================ MMA
-        // Two threads issue the MMAs: thread mt takes the tiles i with
-        // i % 2 == mt, so each accumulator's chain (chunk 0 initialises, the
-        // later chunks accumulate) stays with one thread, while the other
-        // thread's MMAs fill the tensor pipe during this one's barrier waits,
-        // fences and commits (each of which costs the issuing thread on the
-        // order of 150 cycles on this part). Both walk the whole stage
-        // sequence and both release every Q chunk and every TMEM group.
+        // Two threads issue the MMAs (one cannot keep the pipe busy: an MMA
+        // instruction holds its issuing thread for longer than the pipe takes
+        // to run it, and every barrier wait and commit adds to that). Thread
+        // mt takes the tiles i with i % 2 == mt, so each accumulator's chain of
+        // chunks stays with one thread, and the other thread's MMAs keep the
+        // pipe busy through this one's waits and commits. Both walk the whole
+        // stage sequence of the shared A ring: each waits for every stage to be
+        // filled, the owner issues its MMAs and commits the slot's release,
+        // the other thread adds a plain arrival (the release barrier counts
+        // two). So no slot is refilled before both threads have passed its
+        // current use, and neither thread can meet a slot two phases ahead of
+        // the use it waits for. Both release every Q entry and every TMEM
+        // group.
         const int mt = (warp == kMmaWarp) ? 0 : 1;
         if (lane == 0) {
             const uint32_t idesc = idesc_bf16_f32(128, HH);
@@ -486,27 +589,39 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
                             ++jobs1;
                         else
                             ++jobs0;
-                        for (int c = 0; c < n_chunks && ok; ++c) {
+                        for (int cp = 0; cp < n_cp && ok; ++cp) {
                             if (!mbar_wait(&sm->q_full[qs], qph, abort_flag, a.err)) {
                                 ok = false;
                                 break;
                             }
-                            const uint64_t dq = sdesc_k_sw128(smem_u32(q_buf + qs * kQTile));
+                            const uint64_t dq = sdesc_k_sw128(smem_u32(q_buf + qs * kQEntry));
                             for (int i = 0; i < ntg; ++i) {
-                                if ((i & 1) == mt) {
-                                    if (!mbar_wait(&sm->a_full[as], aph, abort_flag, a.err)) {
-                                        ok = false;
-                                        break;
+                                if (!mbar_wait(&sm->a_full[as], aph, abort_flag, a.err)) {
+                                    ok = false;
+                                    break;
+                                }
+                                if ((i & 1) != mt) {
+                                    mbar_arrive(&sm->a_empty[as]);
+                                    if (++as == NA) {
+                                        as = 0;
+                                        aph ^= 1u;
                                     }
-                                    tc_fence_after();
-                                    const uint64_t da = sdesc_k_sw128(smem_u32(a_buf + as * kATile));
-                                    const uint32_t d_tmem = dbase + i * HH;
+                                    continue;
+                                }
+                                tc_fence_after();
+                                const uint64_t da = sdesc_k_sw128(smem_u32(a_buf + as * kAStage));
+                                const uint32_t d_tmem = dbase + i * HH;
+                                // CPS chunks x 4 K-steps; chunks are kATile bytes apart in A and
+                                // kQTile in Q (descriptor start addresses are in 16-byte units)
+#pragma unroll
+                                for (int cc = 0; cc < CPS; ++cc)
 #pragma unroll
                                     for (int kk = 0; kk < 4; ++kk)
-                                        umma_bf16(d_tmem, da + 2 * kk, dq + 2 * kk, idesc, (c | kk) != 0);
-                                    umma_commit(&sm->a_empty[as]);
-                                    issued = true;
-                                }
+                                        umma_bf16(d_tmem, da + (uint64_t)(cc * (kATile >> 4)) + 2 * kk,
+                                                  dq + (uint64_t)(cc * (kQTile >> 4)) + 2 * kk, idesc,
+                                                  ((cp * CPS + cc) | kk) != 0);
+                                umma_commit(&sm->a_empty[as]);
+                                issued = true;
                                 if (++as == NA) {
                                     as = 0;
                                     aph ^= 1u;
@@ -535,17 +650,25 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
     }
     } else {
         // ============================================================ epilogue
-        // Both epilogue warpgroups work on every token: warpgroup hf takes the
-        // tiles [hf*TBH, (hf+1)*TBH) of each TMEM group, so a token's scores
-        // are drained in about half the time of one warpgroup and the TMEM
-        // buffer returns to the MMA threads sooner. Per-head statistics are
-        // combined across the eight warps through shared memory.
+        // Both epilogue warpgroups work on every token. For H >= 32 warpgroup
+        // hf takes the heads [hf*H/2, (hf+1)*H/2) of every tile of a TMEM
+        // group: a thread (one TMEM lane = one slot row per tile) reduces its
+        // own rows first, so a column needs one cross-lane reduction per
+        // warp whatever the tile count; the column max is one redux per
+        // column. The two halves of each row's u are added through shared
+        // memory. (For H = 16 warpgroup hf takes half the tiles instead.)
+        // Per-head statistics are combined across warps through shared memory.
         // warpgroups 3 and 4 execute this one setmaxnreg together
         regs_inc<kHighRegs>();
-        constexpr int TBH = TB / 2;           // tiles per warpgroup and group
-        constexpr int IBH = TBH < 2 ? TBH : 2; // tiles per TMEM load batch
+        constexpr int TBH = TB / 2;           // tiles per warpgroup and group (H = 16)
+        constexpr int IBH = TBH < 2 ? TBH : 2; // tiles per TMEM load batch (H = 16)
+        // H >= 32: warpgroup hf takes heads [hf*HC, (hf+1)*HC) of every tile
+        constexpr int HC = HH / 2;
+        constexpr int NCB = HC >= 16 ? HC / 16 : 1;
+        constexpr int IB = TB < 2 ? TB : 2;   // tiles per TMEM load batch
         const int ew = warp - kEpiWarp0;      // 0..7
-        const int hf = ew >> 2;               // which half of the tiles
+        const int hf = ew >> 2;               // which half of the heads (H >= 32) or tiles (H = 16)
+        const int c_lo = hf * HC;
         const int q = warp & 3;               // TMEM lane quarter
         const int r = q * 32 + lane;          // row within a 128-slot tile
         const int et = ew * 32 + lane;        // 0..255
@@ -553,6 +676,7 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
         constexpr int kEpiThreads = 256;
         EpiState<HH> &st = sm->epi[0];
         float *ub = ubuf;
+        float *uh = ubuf + Kp;                // [2][TB*128] the warpgroups' partial u (H >= 32)
         const float s2 = a.scale * kLog2e;    // scale > 0 (checked on the host)
         const float sink_h = (a.sink && et < HH) ? a.sink[et] : -INFINITY;
         int jobs0 = 0, jobs1 = 0;
@@ -586,8 +710,12 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
             // window log-mass of this token's heads, fetched early
             const float wl_h = (et < HH && a.wl) ? a.wl[(size_t)g * HH + et] : 0.f;
             // leader waits; the named barrier hands the outcome to everyone
-            if (et == 0)
-                st.flag = mbar_wait(&sm->meta_full[m3], (it / kMeta) & 1, abort_flag, a.err) ? 1 : 0;
+            if (ew == 0) {
+                const bool f = warp_mbar_wait(&sm->meta_full[m3], (it / kMeta) & 1, abort_flag, a.err);
+                if (lane == 0)
+                    st.flag = f ? 1 : 0;
+                __syncwarp();
+            }
             named_bar_sync(bar_id, kEpiThreads);
             if (!st.flag)
                 break;
@@ -597,6 +725,7 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
             const int passes = G > 1 ? 2 : 1;
             float *prow = a.p + (size_t)g * K;
             const int32_t *sl = slot + m3 * Kp;
+            const bool ident = sm->ident[m3] != 0;    // slot jj of the compacted order is slot jj
             const uint32_t tbase = tmem + mb * 256 + ((uint32_t)(q * 32) << 16);
             // fused KL: this thread's scores and valid flags (slots et, et+256),
             // loaded now so the latency is hidden behind the token's MMAs
@@ -608,7 +737,7 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
                 for (int i = 0; i < kKlReg; ++i) {
                     const int jj = et + i * kEpiThreads;
                     const bool in = jj < K;
-                    const size_t gi = (size_t)g * K + (in ? sl[jj] : 0);
+                    const size_t gi = (size_t)g * K + (in ? (ident ? jj : sl[jj]) : 0);
                     kl_s[i] = in ? a.kl_scores[gi] : 0.f;
                     kl_v[i] = in ? a.kl_valid[gi] : 0;
                 }
@@ -624,9 +753,12 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
                     const int t0 = hf * TBH;
                     const int t1 = min(ntg, t0 + TBH);
                     named_bar_sync(bar_id, kEpiThreads);   // st.flag is free again
-                    if (et == 0) {
+                    if (ew == 0) {
                         const int jb = mb ? jobs1 : jobs0;
-                        st.flag = mbar_wait(&sm->acc_full[mb], jb & 1, abort_flag, a.err) ? 1 : 0;
+                        const bool f = warp_mbar_wait(&sm->acc_full[mb], jb & 1, abort_flag, a.err);
+                        if (lane == 0)
+                            st.flag = f ? 1 : 0;
+                        __syncwarp();
                     }
                     named_bar_sync(bar_id, kEpiThreads);
                     if (mb)
@@ -639,6 +771,127 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
                     }
                     tc_fence_after();
                     const bool single = (G == 1);
+                    if constexpr (HH >= 32) {
+                    if (pass == 0) {
+                        // ---- column max of the raw dot products over valid rows:
+                        // over this thread's rows first, then across the warp's
+                        // lanes in one instruction per column
+#pragma unroll
+                        for (int cb = 0; cb < NCB; ++cb) {
+                            const int col0 = c_lo + cb * 16;
+                            float m16[16];
+#pragma unroll
+                            for (int e = 0; e < 16; ++e)
+                                m16[e] = -INFINITY;
+#pragma unroll
+                            for (int ib = 0; ib < TB; ib += IB) {
+                                if (ib >= ntg)
+                                    break;
+                                uint32_t v[IB][16];
+#pragma unroll
+                                for (int i = 0; i < IB; ++i)
+                                    if (ib + i < ntg)
+                                        tmem_ld16(tbase + (ib + i) * HH + col0, v[i]);
+                                tmem_ld_wait();
+#pragma unroll
+                                for (int i = 0; i < IB; ++i) {
+                                    if (ib + i < ntg && (i0 + ib + i) * 128 + r < nsel) {
+#pragma unroll
+                                        for (int e = 0; e < 16; ++e)
+                                            m16[e] = fmaxf(m16[e], __uint_as_float(v[i][e]));
+                                    }
+                                }
+                            }
+                            float mine = -INFINITY;
+#pragma unroll
+                            for (int e = 0; e < 16; ++e) {
+                                const float wmax = warp_max_f32(m16[e]);
+                                mine = lane == e ? wmax : mine;
+                            }
+                            if (lane < 16)
+                                st.red_max[q][col0 + lane] = mine;
+                        }
+                        named_bar_sync(bar_id, kEpiThreads);
+                        if (et < HH) {
+                            float mx = st.red_max[0][et];
+#pragma unroll
+                            for (int w = 1; w < 4; ++w)
+                                mx = fmaxf(mx, st.red_max[w][et]);
+                            st.head_a[et] = mx * s2;
+                        }
+                        named_bar_sync(bar_id, kEpiThreads);
+                        // ---- e = 2^(v s2 - max s2), column sums; one group: keep e in TMEM
+#pragma unroll
+                        for (int cb = 0; cb < NCB; ++cb) {
+                            const int col0 = c_lo + cb * 16;
+                            float s16[16], m16[16];
+#pragma unroll
+                            for (int e = 0; e < 16; ++e) {
+                                s16[e] = 0.f;
+                                m16[e] = st.head_a[col0 + e];
+                            }
+#pragma unroll
+                            for (int ib = 0; ib < TB; ib += IB) {
+                                if (ib >= ntg)
+                                    break;
+                                uint32_t v[IB][16];
+#pragma unroll
+                                for (int i = 0; i < IB; ++i)
+                                    if (ib + i < ntg)
+                                        tmem_ld16(tbase + (ib + i) * HH + col0, v[i]);
+                                tmem_ld_wait();
+#pragma unroll
+                                for (int i = 0; i < IB; ++i) {
+                                    if (ib + i < ntg) {
+                                        if ((i0 + ib + i) * 128 + r < nsel) {
+#pragma unroll
+                                            for (int e = 0; e < 16; ++e) {
+                                                const float x =
+                                                    ex2_approx(fmaf(__uint_as_float(v[i][e]), s2, -m16[e]));
+                                                s16[e] += x;
+                                                v[i][e] = __float_as_uint(x);
+                                            }
+                                        } else {
+#pragma unroll
+                                            for (int e = 0; e < 16; ++e)
+                                                v[i][e] = 0u;
+                                        }
+                                    }
+                                }
+                                if (single) {
+#pragma unroll
+                                    for (int i = 0; i < IB; ++i)
+                                        if (ib + i < ntg)
+                                            tmem_st16(tbase + (ib + i) * HH + col0, v[i]);
+                                }
+                            }
+                            const float red = warp_colreduce16(s16, OpAdd());
+                            if (lane < 16)
+                                st.red_sum[q][col0 + lane] = red;
+                        }
+                        if (single)
+                            tmem_st_wait();
+                        named_bar_sync(bar_id, kEpiThreads);
+                        if (et < HH) {
+                            // group statistics in the log2 domain: max M2, sum S
+                            const float gm = st.head_a[et];
+                            float gs = 0.f;
+#pragma unroll
+                            for (int w = 0; w < 4; ++w)
+                                gs += st.red_sum[w][et];
+                            if (grp == 0) {
+                                st.colM[et] = gm;
+                                st.colS[et] = gs;
+                            } else {
+                                const float M0 = st.colM[et], S0 = st.colS[et];
+                                const float M1 = fmaxf(M0, gm);
+                                st.colS[et] = S0 * exp2f(M0 - M1) + gs * exp2f(gm - M1);
+                                st.colM[et] = M1;
+                            }
+                        }
+                        named_bar_sync(bar_id, kEpiThreads);
+                    }
+                    } else {
                     if (pass == 0) {
                         // ---- column max of the raw dot products over valid rows
                         for (int cc = 0; cc < NC16; ++cc) {
@@ -741,6 +994,7 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
                         }
                         named_bar_sync(bar_id, kEpiThreads);
                     }
+                    }
                     if (pass == passes - 1) {
                         if (grp == 0) {
                             // ---- per-head merge with the window and the sink
@@ -773,6 +1027,66 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
                                 st.wprime[et] = expf(st.head_a[et] - At);
                             named_bar_sync(bar_id, kEpiThreads);
                         }
+                        if constexpr (HH >= 32) {
+                        // ---- u'[k] = sum_h e[k,h] w[h]: each warpgroup sums its own
+                        // heads for every tile of the group; the two partial sums of
+                        // a row are added through shared memory
+                        float u[TB];
+#pragma unroll
+                        for (int i = 0; i < TB; ++i)
+                            u[i] = 0.f;
+#pragma unroll
+                        for (int cb = 0; cb < NCB; ++cb) {
+                            const int col0 = c_lo + cb * 16;
+                            float w16[16], cm16[16];
+#pragma unroll
+                            for (int e = 0; e < 16; ++e) {
+                                w16[e] = st.wprime[col0 + e];
+                                cm16[e] = single ? 0.f : st.colM[col0 + e];
+                            }
+#pragma unroll
+                            for (int ib = 0; ib < TB; ib += IB) {
+                                if (ib >= ntg)
+                                    break;
+                                uint32_t v[IB][16];
+#pragma unroll
+                                for (int i = 0; i < IB; ++i)
+                                    if (ib + i < ntg)
+                                        tmem_ld16(tbase + (ib + i) * HH + col0, v[i]);
+                                tmem_ld_wait();
+#pragma unroll
+                                for (int i = 0; i < IB; ++i) {
+                                    if (ib + i < ntg) {
+                                        float acc = u[ib + i];
+                                        if (single) {
+#pragma unroll
+                                            for (int e = 0; e < 16; ++e)
+                                                acc = fmaf(__uint_as_float(v[i][e]), w16[e], acc);
+                                        } else {
+#pragma unroll
+                                            for (int e = 0; e < 16; ++e)
+                                                acc = fmaf(ex2_approx(fmaf(__uint_as_float(v[i][e]), s2, -cm16[e])),
+                                                           w16[e], acc);
+                                        }
+                                        u[ib + i] = acc;
+                                    }
+                                }
+                            }
+                        }
+#pragma unroll
+                        for (int i = 0; i < TB; ++i)
+                            if (i < ntg)
+                                uh[hf * (TB * 128) + i * 128 + r] = u[i];
+                        named_bar_sync(bar_id, kEpiThreads);
+                        for (int i = hf; i < ntg; i += 2) {
+                            const int j = (i0 + i) * 128 + r;
+                            if (j < nsel) {
+                                const float uu = uh[i * 128 + r] + uh[TB * 128 + i * 128 + r];
+                                ub[j] = uu;
+                                m_part += uu;
+                            }
+                        }
+                        } else {
                         // ---- u'[k] = sum_h e[k,h] w[h]
                         float u[TBH];
 #pragma unroll
@@ -821,11 +1135,13 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
                                 m_part += u[i];
                             }
                         }
+                        }
                     }
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0)
                         mbar_arrive(&sm->acc_empty[mb]);
+                    __syncwarp();
                 }
             }
             if (!ok)
@@ -850,7 +1166,7 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
             }
             if (a.p) {
                 for (int jj = et; jj < K; jj += kEpiThreads)
-                    prow[sl[jj]] = (jj < nsel) ? ub[jj] * f : 0.f;
+                    prow[ident ? jj : sl[jj]] = (jj < nsel) ? ub[jj] * f : 0.f;
             }
             if (kl) {
                 // ---- KL(p || softmax(scores)) over the row's valid slots and
@@ -864,7 +1180,7 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
 #pragma unroll
                 for (int i = 0; i < kKlReg; ++i) {
                     const int jj = et + i * kEpiThreads;
-                    kk[i] = jj < K ? sl[jj] : 0;
+                    kk[i] = jj < K ? (ident ? jj : sl[jj]) : 0;
                     pv[i] = (jj < nsel) ? ub[jj] * f : 0.f;
                     if (kl_v[i]) {
                         mx = fmaxf(mx, kl_s[i]);
@@ -943,6 +1259,7 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
             named_bar_sync(bar_id, kEpiThreads);
             if (et == 0)
                 mbar_arrive(&sm->meta_empty[m3]);
+            __syncwarp();
         }
         if (kl && et == 0) {
             // this CTA's KL sum; the last CTA to finish adds them in CTA order
@@ -967,48 +1284,66 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
     }
 }
 
-template <int HH>
+template <int HH, int CPS>
 __host__ __device__ inline size_t fixed_smem_bytes(int K)
 {
     const size_t Kp = (size_t)((K + 3) & ~3);
-    return 1024 + q_stages<HH>() * (HH * 128) + Kp * 4 * (2 * kMeta + 4) + sizeof(TgtSmem<HH>) + 64;
+    const size_t uh = HH >= 32 ? (size_t)2 * (256 / HH) * 128 * 4 : 0;   // partial u of the two warpgroups
+    return 1024 + q_entries<HH, CPS>() * (size_t)(CPS * HH * 128) + Kp * 4 * (2 * kMeta + 4) + uh +
+           sizeof(TgtSmem<HH>) + 64;
 }
 
-// Deepest A-stage ring that fits the per-block smem limit (0 if none does).
-template <int HH>
+// Deepest A-stage ring that fits the per-block smem limit, as a divisor of
+// the eight gather warps (so every slot has the same number of producers),
+// with two slots at least for each of the two MMA threads; 0 if none fits.
+template <int HH, int CPS>
 int stages_for(int K, int smem_limit)
 {
-    const long room = (long)smem_limit - (long)fixed_smem_bytes<HH>(K);
-    long n = room / (long)kATile;
+    const long room = (long)smem_limit - (long)fixed_smem_bytes<HH, CPS>(K);
+    long n = room / (long)(CPS * kATile);
     if (n > kMaxAStages)
         n = kMaxAStages;
-    return n >= 4 ? (int)n : 0;
+    int na = 8;
+    while (na > n)
+        na >>= 1;
+    return na >= 4 ? na : 0;   // two slots at least for each MMA thread
 }
 
-template <int HH>
+template <int HH, int CPS>
 size_t smem_bytes_for(int K, int stages)
 {
-    return fixed_smem_bytes<HH>(K) + (size_t)stages * kATile;
+    return fixed_smem_bytes<HH, CPS>(K) + (size_t)stages * CPS * kATile;
+}
+
+template <int HH, bool FUSE_KL, int CPS>
+cudaError_t launch_hkc(const CUtensorMap &mapQ, const CUtensorMap &mapP, const TgtTcArgs &a, int grid,
+                       cudaStream_t stream)
+{
+    // The register split above is only safe if every thread was launched with
+    // exactly kLaunchRegs registers; refuse to launch otherwise.
+    cudaFuncAttributes fa;
+    cudaError_t e = cudaFuncGetAttributes(&fa, target_tc_kernel<HH, FUSE_KL, CPS>);
+    if (e != cudaSuccess)
+        return e;
+    if (fa.numRegs != kLaunchRegs)
+        return cudaErrorInvalidConfiguration;
+    if (a.n_astages < 1 || kGatherWarps % a.n_astages != 0 || (a.D / 64) % CPS != 0)
+        return cudaErrorInvalidValue;
+    const size_t smem = smem_bytes_for<HH, CPS>(a.K, a.n_astages);
+    e = cudaFuncSetAttribute(target_tc_kernel<HH, FUSE_KL, CPS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem);
+    if (e != cudaSuccess)
+        return e;
+    target_tc_kernel<HH, FUSE_KL, CPS><<<grid, kTgtThreads, smem, stream>>>(mapQ, mapP, a);
+    return cudaGetLastError();
 }
 
 template <int HH, bool FUSE_KL>
 cudaError_t launch_hk(const CUtensorMap &mapQ, const CUtensorMap &mapP, const TgtTcArgs &a, int grid,
                       cudaStream_t stream)
 {
-    // The register split above is only safe if every thread was launched with
-    // exactly kLaunchRegs registers; refuse to launch otherwise.
-    cudaFuncAttributes fa;
-    cudaError_t e = cudaFuncGetAttributes(&fa, target_tc_kernel<HH, FUSE_KL>);
-    if (e != cudaSuccess)
-        return e;
-    if (fa.numRegs != kLaunchRegs)
-        return cudaErrorInvalidConfiguration;
-    const size_t smem = smem_bytes_for<HH>(a.K, a.n_astages);
-    e = cudaFuncSetAttribute(target_tc_kernel<HH, FUSE_KL>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess)
-        return e;
-    target_tc_kernel<HH, FUSE_KL><<<grid, kTgtThreads, smem, stream>>>(mapQ, mapP, a);
-    return cudaGetLastError();
+    return a.cps == 2 ? launch_hkc<HH, FUSE_KL, 2>(mapQ, mapP, a, grid, stream)
+                      : launch_hkc<HH, FUSE_KL, 1>(mapQ, mapP, a, grid, stream);
 }
 
 template <int HH>
@@ -1019,15 +1354,21 @@ cudaError_t launch_h(const CUtensorMap &mapQ, const CUtensorMap &mapP, const Tgt
                        : launch_hk<HH, false>(mapQ, mapP, a, grid, stream);
 }
 
+template <int HH>
+int stages_h(int K, int cps, int smem_limit)
+{
+    return cps == 2 ? stages_for<HH, 2>(K, smem_limit) : stages_for<HH, 1>(K, smem_limit);
+}
+
 }  // namespace
 
-int target_tc_stages(int H, int K, int smem_limit)
+int target_tc_stages(int H, int K, int cps, int smem_limit)
 {
     switch (H) {
-    case 16: return stages_for<16>(K, smem_limit);
-    case 32: return stages_for<32>(K, smem_limit);
-    case 64: return stages_for<64>(K, smem_limit);
-    case 128: return stages_for<128>(K, smem_limit);
+    case 16: return stages_h<16>(K, cps, smem_limit);
+    case 32: return stages_h<32>(K, cps, smem_limit);
+    case 64: return stages_h<64>(K, cps, smem_limit);
+    case 128: return stages_h<128>(K, cps, smem_limit);
     default: return 0;
     }
 }

@@ -2,7 +2,9 @@
 memory (no workspace argument; scratch lives in a fixed array inside the
 library). Checked through the C ABI against sai_distill_kl on two calls in a
 row, so a stale scratch word left by the first call would show up in the
-second. This file is collected last on purpose."""
+second, then a larger grid followed by a smaller one on the shared array,
+the forward-only form through the Python wrapper, and the loss against the
+fp64 oracle. This file is collected last on purpose."""
 import ctypes
 
 import numpy as np
@@ -58,3 +60,22 @@ def test_noalloc_matches_workspace_call_twice(lib, shape):
         assert abs(lg - lr) <= 1e-4 * abs(lr), (call, lg, lr)
         assert torch.max(torch.abs(ds - ds_ref)).item() <= 1e-6
         assert bool(torch.isfinite(ds).all())
+
+
+def test_noalloc_large_grid_then_small_and_forward_only():
+    """The flash shape (the most KL blocks) fills the shared array first; a
+    small shape after it must not read the large call's leftovers. The second
+    call goes through the Python wrapper without dscores (forward only)."""
+    import oracle
+    import sparse_attention_indexer_window_b200 as sai
+    for B, S, K, seed in ((1, 4096, 512, 21), (2, 75, 96, 22)):
+        p, scores, valid = _case(seed, B, S, K)
+        loss = torch.full((1,), float("nan"), device="cuda")
+        ds = torch.full((B, S, K), float("nan"), device="cuda") if S == 4096 else None
+        sai.distill_kl_noalloc(p, scores, valid, 0.01, loss, ds)
+        torch.cuda.synchronize()
+        ol, ods, _ = oracle.distill_kl(p.cpu().numpy().astype(np.float64), scores.cpu().numpy(),
+                                       valid.cpu().numpy(), 0.01)
+        assert abs(float(loss.item()) - ol) <= 1e-4 * abs(ol)
+        if ds is not None:
+            assert np.abs(ds.cpu().numpy().reshape(-1, K) - ods).max() <= 1e-6
