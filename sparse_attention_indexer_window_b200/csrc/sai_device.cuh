@@ -240,6 +240,22 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16])
         : "memory");
 }
 
+// 32 lanes x 8 columns (the x16 form's half).
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&r)[8])
+{
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+                 : "r"(taddr)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8])
+{
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
+                 "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+                 : "memory");
+}
+
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16])
 {
     asm volatile(
@@ -303,6 +319,26 @@ __device__ __forceinline__ float warp_colreduce16(float (&v)[16], Op op)
     }
     const float other = __shfl_xor_sync(0xffffffffu, v[0], 16);
     return op(v[0], other);
+}
+
+// The 8-column form: lane L < 8 returns op over all 32 lanes of v[L].
+template <class Op>
+__device__ __forceinline__ float warp_colreduce8(float (&v)[8], Op op)
+{
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int n = 4; n >= 1; n >>= 1) {
+        const bool upper = (lane & n) != 0;
+#pragma unroll
+        for (int k = 0; k < n; ++k) {
+            const float send = upper ? v[k] : v[k + n];
+            const float keep = upper ? v[k + n] : v[k];
+            const float recv = __shfl_xor_sync(0xffffffffu, send, n);
+            v[k] = op(keep, recv);
+        }
+    }
+    float x = op(v[0], __shfl_xor_sync(0xffffffffu, v[0], 8));
+    return op(x, __shfl_xor_sync(0xffffffffu, x, 16));
 }
 
 // Maximum of v over the 32 lanes of a warp, in every lane (one instruction).

@@ -773,112 +773,90 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
                     const bool single = (G == 1);
                     if constexpr (HH >= 32) {
                     if (pass == 0) {
-                        // ---- column max of the raw dot products over valid rows:
-                        // over this thread's rows first, then across the warp's
-                        // lanes in one instruction per column
+                    if constexpr (TB <= 4) {
+                        // ---- one pass over the group's scores. Per 8-column block,
+                        // every tile's values of this thread's rows come in at once;
+                        // the stabiliser of a column is the warp's maximum over its
+                        // 32 lanes x TB rows (one redux per column), e = 2^(v s2 -
+                        // that) over valid rows (kept in TMEM for a single group),
+                        // and the column sums are taken over the warp. The four TMEM
+                        // lane quarters' (max, sum) pairs are merged per head below;
+                        // the quarter maxima stay in red_max for the u pass.
+#pragma unroll 1
+                        for (int cb = 0; cb < HC / 8; ++cb) {
+                            const int col0 = c_lo + cb * 8;
+                            uint32_t v[TB][8];
 #pragma unroll
-                        for (int cb = 0; cb < NCB; ++cb) {
-                            const int col0 = c_lo + cb * 16;
-                            float m16[16];
+                            for (int i = 0; i < TB; ++i)
+                                if (i < ntg)
+                                    tmem_ld8(tbase + i * HH + col0, v[i]);
+                            tmem_ld_wait();
+                            float m8[8];
 #pragma unroll
-                            for (int e = 0; e < 16; ++e)
-                                m16[e] = -INFINITY;
+                            for (int e = 0; e < 8; ++e)
+                                m8[e] = -INFINITY;
 #pragma unroll
-                            for (int ib = 0; ib < TB; ib += IB) {
-                                if (ib >= ntg)
-                                    break;
-                                uint32_t v[IB][16];
+                            for (int i = 0; i < TB; ++i) {
+                                if (i < ntg && (i0 + i) * 128 + r < nsel) {
 #pragma unroll
-                                for (int i = 0; i < IB; ++i)
-                                    if (ib + i < ntg)
-                                        tmem_ld16(tbase + (ib + i) * HH + col0, v[i]);
-                                tmem_ld_wait();
-#pragma unroll
-                                for (int i = 0; i < IB; ++i) {
-                                    if (ib + i < ntg && (i0 + ib + i) * 128 + r < nsel) {
-#pragma unroll
-                                        for (int e = 0; e < 16; ++e)
-                                            m16[e] = fmaxf(m16[e], __uint_as_float(v[i][e]));
-                                    }
+                                    for (int e = 0; e < 8; ++e)
+                                        m8[e] = fmaxf(m8[e], __uint_as_float(v[i][e]));
                                 }
                             }
                             float mine = -INFINITY;
 #pragma unroll
-                            for (int e = 0; e < 16; ++e) {
-                                const float wmax = warp_max_f32(m16[e]);
-                                mine = lane == e ? wmax : mine;
+                            for (int e = 0; e < 8; ++e) {
+                                m8[e] = warp_max_f32(m8[e]) * s2;
+                                mine = lane == e ? m8[e] : mine;
                             }
-                            if (lane < 16)
-                                st.red_max[q][col0 + lane] = mine;
-                        }
-                        named_bar_sync(bar_id, kEpiThreads);
-                        if (et < HH) {
-                            float mx = st.red_max[0][et];
+                            float s8[8];
 #pragma unroll
-                            for (int w = 1; w < 4; ++w)
-                                mx = fmaxf(mx, st.red_max[w][et]);
-                            st.head_a[et] = mx * s2;
-                        }
-                        named_bar_sync(bar_id, kEpiThreads);
-                        // ---- e = 2^(v s2 - max s2), column sums; one group: keep e in TMEM
+                            for (int e = 0; e < 8; ++e)
+                                s8[e] = 0.f;
 #pragma unroll
-                        for (int cb = 0; cb < NCB; ++cb) {
-                            const int col0 = c_lo + cb * 16;
-                            float s16[16], m16[16];
+                            for (int i = 0; i < TB; ++i) {
+                                if (i < ntg) {
+                                    if ((i0 + i) * 128 + r < nsel) {
 #pragma unroll
-                            for (int e = 0; e < 16; ++e) {
-                                s16[e] = 0.f;
-                                m16[e] = st.head_a[col0 + e];
-                            }
-#pragma unroll
-                            for (int ib = 0; ib < TB; ib += IB) {
-                                if (ib >= ntg)
-                                    break;
-                                uint32_t v[IB][16];
-#pragma unroll
-                                for (int i = 0; i < IB; ++i)
-                                    if (ib + i < ntg)
-                                        tmem_ld16(tbase + (ib + i) * HH + col0, v[i]);
-                                tmem_ld_wait();
-#pragma unroll
-                                for (int i = 0; i < IB; ++i) {
-                                    if (ib + i < ntg) {
-                                        if ((i0 + ib + i) * 128 + r < nsel) {
-#pragma unroll
-                                            for (int e = 0; e < 16; ++e) {
-                                                const float x =
-                                                    ex2_approx(fmaf(__uint_as_float(v[i][e]), s2, -m16[e]));
-                                                s16[e] += x;
-                                                v[i][e] = __float_as_uint(x);
-                                            }
-                                        } else {
-#pragma unroll
-                                            for (int e = 0; e < 16; ++e)
-                                                v[i][e] = 0u;
+                                        for (int e = 0; e < 8; ++e) {
+                                            const float x = ex2_approx(fmaf(__uint_as_float(v[i][e]), s2, -m8[e]));
+                                            s8[e] += x;
+                                            v[i][e] = __float_as_uint(x);
                                         }
+                                    } else {
+#pragma unroll
+                                        for (int e = 0; e < 8; ++e)
+                                            v[i][e] = 0u;
                                     }
                                 }
-                                if (single) {
-#pragma unroll
-                                    for (int i = 0; i < IB; ++i)
-                                        if (ib + i < ntg)
-                                            tmem_st16(tbase + (ib + i) * HH + col0, v[i]);
-                                }
                             }
-                            const float red = warp_colreduce16(s16, OpAdd());
-                            if (lane < 16)
+                            if (single) {
+#pragma unroll
+                                for (int i = 0; i < TB; ++i)
+                                    if (i < ntg)
+                                        tmem_st8(tbase + i * HH + col0, v[i]);
+                            }
+                            const float red = warp_colreduce8(s8, OpAdd());
+                            if (lane < 8) {
+                                st.red_max[q][col0 + lane] = mine;
                                 st.red_sum[q][col0 + lane] = red;
+                            }
                         }
                         if (single)
                             tmem_st_wait();
                         named_bar_sync(bar_id, kEpiThreads);
                         if (et < HH) {
                             // group statistics in the log2 domain: max M2, sum S
-                            const float gm = st.head_a[et];
-                            float gs = 0.f;
+                            float gm = st.red_max[0][et];
 #pragma unroll
-                            for (int w = 0; w < 4; ++w)
-                                gs += st.red_sum[w][et];
+                            for (int w = 1; w < 4; ++w)
+                                gm = fmaxf(gm, st.red_max[w][et]);
+                            float gs = 0.f;
+                            if (gm != -INFINITY) {
+#pragma unroll
+                                for (int w = 0; w < 4; ++w)
+                                    gs += st.red_sum[w][et] * exp2f(st.red_max[w][et] - gm);
+                            }
                             if (grp == 0) {
                                 st.colM[et] = gm;
                                 st.colS[et] = gs;
@@ -889,6 +867,124 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
                                 st.colM[et] = M1;
                             }
                         }
+                    } else {
+                            // ---- column max of the raw dot products over valid rows:
+                            // over this thread's rows first, then across the warp's
+                            // lanes in one instruction per column
+#pragma unroll
+                            for (int cb = 0; cb < NCB; ++cb) {
+                                const int col0 = c_lo + cb * 16;
+                                float m16[16];
+#pragma unroll
+                                for (int e = 0; e < 16; ++e)
+                                    m16[e] = -INFINITY;
+#pragma unroll
+                                for (int ib = 0; ib < TB; ib += IB) {
+                                    if (ib >= ntg)
+                                        break;
+                                    uint32_t v[IB][16];
+#pragma unroll
+                                    for (int i = 0; i < IB; ++i)
+                                        if (ib + i < ntg)
+                                            tmem_ld16(tbase + (ib + i) * HH + col0, v[i]);
+                                    tmem_ld_wait();
+#pragma unroll
+                                    for (int i = 0; i < IB; ++i) {
+                                        if (ib + i < ntg && (i0 + ib + i) * 128 + r < nsel) {
+#pragma unroll
+                                            for (int e = 0; e < 16; ++e)
+                                                m16[e] = fmaxf(m16[e], __uint_as_float(v[i][e]));
+                                        }
+                                    }
+                                }
+                                float mine = -INFINITY;
+#pragma unroll
+                                for (int e = 0; e < 16; ++e) {
+                                    const float wmax = warp_max_f32(m16[e]);
+                                    mine = lane == e ? wmax : mine;
+                                }
+                                if (lane < 16)
+                                    st.red_max[q][col0 + lane] = mine;
+                            }
+                            named_bar_sync(bar_id, kEpiThreads);
+                            if (et < HH) {
+                                float mx = st.red_max[0][et];
+#pragma unroll
+                                for (int w = 1; w < 4; ++w)
+                                    mx = fmaxf(mx, st.red_max[w][et]);
+                                st.head_a[et] = mx * s2;
+                            }
+                            named_bar_sync(bar_id, kEpiThreads);
+                            // ---- e = 2^(v s2 - max s2), column sums; one group: keep e in TMEM
+#pragma unroll
+                            for (int cb = 0; cb < NCB; ++cb) {
+                                const int col0 = c_lo + cb * 16;
+                                float s16[16], m16[16];
+#pragma unroll
+                                for (int e = 0; e < 16; ++e) {
+                                    s16[e] = 0.f;
+                                    m16[e] = st.head_a[col0 + e];
+                                }
+#pragma unroll
+                                for (int ib = 0; ib < TB; ib += IB) {
+                                    if (ib >= ntg)
+                                        break;
+                                    uint32_t v[IB][16];
+#pragma unroll
+                                    for (int i = 0; i < IB; ++i)
+                                        if (ib + i < ntg)
+                                            tmem_ld16(tbase + (ib + i) * HH + col0, v[i]);
+                                    tmem_ld_wait();
+#pragma unroll
+                                    for (int i = 0; i < IB; ++i) {
+                                        if (ib + i < ntg) {
+                                            if ((i0 + ib + i) * 128 + r < nsel) {
+#pragma unroll
+                                                for (int e = 0; e < 16; ++e) {
+                                                    const float x =
+                                                        ex2_approx(fmaf(__uint_as_float(v[i][e]), s2, -m16[e]));
+                                                    s16[e] += x;
+                                                    v[i][e] = __float_as_uint(x);
+                                                }
+                                            } else {
+#pragma unroll
+                                                for (int e = 0; e < 16; ++e)
+                                                    v[i][e] = 0u;
+                                            }
+                                        }
+                                    }
+                                    if (single) {
+#pragma unroll
+                                        for (int i = 0; i < IB; ++i)
+                                            if (ib + i < ntg)
+                                                tmem_st16(tbase + (ib + i) * HH + col0, v[i]);
+                                    }
+                                }
+                                const float red = warp_colreduce16(s16, OpAdd());
+                                if (lane < 16)
+                                    st.red_sum[q][col0 + lane] = red;
+                            }
+                            if (single)
+                                tmem_st_wait();
+                            named_bar_sync(bar_id, kEpiThreads);
+                            if (et < HH) {
+                                // group statistics in the log2 domain: max M2, sum S
+                                const float gm = st.head_a[et];
+                                float gs = 0.f;
+#pragma unroll
+                                for (int w = 0; w < 4; ++w)
+                                    gs += st.red_sum[w][et];
+                                if (grp == 0) {
+                                    st.colM[et] = gm;
+                                    st.colS[et] = gs;
+                                } else {
+                                    const float M0 = st.colM[et], S0 = st.colS[et];
+                                    const float M1 = fmaxf(M0, gm);
+                                    st.colS[et] = S0 * exp2f(M0 - M1) + gs * exp2f(gm - M1);
+                                    st.colM[et] = M1;
+                                }
+                            }
+                    }
                         named_bar_sync(bar_id, kEpiThreads);
                     }
                     } else {
@@ -1023,8 +1119,20 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
                             for (int o = 16; o >= 1; o >>= 1)
                                 x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
                             At = x;
-                            if (et < HH)
-                                st.wprime[et] = expf(st.head_a[et] - At);
+                            if (et < HH) {
+                                const float wp = expf(st.head_a[et] - At);
+                                st.wprime[et] = wp;
+                                if constexpr (HH >= 32 && TB <= 4) {
+                                    // a single group's e are relative to their lane
+                                    // quarter's maximum: fold the rescale to the head's
+                                    // maximum into the weight, per quarter
+                                    if (single) {
+#pragma unroll
+                                        for (int w = 0; w < 4; ++w)
+                                            st.red_max[w][et] = wp * exp2f(st.red_max[w][et] - st.colM[et]);
+                                    }
+                                }
+                            }
                             named_bar_sync(bar_id, kEpiThreads);
                         }
                         if constexpr (HH >= 32) {
@@ -1041,7 +1149,7 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
                             float w16[16], cm16[16];
 #pragma unroll
                             for (int e = 0; e < 16; ++e) {
-                                w16[e] = st.wprime[col0 + e];
+                                w16[e] = (TB <= 4 && single) ? st.red_max[q][col0 + e] : st.wprime[col0 + e];
                                 cm16[e] = single ? 0.f : st.colM[col0 + e];
                             }
 #pragma unroll
