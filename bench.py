@@ -540,7 +540,7 @@ def main():
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "steps": args.e2e_steps},
             "long": long_line,
-            "gpu_launches": 4 * nsteps * world,   # window, target, KL count, KL rows; every rank
+            "gpu_launches": 3 * nsteps * world,   # window, target, KL (one cooperative launch); every rank
             "clocks": clk,
             "loss": loss_all,
         }
