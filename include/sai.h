@@ -11,7 +11,9 @@
  *   sai_distill_kl      p, scores, valid -> loss (device scalar), dscores [B,S,K]
  *
  * Around them: sai_distill_target_ex (the per-branch target, or the target
- * from the attention forward's own LSE), sai_distill_target_kl (target and
+ * from the attention forward's own LSE), sai_distill_target_ws (the target
+ * with a spill workspace, so long selections are gathered and multiplied
+ * once), sai_distill_target_kl (target and
  * KL in one call), sai_distill_kl_noalloc (no workspace argument),
  * sai_indexer_topk, the block selection that produces idx, scores and valid
  * from the indexer's scores, and the calls for splitting sequences across
@@ -228,6 +230,39 @@ sai_status sai_distill_target_range(const uint16_t *Q, const uint16_t *pool, con
                                     const float *window_lse, const float *sink, const int32_t *doc_start,
                                     int B, int S, int S_seq, int t_begin, int H, int D, int K, int cr,
                                     float scale, unsigned flags, float *p, int32_t *d_err, void *stream);
+
+/*
+ * sai_distill_target_workspace_bytes / sai_distill_target_ws -- the target
+ * with a spill workspace for long selections.
+ *
+ * The tensor-core kernel keeps a token's scores in tensor memory, at most
+ * 256/H tiles of 128 slots at a time (K <= 512 at H = 64). A token with more
+ * selected slots is taken in groups: the per-head log-sum-exp needs every
+ * group before any u can be formed (Primus page "perf(deepseek-v4): fuse and
+ * enable the indexer distillation loss", second commit message: the target
+ * normalises each head over the whole row). Without a workspace the groups
+ * are gathered and multiplied a second time for u. With one, the first sweep
+ * also stores each group's raw fp32 scores there, and u is formed from them:
+ * every pool row is gathered and every product formed once.
+ *
+ *   sai_distill_target_workspace_bytes(B, S, H, D, K): bytes needed on the
+ *     current device (one part per CTA of the kernel: groups x 256/H tiles x
+ *     H x 128 floats); 0 when no token can need a second group (K <= 256/H
+ *     tiles, H < 64, or a shape the tensor-core kernel does not take).
+ *   sai_distill_target_ws(...): sai_distill_target_range plus the workspace.
+ *     workspace: device memory, 16-byte aligned, owned by the caller, read
+ *     and written by the kernel, no contents required or kept between calls;
+ *     calls that overlap on the GPU must not share it. NULL, or ws_bytes
+ *     below the size above: the second sweep is used, with identical
+ *     results. Errors as for sai_distill_target_range, and SAI_ERR_ALIGN for
+ *     a misaligned workspace.
+ */
+size_t sai_distill_target_workspace_bytes(int B, int S, int H, int D, int K);
+sai_status sai_distill_target_ws(const uint16_t *Q, const uint16_t *pool, const int32_t *idx,
+                                 const float *window_lse, const float *sink, const int32_t *doc_start,
+                                 int B, int S, int S_seq, int t_begin, int H, int D, int K, int cr, float scale,
+                                 unsigned flags, float *p, int32_t *d_err, void *workspace, size_t ws_bytes,
+                                 void *stream);
 
 /* Bytes of device workspace sai_distill_target_kl needs for these sizes. */
 size_t sai_distill_target_kl_workspace_bytes(int B, int S, int K);

@@ -68,6 +68,11 @@ _lib.sai_window_lse_range.restype = _I
 _lib.sai_distill_target_range.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F,
                                           ctypes.c_uint, _P, _P, _P]
 _lib.sai_distill_target_range.restype = _I
+_lib.sai_distill_target_workspace_bytes.argtypes = [_I, _I, _I, _I, _I]
+_lib.sai_distill_target_workspace_bytes.restype = ctypes.c_size_t
+_lib.sai_distill_target_ws.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F,
+                                       ctypes.c_uint, _P, _P, _P, ctypes.c_size_t, _P]
+_lib.sai_distill_target_ws.restype = _I
 _lib.sai_count_valid_rows.argtypes = [_P, _I, _I, _I, _P, _P]
 _lib.sai_count_valid_rows.restype = _I
 _lib.sai_distill_kl_ex.argtypes = [_P, _P, _P, _I, _I, _I, _F, _P, _P, _P, _P, ctypes.c_size_t, _P]
@@ -213,11 +218,28 @@ def _target_inputs(Q, pool, idx, wl, cr, sink, doc_start, err, per_branch, full_
     return Q, pool, K, wl, sink, flags
 
 
+def target_workspace_bytes(B: int, S: int, H: int, D: int, K: int, device=None) -> int:
+    """Bytes of the raw-score spill sai_distill_target_ws uses for tokens of
+    more than one TMEM group (0 when it needs none), on `device`."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    with torch.cuda.device(dev):
+        return int(_lib.sai_distill_target_workspace_bytes(B, S, H, D, K))
+
+
+def _target_workspace(dev: torch.device, B: int, S: int, H: int, D: int, K: int):
+    nb = target_workspace_bytes(B, S, H, D, K, dev)
+    if nb == 0:
+        return None, 0
+    return torch.empty(nb, dtype=torch.uint8, device=dev), nb
+
+
 def distill_target(Q: torch.Tensor, pool: torch.Tensor, idx: Optional[torch.Tensor], wl: Optional[torch.Tensor], cr: int,
                    scale: float, sink: Optional[torch.Tensor] = None, doc_start: Optional[torch.Tensor] = None,
                    err: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
                    per_branch: bool = False, full_lse: bool = False) -> torch.Tensor:
-    """p[B,S,K] through sai_distill_target_ex. per_branch=True selects the
+    """p[B,S,K] through sai_distill_target_ws (with its spill workspace, so
+    tokens of more than one TMEM group are gathered and multiplied once).
+    per_branch=True selects the
     earlier per-branch target; wl and sink are then not used (may be None).
     full_lse=True says wl already holds lse_full, each head's log-normaliser
     over the window, the selected entries and the sink, as a CSA attention
@@ -228,9 +250,10 @@ def distill_target(Q: torch.Tensor, pool: torch.Tensor, idx: Optional[torch.Tens
     if out is None:
         out = torch.empty((B, S, K), dtype=torch.float32, device=Q.device)
     _want(out, "out", torch.float32, (B, S, K))
-    st = _call(_lib.sai_distill_target_ex, Q.device, _ptr(Q), _ptr(pool), _ptr(idx), _ptr(wl), _ptr(sink),
-               _ptr(doc_start), B, S, H, D, K, int(cr), float(scale), flags, _ptr(out), _ptr(err))
-    _check(st, "sai_distill_target_ex")
+    ws, nb = _target_workspace(Q.device, B, S, H, D, K)
+    st = _call(_lib.sai_distill_target_ws, Q.device, _ptr(Q), _ptr(pool), _ptr(idx), _ptr(wl), _ptr(sink),
+               _ptr(doc_start), B, S, S, 0, H, D, K, int(cr), float(scale), flags, _ptr(out), _ptr(err), _ptr(ws), nb)
+    _check(st, "sai_distill_target_ws")
     return out
 
 
@@ -240,7 +263,7 @@ def distill_target_range(Q: torch.Tensor, pool: torch.Tensor, idx: Optional[torc
                          err: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
                          per_branch: bool = False, full_lse: bool = False) -> torch.Tensor:
     """p for sequence positions t_begin .. t_begin+S-1 of sequences of S_seq
-    tokens, through sai_distill_target_range: Q, idx, wl and doc_start are the
+    tokens, through sai_distill_target_ws: Q, idx, wl and doc_start are the
     range's rows, pool is the whole sequence's [B,S_seq/cr,D]."""
     B, S, H, D = Q.shape
     Q, pool, K, wl, sink, flags = _target_inputs(Q, pool, idx, wl, cr, sink, doc_start, err, per_branch,
@@ -248,10 +271,11 @@ def distill_target_range(Q: torch.Tensor, pool: torch.Tensor, idx: Optional[torc
     if out is None:
         out = torch.empty((B, S, K), dtype=torch.float32, device=Q.device)
     _want(out, "out", torch.float32, (B, S, K))
-    st = _call(_lib.sai_distill_target_range, Q.device, _ptr(Q), _ptr(pool), _ptr(idx), _ptr(wl), _ptr(sink),
+    ws, nb = _target_workspace(Q.device, B, S, H, D, K)
+    st = _call(_lib.sai_distill_target_ws, Q.device, _ptr(Q), _ptr(pool), _ptr(idx), _ptr(wl), _ptr(sink),
                _ptr(doc_start), B, S, int(S_seq), int(t_begin), H, D, K, int(cr), float(scale), flags,
-               _ptr(out), _ptr(err))
-    _check(st, "sai_distill_target_range")
+               _ptr(out), _ptr(err), _ptr(ws), nb)
+    _check(st, "sai_distill_target_ws")
     return out
 
 

@@ -200,12 +200,37 @@ size_t fused_ws_bytes(const sai::KlPlan &pl)
     return a + parts;
 }
 
+// Floats of raw-score spill per CTA of the target kernel: every TMEM group of
+// a token whose K slots need more than one (H >= 64; 0 otherwise).
+size_t spill_floats_per_cta(int H, int K)
+{
+    if (!tc_heads(H) || H < 64)
+        return 0;
+    const int tb = 256 / H;
+    const int tiles = (K + 127) / 128;
+    const int groups = (tiles + tb - 1) / tb;
+    return groups > 1 ? (size_t)groups * tb * H * 128 : 0;
+}
+
+// CTAs of the target kernel for n_tok tokens.
+int target_grid(int64_t n_tok)
+{
+    int grid = sm_count();
+    if (grid <= 0)
+        return 0;
+    if (grid > n_tok)
+        grid = (int)n_tok;
+    return grid > kMaxTargetCtas ? kMaxTargetCtas : grid;
+}
+
 // S local tokens per sequence starting at position t_begin of sequences of
-// S_seq tokens (the whole sequence: S_seq == S, t_begin == 0).
+// S_seq tokens (the whole sequence: S_seq == S, t_begin == 0). ws: the
+// optional raw-score spill (NULL: tokens of more than one TMEM group are
+// gathered and multiplied twice).
 sai_status target_impl(const uint16_t *Q, const uint16_t *pool, const int32_t *idx, const float *window_lse,
                        const float *sink, const int32_t *doc_start, int B, int S, int S_seq, int t_begin, int H,
                        int D, int K, int cr, float scale, unsigned flags, float *p, int32_t *d_err,
-                       cudaStream_t st, const KlFuse *kf)
+                       cudaStream_t st, const KlFuse *kf, void *ws = nullptr, size_t ws_bytes = 0)
 {
     if ((flags & ~(SAI_TARGET_PER_BRANCH | SAI_TARGET_FULL_LSE)) ||
         (flags & (SAI_TARGET_PER_BRANCH | SAI_TARGET_FULL_LSE)) == (SAI_TARGET_PER_BRANCH | SAI_TARGET_FULL_LSE))
@@ -283,17 +308,20 @@ sai_status target_impl(const uint16_t *Q, const uint16_t *pool, const int32_t *i
         a.kl_count_blocks = 0;
         a.kl_part = nullptr;
         a.kl_done = nullptr;
+        a.spill = nullptr;
+        a.spill_stride = 0;
         CUtensorMap mq, mp;
         if (!make_map_bf16(&mq, Q, (uint64_t)B * S * H, D, (uint32_t)H) ||
             !make_map_bf16(&mp, pool, (uint64_t)B * P, D, (uint32_t)a.pool_box_rows))
             return SAI_ERR_CUDA;
-        int grid = sm_count();
+        const int grid = target_grid(a.n_tok);
         if (grid <= 0)
             return SAI_ERR_CUDA;
-        if (grid > a.n_tok)
-            grid = a.n_tok;
-        if (grid > kMaxTargetCtas)
-            grid = kMaxTargetCtas;
+        const size_t spf = spill_floats_per_cta(H, K);
+        if (spf && ws && ws_bytes >= (size_t)grid * spf * sizeof(float)) {
+            a.spill = reinterpret_cast<float *>(ws);
+            a.spill_stride = (int)spf;
+        }
         if (fuse_here) {
             // N first: per-block valid-row counts (this also zeroes the counter)
             sai_status e = cuda_status(sai::launch_kl_count(kf->plan, kf->valid, kf->ws, st));
@@ -344,6 +372,28 @@ sai_status sai_distill_target_range(const uint16_t *Q, const uint16_t *pool, con
 {
     return target_impl(Q, pool, idx, window_lse, sink, doc_start, B, S, S_seq, t_begin, H, D, K, cr, scale, flags,
                        p, d_err, reinterpret_cast<cudaStream_t>(stream), nullptr);
+}
+
+size_t sai_distill_target_workspace_bytes(int B, int S, int H, int D, int K)
+{
+    if (B < 1 || S < 1 || H < 1 || D < 1 || K < 1 || (D % 64) != 0)
+        return 0;
+    const size_t spf = spill_floats_per_cta(H, K);
+    if (!spf)
+        return 0;
+    const int grid = target_grid((int64_t)B * S);
+    return grid > 0 ? (size_t)grid * spf * sizeof(float) : 0;
+}
+
+sai_status sai_distill_target_ws(const uint16_t *Q, const uint16_t *pool, const int32_t *idx,
+                                 const float *window_lse, const float *sink, const int32_t *doc_start, int B, int S,
+                                 int S_seq, int t_begin, int H, int D, int K, int cr, float scale, unsigned flags,
+                                 float *p, int32_t *d_err, void *workspace, size_t ws_bytes, void *stream)
+{
+    if (workspace && !al16(workspace))
+        return SAI_ERR_ALIGN;
+    return target_impl(Q, pool, idx, window_lse, sink, doc_start, B, S, S_seq, t_begin, H, D, K, cr, scale, flags,
+                       p, d_err, reinterpret_cast<cudaStream_t>(stream), nullptr, workspace, ws_bytes);
 }
 
 size_t sai_distill_target_kl_workspace_bytes(int B, int S, int K)

@@ -51,6 +51,12 @@ struct TgtTcArgs {
     const int32_t *doc_start;
     float *p;             // may be NULL when the KL is fused (kl_scores set)
     int32_t *err;
+    // Raw scores of every TMEM group of a token with more than one group
+    // (H >= 64 only): [grid][spill_stride] fp32, each CTA its own part. Set:
+    // one sweep of gathers and MMAs per token, the u pass reads the scores
+    // back. NULL: the groups are gathered and multiplied a second time.
+    float *spill;
+    int spill_stride;     // floats per CTA: groups x tiles per group x H x 128
     // KL fused into the epilogue (kl_scores NULL: not fused). N comes from the
     // per-block valid-row counts of kl_count_kernel, run before on the stream.
     const float *kl_scores;     // [n_tok, K]

@@ -36,15 +36,19 @@
 // it can form u, so a token's scores stay in TMEM until it is done: up to
 // 256/H tiles (512 slots at H=64) per accumulator. Tokens alternate between
 // two 256-column accumulators, so one token's epilogue overlaps the next
-// token's MMA; both epilogue warpgroups work on each token (half the tiles
-// each), which keeps the epilogue shorter than the MMAs of a token. Tokens
-// with more selected slots run in groups: a first pass over the groups merges
-// per-head (max, sum-exp) statistics, a second pass recomputes each group and
-// forms u. When the KL stage is fused (sai_distill_target_kl), the epilogue
-// then computes each row's KL and dscores from the target in shared memory.
+// token's MMA; both epilogue warpgroups work on each token (half the heads
+// each at H >= 32). Tokens with more selected slots run in groups: a first
+// pass over the groups merges per-head (max, sum-exp) statistics, a second
+// forms u. With a spill buffer (H >= 64, its own instantiation) the first
+// pass also stores each group's raw scores there and the second reads them
+// back, so every row is gathered and multiplied once; without one the second
+// pass gathers and multiplies each group again. When the KL stage is fused
+// (sai_distill_target_kl), the epilogue then computes each row's KL and
+// dscores from the target in shared memory.
 //
 // Epilogue arithmetic (one exponential per score):
-//   M[h] = max_k z[k,h]  (column max: transposing warp butterfly + smem)
+//   M[h] = max_k z[k,h]  (per 8 columns: each warp's maximum by one redux,
+//          then the four lane quarters merged per head through smem)
 //   e[k,h] = exp(z[k,h] - M[h]) written back to TMEM, S[h] = sum_k e[k,h]
 //   a[h] = M[h] - lse_full[h],  A = max_h a[h],  w[h] = exp(a[h] - A) in (0,1]
 //   u'[k] = sum_h e[k,h] w[h]   (per thread: one TMEM lane = one slot)
@@ -149,12 +153,14 @@ __device__ __forceinline__ bool selected(int j, int t, int d0, int P, int cr)
 // behind one barrier wait, one fence and one commit; on this part a commit
 // every 4 MMAs leaves the tensor pipe idle about half the time, so CPS = 2
 // whenever D allows it.
-template <int HH, bool FUSE_KL, int CPS>
+template <int HH, bool FUSE_KL, int CPS, bool SPILL>
 __global__ void __launch_bounds__(kTgtThreads, 1)
     target_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapP,
                      const TgtTcArgs a)
 {
     constexpr int TB = 256 / HH;                 // tiles per accumulator
+    // the raw-score spill exists only in its own instantiation (H >= 64)
+    constexpr bool kSpill = SPILL && TB <= 4;
     constexpr uint32_t kQTile = HH * 128;        // one chunk of Q[t]: H rows x 128 bytes
     constexpr uint32_t kQEntry = CPS * kQTile;   // one Q ring entry
     constexpr uint32_t kAStage = CPS * kATile;   // one A ring stage: 128 rows x CPS chunks
@@ -411,7 +417,7 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
                 break;
             const int nsel = sm->nsel[m3];
             const int G = n_groups(nsel, TB);
-            const int nq = (G > 1 ? 2 : 1) * G * n_cp;
+            const int nq = (G > 1 && !kSpill ? 2 : 1) * G * n_cp;
             for (int qi = 0; qi < nq && ok; ++qi) {
                 const int c0 = (qi % n_cp) * CPS;
                 ok = warp_mbar_wait(&sm->q_empty[qs], qph ^ 1u, abort_flag, a.err);
@@ -474,7 +480,7 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
                 const uint32_t *rw = rowoff + m3 * Kp;
                 const int nt = (nsel + 127) / 128;
                 const int G = n_groups(nsel, TB);
-                const int passes = G > 1 ? 2 : 1;
+                const int passes = G > 1 && !kSpill ? 2 : 1;
                 for (int pass = 0; pass < passes && ok; ++pass) {
                     for (int grp = 0; grp < G && ok; ++grp) {
                         const int i0 = grp * TB;
@@ -574,7 +580,7 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
                 const int nsel = sm->nsel[m3];
                 const int nt = (nsel + 127) / 128;
                 const int G = n_groups(nsel, TB);
-                const int passes = G > 1 ? 2 : 1;
+                const int passes = G > 1 && !kSpill ? 2 : 1;
                 const uint32_t dbase = tmem + mb * 256;
                 for (int pass = 0; pass < passes && ok; ++pass) {
                     for (int grp = 0; grp < G && ok; ++grp) {
@@ -723,6 +729,10 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
             const int nt = (nsel + 127) / 128;
             const int G = n_groups(nsel, TB);
             const int passes = G > 1 ? 2 : 1;
+            // more than one group and a spill buffer: the second pass reads the
+            // groups' raw scores back instead of waiting for them again
+            const bool spill = kSpill && G > 1;
+            float *scr = kSpill ? a.spill + (size_t)blockIdx.x * a.spill_stride : nullptr;
             float *prow = a.p + (size_t)g * K;
             const int32_t *sl = slot + m3 * Kp;
             const bool ident = sm->ident[m3] != 0;    // slot jj of the compacted order is slot jj
@@ -752,24 +762,27 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
                     // this warpgroup's tiles of the group: [t0, t1) (possibly empty)
                     const int t0 = hf * TBH;
                     const int t1 = min(ntg, t0 + TBH);
-                    named_bar_sync(bar_id, kEpiThreads);   // st.flag is free again
-                    if (ew == 0) {
-                        const int jb = mb ? jobs1 : jobs0;
-                        const bool f = warp_mbar_wait(&sm->acc_full[mb], jb & 1, abort_flag, a.err);
-                        if (lane == 0)
-                            st.flag = f ? 1 : 0;
-                        __syncwarp();
+                    const bool from_spill = spill && pass == 1;   // this group's scores are in scr
+                    if (!from_spill) {
+                        named_bar_sync(bar_id, kEpiThreads);   // st.flag is free again
+                        if (ew == 0) {
+                            const int jb = mb ? jobs1 : jobs0;
+                            const bool f = warp_mbar_wait(&sm->acc_full[mb], jb & 1, abort_flag, a.err);
+                            if (lane == 0)
+                                st.flag = f ? 1 : 0;
+                            __syncwarp();
+                        }
+                        named_bar_sync(bar_id, kEpiThreads);
+                        if (mb)
+                            ++jobs1;
+                        else
+                            ++jobs0;
+                        if (!st.flag) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
                     }
-                    named_bar_sync(bar_id, kEpiThreads);
-                    if (mb)
-                        ++jobs1;
-                    else
-                        ++jobs0;
-                    if (!st.flag) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
                     const bool single = (G == 1);
                     if constexpr (HH >= 32) {
                     if (pass == 0) {
@@ -791,6 +804,17 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
                                 if (i < ntg)
                                     tmem_ld8(tbase + i * HH + col0, v[i]);
                             tmem_ld_wait();
+                            if (spill) {
+                                // raw scores, lane-contiguous per (tile, head)
+#pragma unroll
+                                for (int i = 0; i < TB; ++i)
+                                    if (i < ntg) {
+                                        float *dst = scr + ((size_t)(grp * TB + i) * HH + col0) * 128 + r;
+#pragma unroll
+                                        for (int e = 0; e < 8; ++e)
+                                            __stcg(dst + e * 128, __uint_as_float(v[i][e]));
+                                    }
+                            }
                             float m8[8];
 #pragma unroll
                             for (int e = 0; e < 8; ++e)
@@ -1157,11 +1181,22 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
                                 if (ib >= ntg)
                                     break;
                                 uint32_t v[IB][16];
+                                if (from_spill) {
 #pragma unroll
-                                for (int i = 0; i < IB; ++i)
-                                    if (ib + i < ntg)
-                                        tmem_ld16(tbase + (ib + i) * HH + col0, v[i]);
-                                tmem_ld_wait();
+                                    for (int i = 0; i < IB; ++i)
+                                        if (ib + i < ntg) {
+                                            const float *src = scr + ((size_t)(grp * TB + ib + i) * HH + col0) * 128 + r;
+#pragma unroll
+                                            for (int e = 0; e < 16; ++e)
+                                                v[i][e] = __float_as_uint(__ldcg(src + e * 128));
+                                        }
+                                } else {
+#pragma unroll
+                                    for (int i = 0; i < IB; ++i)
+                                        if (ib + i < ntg)
+                                            tmem_ld16(tbase + (ib + i) * HH + col0, v[i]);
+                                    tmem_ld_wait();
+                                }
 #pragma unroll
                                 for (int i = 0; i < IB; ++i) {
                                     if (ib + i < ntg) {
@@ -1245,11 +1280,13 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
                         }
                         }
                     }
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0)
-                        mbar_arrive(&sm->acc_empty[mb]);
-                    __syncwarp();
+                    if (!from_spill) {
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0)
+                            mbar_arrive(&sm->acc_empty[mb]);
+                        __syncwarp();
+                    }
                 }
             }
             if (!ok)
@@ -1423,14 +1460,14 @@ size_t smem_bytes_for(int K, int stages)
     return fixed_smem_bytes<HH, CPS>(K) + (size_t)stages * CPS * kATile;
 }
 
-template <int HH, bool FUSE_KL, int CPS>
-cudaError_t launch_hkc(const CUtensorMap &mapQ, const CUtensorMap &mapP, const TgtTcArgs &a, int grid,
+template <int HH, bool FUSE_KL, int CPS, bool SPILL>
+cudaError_t launch_hkcs(const CUtensorMap &mapQ, const CUtensorMap &mapP, const TgtTcArgs &a, int grid,
                        cudaStream_t stream)
 {
     // The register split above is only safe if every thread was launched with
     // exactly kLaunchRegs registers; refuse to launch otherwise.
     cudaFuncAttributes fa;
-    cudaError_t e = cudaFuncGetAttributes(&fa, target_tc_kernel<HH, FUSE_KL, CPS>);
+    cudaError_t e = cudaFuncGetAttributes(&fa, target_tc_kernel<HH, FUSE_KL, CPS, SPILL>);
     if (e != cudaSuccess)
         return e;
     if (fa.numRegs != kLaunchRegs)
@@ -1438,12 +1475,26 @@ cudaError_t launch_hkc(const CUtensorMap &mapQ, const CUtensorMap &mapP, const T
     if (a.n_astages < 1 || kGatherWarps % a.n_astages != 0 || (a.D / 64) % CPS != 0)
         return cudaErrorInvalidValue;
     const size_t smem = smem_bytes_for<HH, CPS>(a.K, a.n_astages);
-    e = cudaFuncSetAttribute(target_tc_kernel<HH, FUSE_KL, CPS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(target_tc_kernel<HH, FUSE_KL, CPS, SPILL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem);
     if (e != cudaSuccess)
         return e;
-    target_tc_kernel<HH, FUSE_KL, CPS><<<grid, kTgtThreads, smem, stream>>>(mapQ, mapP, a);
+    target_tc_kernel<HH, FUSE_KL, CPS, SPILL><<<grid, kTgtThreads, smem, stream>>>(mapQ, mapP, a);
     return cudaGetLastError();
+}
+
+// The spill instantiation only where it can be used (H >= 64, no fused KL).
+template <int HH, bool FUSE_KL, int CPS>
+cudaError_t launch_hkc(const CUtensorMap &mapQ, const CUtensorMap &mapP, const TgtTcArgs &a, int grid,
+                       cudaStream_t stream)
+{
+    if constexpr (HH >= 64 && !FUSE_KL) {
+        if (a.spill)
+            return launch_hkcs<HH, FUSE_KL, CPS, true>(mapQ, mapP, a, grid, stream);
+    }
+    if (a.spill)
+        return cudaErrorInvalidValue;
+    return launch_hkcs<HH, FUSE_KL, CPS, false>(mapQ, mapP, a, grid, stream);
 }
 
 template <int HH, bool FUSE_KL>

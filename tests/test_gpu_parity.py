@@ -9,6 +9,8 @@ benchmark times. Tolerances (tests/gpu_util.py): p 1e-5, loss 1e-4 relative,
 dscores 1e-6 (and 1e-3 of max|dscores|), window_lse 1e-5 relative to max(1,|x|).
 Index and mask work must be exact: p and dscores are exactly 0 on masked slots.
 """
+import ctypes
+
 import numpy as np
 import pytest
 
@@ -178,6 +180,35 @@ def test_multi_group_tokens(sai):
     assert_close("window_lse", wl.cpu().numpy().reshape(-1, w.H)[tok] - owl, 0 * owl, tol_wl(owl))
     assert_close("p", p.cpu().numpy().reshape(-1, w.K)[tok], op, TOL_P)
     assert_close("dscores", ds.cpu().numpy().reshape(-1, w.K)[tok], ods, TOL_DS)
+
+
+@pytest.mark.parametrize("K,S", [(576, 2304), (1000, 4096), (2048, 8192)])
+def test_spill_matches_second_sweep(sai, K, S):
+    """Tokens of two to four TMEM groups (K > 512 at H=64): the target with its
+    raw-score spill (one sweep of gathers and MMAs) is bit-identical to the
+    two-sweep target without a workspace, and both match the oracle on late
+    tokens (the most groups) and a sample of the rest. K=1000 leaves a
+    ragged last group."""
+    w = workload(f"long_s{S}_k{K}", name="long", S=S, K=K)
+    t = to_dev(w)
+    B, H, D = w.B, w.H, w.D
+    assert sai.target_workspace_bytes(B, S, H, D, K) > 0
+    wl = sai.window_lse(t["Q"], t["Kw"], w.W, w.scale, t["doc_start"])
+    p_ws = sai.distill_target(t["Q"], t["pool"], t["idx"], wl, w.cr, w.scale, sink=t["sink"],
+                              doc_start=t["doc_start"])
+    p_two = torch.full((B, S, K), float("nan"), device="cuda")
+    lib = sai.lib()
+    st = lib.sai_distill_target_ws(
+        ctypes.c_void_p(t["Q"].data_ptr()), ctypes.c_void_p(t["pool"].data_ptr()),
+        ctypes.c_void_p(t["idx"].data_ptr()), ctypes.c_void_p(wl.data_ptr()),
+        ctypes.c_void_p(t["sink"].data_ptr()), None, B, S, S, 0, H, D, K, w.cr, ctypes.c_float(w.scale), 0,
+        ctypes.c_void_p(p_two.data_ptr()), None, None, 0, ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert st == 0
+    torch.cuda.synchronize()
+    assert torch.equal(p_ws, p_two)
+    tok = np.unique(np.concatenate([np.arange(w.S - 24, w.S), synth.sample_tokens(w.B, w.S, 24)]))
+    _, op, _, _, _ = oracle.run_all(w, tok)
+    assert_close("p", p_ws.cpu().numpy().reshape(-1, w.K)[tok], op, TOL_P)
 
 
 def test_deterministic(sai):
