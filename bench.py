@@ -48,6 +48,8 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--long-steps", type=int, default=30,
                     help="timed steps of the long-context side line (0: skip it)")
+    ap.add_argument("--packed-steps", type=int, default=50,
+                    help="timed steps of the packed-documents side line (0: skip it)")
     return ap.parse_args()
 
 
@@ -272,6 +274,62 @@ def run_reference(args):
     return 0
 
 
+
+def side_line(name, steps, dev, stream, rank, err, flush_l2):
+    """window_lse -> distill_target -> distill_kl on another workload, `steps`
+    timed steps after 3 warm-up steps, L2 flushed before each; the target's
+    spill workspace and the KL's are allocated once, outside the timed loop."""
+    import torch
+    import sparse_attention_indexer_window_b200 as sai
+    from sparse_attention_indexer_window_b200 import shard
+    import synth
+    wX = synth.make(name, seed=shard.rank_seed(synth.CONFIGS[name].seed, rank))
+    tX = to_dev(wX, dev)
+    wl = torch.empty((wX.B, wX.S, wX.H), device=dev)
+    p = torch.empty((wX.B, wX.S, wX.K), device=dev)
+    ds = torch.empty((wX.B, wX.S, wX.K), device=dev)
+    loss = torch.empty(1, device=dev)
+    ws_kl = torch.empty(sai.kl_workspace_bytes(wX.B, wX.S, wX.K), dtype=torch.uint8, device=dev)
+    nb = sai.target_workspace_bytes(wX.B, wX.S, wX.H, wX.D, wX.K, dev)
+    ws_t = torch.empty(nb, dtype=torch.uint8, device=dev) if nb else None
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    for i in range(3 + steps):
+        flush_l2(i)
+        if i >= 3:
+            ev[i - 3][0].record(stream)
+        sai.window_lse(tX["Q"], tX["Kw"], wX.W, wX.scale, tX["doc_start"], out=wl)
+        if i >= 3:
+            ev[i - 3][1].record(stream)
+        sai.distill_target(tX["Q"], tX["pool"], tX["idx"], wl, wX.cr, wX.scale, sink=tX["sink"],
+                           doc_start=tX["doc_start"], err=err, out=p, workspace=ws_t)
+        if i >= 3:
+            ev[i - 3][2].record(stream)
+        sai.distill_kl(p, tX["scores"], tX["valid"], wX.coeff, workspace=ws_kl, loss=loss, dscores=ds)
+        if i >= 3:
+            ev[i - 3][3].record(stream)
+    torch.cuda.synchronize(dev)
+    assert int(err.item()) == 0
+    sel, win = algorithmic_counts(wX)
+    ms = statistics.mean(e[0].elapsed_time(e[3]) for e in ev)
+    tgt = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
+    recipe = {"long": "random distinct causal blocks, -1 tail",
+              "packed": "top-K of a random causal score per document, sorted ascending"}[name]
+    line = {
+        "workload": f"{name}: B={wX.B} S={wX.S} H={wX.H} D={wX.D} cr={wX.cr} K={wX.K} W={wX.W}, {recipe}; "
+                    f"same value distributions",
+        "steps": steps, "ms_per_step": ms, "tokens_per_s": wX.B * wX.S / (ms / 1e3),
+        "kernels_ms": {"window_lse": statistics.mean(e[0].elapsed_time(e[1]) for e in ev),
+                       "distill_target": tgt,
+                       "distill_kl": statistics.mean(e[2].elapsed_time(e[3]) for e in ev)},
+        "selected_slots": sel, "window_keys": win,
+        "distill_target_tflops": 2.0 * wX.H * wX.D * sel / (tgt / 1e3) / 1e12,
+        "step_tflops": 2.0 * wX.H * wX.D * (sel + win) / (ms / 1e3) / 1e12,
+        "target_spill_workspace_bytes": nb,
+    }
+    del tX
+    torch.cuda.empty_cache()
+    return line
+
 def main():
     args = parse()
     if args.impl == "reference":
@@ -427,53 +485,16 @@ def main():
     sel_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in sel_ev)
     del isc
 
-    # ------------------------------------------- long context (side line)
+    # ------------------------------------------- side lines: long, packed
     # The same three calls on the long-context workload (S=16384, K=2048: up
-    # to 2048 selected blocks per token), timed like the step above; not part
-    # of `value`.
-    long_line = None
-    if args.long_steps > 0:
-        del t
-        torch.cuda.empty_cache()
-        wL = synth.make("long", seed=shard.rank_seed(synth.CONFIGS["long"].seed, rank))
-        tL = to_dev(wL, dev)
-        wlL = torch.empty((wL.B, wL.S, wL.H), device=dev)
-        pL = torch.empty((wL.B, wL.S, wL.K), device=dev)
-        dsL = torch.empty((wL.B, wL.S, wL.K), device=dev)
-        lossL = torch.empty(1, device=dev)
-        wsL = torch.empty(sai.kl_workspace_bytes(wL.B, wL.S, wL.K), dtype=torch.uint8, device=dev)
-        evL = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.long_steps)]
-        for i in range(3 + args.long_steps):
-            flush_l2(i)
-            if i >= 3:
-                evL[i - 3][0].record(stream)
-            sai.window_lse(tL["Q"], tL["Kw"], wL.W, wL.scale, tL["doc_start"], out=wlL)
-            if i >= 3:
-                evL[i - 3][1].record(stream)
-            sai.distill_target(tL["Q"], tL["pool"], tL["idx"], wlL, wL.cr, wL.scale, sink=tL["sink"],
-                               doc_start=tL["doc_start"], err=err, out=pL)
-            if i >= 3:
-                evL[i - 3][2].record(stream)
-            sai.distill_kl(pL, tL["scores"], tL["valid"], wL.coeff, workspace=wsL, loss=lossL, dscores=dsL)
-            if i >= 3:
-                evL[i - 3][3].record(stream)
-        torch.cuda.synchronize(dev)
-        assert int(err.item()) == 0
-        selL, winL = algorithmic_counts(wL)
-        msL = statistics.mean(e[0].elapsed_time(e[3]) for e in evL)
-        tgtL = statistics.mean(e[1].elapsed_time(e[2]) for e in evL)
-        long_line = {
-            "workload": f"long: B={wL.B} S={wL.S} H={wL.H} D={wL.D} cr={wL.cr} K={wL.K} W={wL.W}, random "
-                        f"distinct causal blocks, -1 tail; same value distributions",
-            "steps": args.long_steps, "ms_per_step": msL, "tokens_per_s": wL.B * wL.S / (msL / 1e3),
-            "kernels_ms": {"window_lse": statistics.mean(e[0].elapsed_time(e[1]) for e in evL),
-                           "distill_target": tgtL,
-                           "distill_kl": statistics.mean(e[2].elapsed_time(e[3]) for e in evL)},
-            "selected_slots": selL, "window_keys": winL,
-            "distill_target_tflops": 2.0 * wL.H * wL.D * selL / (tgtL / 1e3) / 1e12,
-            "step_tflops": 2.0 * wL.H * wL.D * (selL + winL) / (msL / 1e3) / 1e12,
-        }
-        del tL
+    # to 2048 selected blocks per token) and the packed one (B=4, two
+    # documents per row), timed like the step above; not part of `value`.
+    del t
+    torch.cuda.empty_cache()
+    long_line = side_line("long", args.long_steps, dev, stream, rank, err, flush_l2) \
+        if args.long_steps > 0 else None
+    packed_line = side_line("packed", args.packed_steps, dev, stream, rank, err, flush_l2) \
+        if args.packed_steps > 0 else None
 
     # batch-wide loss over all ranks, for the record (not part of the timed path)
     n_rows = int((w.valid.reshape(-1, K) != 0).any(axis=1).sum())
@@ -540,13 +561,15 @@ def main():
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "steps": args.e2e_steps},
             "long": long_line,
+            "packed": packed_line,
             "gpu_launches": 3 * nsteps * world,   # window, target, KL (one cooperative launch); every rank
             "clocks": clk,
             "loss": loss_all,
         }
-        if long_line is not None:
-            long_line["distill_target_frac"] = long_line["distill_target_tflops"] / peak_tf
-            long_line["step_frac"] = long_line["step_tflops"] / peak_tf
+        for sl in (long_line, packed_line):
+            if sl is not None:
+                sl["distill_target_frac"] = sl["distill_target_tflops"] / peak_tf
+                sl["step_frac"] = sl["step_tflops"] / peak_tf
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
         print(json.dumps(line), flush=True)

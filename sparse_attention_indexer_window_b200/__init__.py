@@ -226,17 +226,26 @@ def target_workspace_bytes(B: int, S: int, H: int, D: int, K: int, device=None) 
         return int(_lib.sai_distill_target_workspace_bytes(B, S, H, D, K))
 
 
-def _target_workspace(dev: torch.device, B: int, S: int, H: int, D: int, K: int):
+def _target_workspace(dev: torch.device, B: int, S: int, H: int, D: int, K: int,
+                      given: Optional[torch.Tensor] = None):
+    """The spill workspace: the caller's (uint8, on dev, large enough), else a
+    new one when the shape needs it."""
     nb = target_workspace_bytes(B, S, H, D, K, dev)
     if nb == 0:
         return None, 0
+    if given is not None:
+        _want(given, "workspace", torch.uint8)
+        if given.numel() < nb:
+            raise ValueError(f"workspace holds {given.numel()} bytes, {nb} needed")
+        return given, given.numel()
     return torch.empty(nb, dtype=torch.uint8, device=dev), nb
 
 
 def distill_target(Q: torch.Tensor, pool: torch.Tensor, idx: Optional[torch.Tensor], wl: Optional[torch.Tensor], cr: int,
                    scale: float, sink: Optional[torch.Tensor] = None, doc_start: Optional[torch.Tensor] = None,
                    err: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
-                   per_branch: bool = False, full_lse: bool = False) -> torch.Tensor:
+                   per_branch: bool = False, full_lse: bool = False,
+                   workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
     """p[B,S,K] through sai_distill_target_ws (with its spill workspace, so
     tokens of more than one TMEM group are gathered and multiplied once).
     per_branch=True selects the
@@ -250,7 +259,7 @@ def distill_target(Q: torch.Tensor, pool: torch.Tensor, idx: Optional[torch.Tens
     if out is None:
         out = torch.empty((B, S, K), dtype=torch.float32, device=Q.device)
     _want(out, "out", torch.float32, (B, S, K))
-    ws, nb = _target_workspace(Q.device, B, S, H, D, K)
+    ws, nb = _target_workspace(Q.device, B, S, H, D, K, workspace)
     st = _call(_lib.sai_distill_target_ws, Q.device, _ptr(Q), _ptr(pool), _ptr(idx), _ptr(wl), _ptr(sink),
                _ptr(doc_start), B, S, S, 0, H, D, K, int(cr), float(scale), flags, _ptr(out), _ptr(err), _ptr(ws), nb)
     _check(st, "sai_distill_target_ws")
