@@ -262,13 +262,21 @@ sai_status target_impl(const uint16_t *Q, const uint16_t *pool, const int32_t *i
 
     // the tensor-core kernel addresses pool rows with 32-bit byte offsets
     const bool pool_fits = (uint64_t)B * P * D * 2 < 0xffffffffull;
-    // two 64-column chunks of D per pipeline stage where D and shared memory
-    // allow it (half the per-stage synchronisation), else one
-    int cps = (D % 128) == 0 ? 2 : 1;
-    int n_astages = tc_heads(H) && (D % 64) == 0 && pool_fits ? sai::target_tc_stages(H, K, cps, smem_cap) : 0;
-    if (n_astages == 0 && cps == 2) {
-        cps = 1;
-        n_astages = tc_heads(H) && (D % 64) == 0 && pool_fits ? sai::target_tc_stages(H, K, cps, smem_cap) : 0;
+    // Shared-memory layout, the first that fits: two 64-column chunks of D
+    // per pipeline stage (half the per-stage synchronisation) with a
+    // four-token compaction ring and staged idx rows; the same with a
+    // two-token ring and idx read from global memory (large K); then one
+    // chunk per stage, in the same two forms.
+    const bool idx_vec = idx && (K % 4) == 0 && al16(idx);
+    const bool tc_ok = tc_heads(H) && (D % 64) == 0 && pool_fits;
+    int cps = 1, n_meta = 4, idx_stage = 0, n_astages = 0;
+    for (int c = 0; c < 4 && tc_ok && n_astages == 0; ++c) {
+        cps = (c < 2 && (D % 128) == 0) ? 2 : 1;
+        if (c < 2 && cps == 1)
+            continue;
+        n_meta = (c % 2 == 0) ? 4 : 2;
+        idx_stage = (c % 2 == 0 && idx_vec) ? 1 : 0;
+        n_astages = sai::target_tc_stages(H, K, cps, n_meta, idx_stage, smem_cap);
     }
     // the epilogue computes the KL from two slots per thread (K <= 512)
     const bool fuse_here = kf && n_astages > 0 && K <= 512;
@@ -286,7 +294,9 @@ sai_status target_impl(const uint16_t *Q, const uint16_t *pool, const int32_t *i
         a.t_begin = t_begin;
         a.n_tok = B * S;
         a.tiles_per_group = 256 / H;
-        a.idx_bulk = (idx && (K % 4) == 0 && al16(idx)) ? 1 : 0;
+        a.idx_bulk = idx_vec ? 1 : 0;
+        a.idx_stage = idx_stage;
+        a.n_meta = n_meta;
         a.n_astages = n_astages;
         a.cps = cps;
         a.lse_mode = lse_mode;

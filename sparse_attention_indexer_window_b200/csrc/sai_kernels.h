@@ -38,7 +38,9 @@ struct TgtTcArgs {
     int t_begin;          // sequence position of local token 0 (token-range calls; else 0)
     int n_tok;            // B*S
     int tiles_per_group;  // 128-slot tiles per TMEM accumulator (256 / H)
-    int idx_bulk;         // idx rows are 16-byte aligned (K % 4 == 0): stage them by bulk copy
+    int idx_bulk;         // idx rows are 16-byte aligned (K % 4 == 0): read 16 bytes at a time
+    int idx_stage;        // idx rows staged in shared memory two tokens ahead (needs idx_bulk)
+    int n_meta;           // compaction ring depth: 4, or 2 where shared memory is short (large K)
     int n_astages;        // depth of the gathered-row stage ring (divides 8)
     int cps;              // 64-column chunks of D per stage (1 or 2; D/64 % cps == 0)
     int pool_box_rows;    // rows of the pool's TMA box (min(128, B*P))
@@ -70,8 +72,9 @@ struct TgtTcArgs {
     uint32_t *kl_done;          // completion counter, zeroed by kl_count_kernel
 };
 // Deepest gathered-row stage ring of `cps`-chunk stages that fits
-// `smem_limit` bytes (0: none).
-int target_tc_stages(int H, int K, int cps, int smem_limit);
+// `smem_limit` bytes beside a compaction ring of n_meta tokens, with or
+// without the staged idx rows (0: none).
+int target_tc_stages(int H, int K, int cps, int n_meta, int idx_stage, int smem_limit);
 cudaError_t launch_target_tc(const CUtensorMap &mapQ, const CUtensorMap &mapP, const TgtTcArgs &a, int grid,
                              cudaStream_t stream);
 

@@ -97,7 +97,7 @@ constexpr int kQStagesMax = 6;
 // CPS chunks (the chunks one stage's MMAs read); at least two entries.
 template <int HH, int CPS>
 constexpr int q_entries() { return (HH <= 64 ? 6 : 3) / CPS >= 2 ? (HH <= 64 ? 6 : 3) / CPS : 2; }
-constexpr int kMeta = 4;                            // compaction runs up to three tokens ahead
+constexpr int kMeta = 4;   // compaction ring: at most four tokens (a.n_meta: 4, or 2 for large K)
 constexpr uint32_t kATile = 128 * 128;              // 128 rows x 128 bytes
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLnFltMin = -87.33654475055310898657f;  // log(2^-126)
@@ -175,10 +175,12 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
     constexpr int QS = q_entries<HH, CPS>();
     uint8_t *q_buf = a_buf + NA * kAStage;                                   // QS x kQEntry
     // byte offset in pool of every selected slot's row, compacted per token
-    uint32_t *rowoff = reinterpret_cast<uint32_t *>(q_buf + QS * kQEntry);   // [kMeta][Kp]
-    int32_t *slot = reinterpret_cast<int32_t *>(rowoff + kMeta * Kp);        // [kMeta][Kp]
-    int32_t *idxs = slot + kMeta * Kp;                                       // [3][Kp] staged idx rows
-    float *ubuf = reinterpret_cast<float *>(idxs + 3 * Kp);                  // [Kp] u' of a token
+    const int NM = a.n_meta;                 // compaction ring depth (4, or 2 for large K)
+    const bool idx_stage = a.idx_stage != 0; // idx rows staged in smem (else read from global)
+    uint32_t *rowoff = reinterpret_cast<uint32_t *>(q_buf + QS * kQEntry);   // [NM][Kp]
+    int32_t *slot = reinterpret_cast<int32_t *>(rowoff + NM * Kp);           // [NM][Kp]
+    int32_t *idxs = slot + NM * Kp;                                          // [3][Kp] staged idx rows
+    float *ubuf = reinterpret_cast<float *>(idxs + (idx_stage ? 3 * Kp : 0)); // [Kp] u' of a token
     // then [2][TB*128] partial u of the two epilogue warpgroups (H >= 32)
     TgtSmem<HH> *sm = reinterpret_cast<TgtSmem<HH> *>(ubuf + Kp + (HH >= 32 ? 2 * TB * 128 : 0));
 
@@ -187,7 +189,7 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
     const int n_chunks = a.D / 64;
     const int n_cp = n_chunks / CPS;             // stages per tile (D / 64 is a multiple of CPS)
     const int WPS = kGatherWarps / NA;           // gather warps filling each A slot
-    const bool idx_bulk = a.idx_bulk != 0;       // idx rows staged by bulk copy
+    const bool idx_bulk = a.idx_bulk != 0;       // idx rows 16-byte aligned, K % 4 == 0
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < NA; ++s) {
@@ -202,7 +204,7 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
             mbar_init(&sm->acc_full[b], 2);     // both MMA threads commit a group
             mbar_init(&sm->acc_empty[b], 8);    // lane 0 of each epilogue warp
         }
-        for (int b = 0; b < kMeta; ++b) {
+        for (int b = 0; b < NM; ++b) {
             mbar_init(&sm->meta_full[b], 1);
             mbar_init(&sm->meta_empty[b], 1);
         }
@@ -232,7 +234,7 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
         // SM and arrived late.)
         const int n_vec = K / 4;                 // 16-byte pieces of an idx row (idx_bulk: K % 4 == 0)
         auto stage_idx = [&](int gts, int buf) {
-            if (idx_bulk && gts < a.n_tok) {
+            if (idx_stage && gts < a.n_tok) {
                 const int gs = a.n_tok - 1 - gts;
                 const char *src = reinterpret_cast<const char *>(a.idx + (size_t)gs * K);
                 const uint32_t dst = smem_u32(idxs + buf * Kp);
@@ -249,12 +251,12 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
             const int g = a.n_tok - 1 - gt;
             const int b = g / a.S;
             const int t = g - b * a.S + a.t_begin;   // sequence position
-            const int m3 = it % kMeta;
+            const int m3 = it % NM;
             int32_t *ib = idxs + (it % 3) * Kp;
             stage_idx(gt + 2 * (int)gridDim.x, (it + 2) % 3);
             cp_async_wait<2>();                  // this token's row has landed
             __syncwarp();
-            ok = warp_mbar_wait(&sm->meta_empty[m3], ((it / kMeta) & 1) ^ 1u, abort_flag, a.err);
+            ok = warp_mbar_wait(&sm->meta_empty[m3], ((it / NM) & 1) ^ 1u, abort_flag, a.err);
             if (!ok)
                 break;
             int d0 = 0;
@@ -289,7 +291,8 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
                 if (idx_bulk) {
                     int4 v = make_int4(-1, -1, -1, -1);
                     if (k < K)
-                        v = *reinterpret_cast<const int4 *>(ib + k);
+                        v = idx_stage ? *reinterpret_cast<const int4 *>(ib + k)
+                                      : __ldg(reinterpret_cast<const int4 *>(grow + k));
                     j[0] = v.x;
                     j[1] = v.y;
                     j[2] = v.z;
@@ -342,7 +345,8 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
                 if (idx_bulk) {
                     int4 v = make_int4(-1, -1, -1, -1);
                     if (k < K)
-                        v = *reinterpret_cast<const int4 *>(ib + k);
+                        v = idx_stage ? *reinterpret_cast<const int4 *>(ib + k)
+                                      : __ldg(reinterpret_cast<const int4 *>(grow + k));
                     j[0] = v.x;
                     j[1] = v.y;
                     j[2] = v.z;
@@ -411,8 +415,8 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
             tma_prefetch_desc(&mapQ);
         for (int gt = blockIdx.x; gt < a.n_tok && ok; gt += gridDim.x, ++it) {
             const int g = a.n_tok - 1 - gt;
-            const int m3 = it % kMeta;
-            ok = warp_mbar_wait(&sm->meta_full[m3], (it / kMeta) & 1, abort_flag, a.err);
+            const int m3 = it % NM;
+            ok = warp_mbar_wait(&sm->meta_full[m3], (it / NM) & 1, abort_flag, a.err);
             if (!ok)
                 break;
             const int nsel = sm->nsel[m3];
@@ -471,8 +475,8 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
             bool ok = true;
             int it = 0;
             for (int gt = blockIdx.x; gt < a.n_tok && ok; gt += gridDim.x, ++it) {
-                const int m3 = it % kMeta;
-                ok = warp_mbar_wait(&sm->meta_full[m3], (it / kMeta) & 1, abort_flag, a.err);
+                const int m3 = it % NM;
+                ok = warp_mbar_wait(&sm->meta_full[m3], (it / NM) & 1, abort_flag, a.err);
                 if (!ok)
                     break;
                 const int nsel = sm->nsel[m3];
@@ -572,8 +576,8 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
             int jobs0 = 0, jobs1 = 0;
             for (int gt = blockIdx.x; gt < a.n_tok && ok; gt += gridDim.x, ++it) {
                 const int mb = it & 1;
-                const int m3 = it % kMeta;
-                if (!mbar_wait(&sm->meta_full[m3], (it / kMeta) & 1, abort_flag, a.err)) {
+                const int m3 = it % NM;
+                if (!mbar_wait(&sm->meta_full[m3], (it / NM) & 1, abort_flag, a.err)) {
                     ok = false;
                     break;
                 }
@@ -711,13 +715,13 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
         for (int it = 0; blockIdx.x + it * (int)gridDim.x < a.n_tok; ++it) {
             const int gt = blockIdx.x + it * gridDim.x;
             const int g = a.n_tok - 1 - gt;
-            const int m3 = it % kMeta;
+            const int m3 = it % NM;
             const int mb = it & 1;
             // window log-mass of this token's heads, fetched early
             const float wl_h = (et < HH && a.wl) ? a.wl[(size_t)g * HH + et] : 0.f;
             // leader waits; the named barrier hands the outcome to everyone
             if (ew == 0) {
-                const bool f = warp_mbar_wait(&sm->meta_full[m3], (it / kMeta) & 1, abort_flag, a.err);
+                const bool f = warp_mbar_wait(&sm->meta_full[m3], (it / NM) & 1, abort_flag, a.err);
                 if (lane == 0)
                     st.flag = f ? 1 : 0;
                 __syncwarp();
@@ -1430,21 +1434,21 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
 }
 
 template <int HH, int CPS>
-__host__ __device__ inline size_t fixed_smem_bytes(int K)
+__host__ __device__ inline size_t fixed_smem_bytes(int K, int n_meta, int idx_stage)
 {
     const size_t Kp = (size_t)((K + 3) & ~3);
     const size_t uh = HH >= 32 ? (size_t)2 * (256 / HH) * 128 * 4 : 0;   // partial u of the two warpgroups
-    return 1024 + q_entries<HH, CPS>() * (size_t)(CPS * HH * 128) + Kp * 4 * (2 * kMeta + 4) + uh +
-           sizeof(TgtSmem<HH>) + 64;
+    const size_t rows = 2 * (size_t)n_meta + (idx_stage ? 3 : 0) + 1;    // row offsets, slots, idx, u'
+    return 1024 + q_entries<HH, CPS>() * (size_t)(CPS * HH * 128) + Kp * 4 * rows + uh + sizeof(TgtSmem<HH>) + 64;
 }
 
 // Deepest A-stage ring that fits the per-block smem limit, as a divisor of
 // the eight gather warps (so every slot has the same number of producers),
 // with two slots at least for each of the two MMA threads; 0 if none fits.
 template <int HH, int CPS>
-int stages_for(int K, int smem_limit)
+int stages_for(int K, int n_meta, int idx_stage, int smem_limit)
 {
-    const long room = (long)smem_limit - (long)fixed_smem_bytes<HH, CPS>(K);
+    const long room = (long)smem_limit - (long)fixed_smem_bytes<HH, CPS>(K, n_meta, idx_stage);
     long n = room / (long)(CPS * kATile);
     if (n > kMaxAStages)
         n = kMaxAStages;
@@ -1455,9 +1459,9 @@ int stages_for(int K, int smem_limit)
 }
 
 template <int HH, int CPS>
-size_t smem_bytes_for(int K, int stages)
+size_t smem_bytes_for(int K, int n_meta, int idx_stage, int stages)
 {
-    return fixed_smem_bytes<HH, CPS>(K) + (size_t)stages * CPS * kATile;
+    return fixed_smem_bytes<HH, CPS>(K, n_meta, idx_stage) + (size_t)stages * CPS * kATile;
 }
 
 template <int HH, bool FUSE_KL, int CPS, bool SPILL>
@@ -1472,9 +1476,10 @@ cudaError_t launch_hkcs(const CUtensorMap &mapQ, const CUtensorMap &mapP, const 
         return e;
     if (fa.numRegs != kLaunchRegs)
         return cudaErrorInvalidConfiguration;
-    if (a.n_astages < 1 || kGatherWarps % a.n_astages != 0 || (a.D / 64) % CPS != 0)
+    if (a.n_astages < 1 || kGatherWarps % a.n_astages != 0 || (a.D / 64) % CPS != 0 ||
+        (a.n_meta != 2 && a.n_meta != 4) || (a.idx_stage && !a.idx_bulk))
         return cudaErrorInvalidValue;
-    const size_t smem = smem_bytes_for<HH, CPS>(a.K, a.n_astages);
+    const size_t smem = smem_bytes_for<HH, CPS>(a.K, a.n_meta, a.idx_stage, a.n_astages);
     e = cudaFuncSetAttribute(target_tc_kernel<HH, FUSE_KL, CPS, SPILL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem);
     if (e != cudaSuccess)
@@ -1514,20 +1519,21 @@ cudaError_t launch_h(const CUtensorMap &mapQ, const CUtensorMap &mapP, const Tgt
 }
 
 template <int HH>
-int stages_h(int K, int cps, int smem_limit)
+int stages_h(int K, int cps, int n_meta, int idx_stage, int smem_limit)
 {
-    return cps == 2 ? stages_for<HH, 2>(K, smem_limit) : stages_for<HH, 1>(K, smem_limit);
+    return cps == 2 ? stages_for<HH, 2>(K, n_meta, idx_stage, smem_limit)
+                    : stages_for<HH, 1>(K, n_meta, idx_stage, smem_limit);
 }
 
 }  // namespace
 
-int target_tc_stages(int H, int K, int cps, int smem_limit)
+int target_tc_stages(int H, int K, int cps, int n_meta, int idx_stage, int smem_limit)
 {
     switch (H) {
-    case 16: return stages_h<16>(K, cps, smem_limit);
-    case 32: return stages_h<32>(K, cps, smem_limit);
-    case 64: return stages_h<64>(K, cps, smem_limit);
-    case 128: return stages_h<128>(K, cps, smem_limit);
+    case 16: return stages_h<16>(K, cps, n_meta, idx_stage, smem_limit);
+    case 32: return stages_h<32>(K, cps, n_meta, idx_stage, smem_limit);
+    case 64: return stages_h<64>(K, cps, n_meta, idx_stage, smem_limit);
+    case 128: return stages_h<128>(K, cps, n_meta, idx_stage, smem_limit);
     default: return 0;
     }
 }
