@@ -113,7 +113,6 @@ struct EpiState {                 // one per epilogue warpgroup
     float wprime[HH];
     float red_m[8];
     float klred[8][3];   // fused KL: per-warp partials of the row reductions
-    int flag;
 };
 
 template <int HH>
@@ -719,15 +718,11 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
             const int mb = it & 1;
             // window log-mass of this token's heads, fetched early
             const float wl_h = (et < HH && a.wl) ? a.wl[(size_t)g * HH + et] : 0.f;
-            // leader waits; the named barrier hands the outcome to everyone
-            if (ew == 0) {
-                const bool f = warp_mbar_wait(&sm->meta_full[m3], (it / NM) & 1, abort_flag, a.err);
-                if (lane == 0)
-                    st.flag = f ? 1 : 0;
-                __syncwarp();
-            }
-            named_bar_sync(bar_id, kEpiThreads);
-            if (!st.flag)
+            // the first warp waits; the barrier hands the outcome to everyone
+            bool fm = true;
+            if (ew == 0)
+                fm = warp_mbar_wait(&sm->meta_full[m3], (it / NM) & 1, abort_flag, a.err);
+            if (!named_bar_and(bar_id, kEpiThreads, fm))
                 break;
             const int nsel = sm->nsel[m3];
             const int nt = (nsel + 127) / 128;
@@ -768,20 +763,17 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
                     const int t1 = min(ntg, t0 + TBH);
                     const bool from_spill = spill && pass == 1;   // this group's scores are in scr
                     if (!from_spill) {
-                        named_bar_sync(bar_id, kEpiThreads);   // st.flag is free again
+                        bool fa = true;
                         if (ew == 0) {
                             const int jb = mb ? jobs1 : jobs0;
-                            const bool f = warp_mbar_wait(&sm->acc_full[mb], jb & 1, abort_flag, a.err);
-                            if (lane == 0)
-                                st.flag = f ? 1 : 0;
-                            __syncwarp();
+                            fa = warp_mbar_wait(&sm->acc_full[mb], jb & 1, abort_flag, a.err);
                         }
-                        named_bar_sync(bar_id, kEpiThreads);
+                        fa = named_bar_and(bar_id, kEpiThreads, fa);
                         if (mb)
                             ++jobs1;
                         else
                             ++jobs0;
-                        if (!st.flag) {
+                        if (!fa) {
                             ok = false;
                             break;
                         }
