@@ -92,6 +92,25 @@ def test_distill_target_ex_host_errors(sai):
     assert f(*args(FAKE, 1)[:6], 1, 64, 4, 32, 8, 3, 0.1, 1, FAKE, None, None) == 2   # S % cr, per-branch
 
 
+def test_distill_target_ws_host_errors_and_size(sai):
+    """The spill-workspace variant: a misaligned workspace is refused before
+    anything else; NULL workspace is allowed (the two-sweep path); the usual
+    argument checks apply. No spill is needed at K=512, H=64 (one TMEM group)
+    or below H=64; sizes the kernel does not take report 0."""
+    lib = sai.lib()
+    f = lib.sai_distill_target_ws
+    args = lambda ws, nb, S=64, K=8, cr=4: (FAKE, FAKE, FAKE, FAKE, None, None, 1, S, S, 0, 4, 32, K, cr, 0.1, 0,
+                                             FAKE, None, ws, nb, None)
+    assert f(*args(FAKE_MIS, 1 << 20)) == 7          # SAI_ERR_ALIGN: workspace
+    assert f(*args(None, 0, cr=3)) == 2              # S % cr, no workspace
+    assert f(*args(FAKE, 1 << 20, K=17)) == 2        # K > S/cr
+    sz = lib.sai_distill_target_workspace_bytes
+    assert sz(1, 4096, 64, 512, 512) == 0             # one group of four tiles
+    assert sz(1, 4096, 32, 512, 2048) == 0            # below H = 64: the two-sweep path only
+    assert sz(1, 4096, 64, 500, 2048) == 0            # D % 64 != 0: not the tensor-core kernel
+    assert sz(0, 4096, 64, 512, 2048) == 0
+
+
 def test_distill_target_kl_host_errors(sai):
     """The fused target + KL call refuses missing KL buffers and a short or
     misaligned workspace before launching anything."""
