@@ -35,9 +35,10 @@
 // The epilogue needs the per-head log-sum-exp over ALL selected slots before
 // it can form u, so a token's scores stay in TMEM until it is done: up to
 // 256/H tiles (512 slots at H=64) per accumulator. Tokens alternate between
-// two 256-column accumulators, so one token's epilogue overlaps the next
-// token's MMA; both epilogue warpgroups work on each token (half the heads
-// each at H >= 32). Tokens with more selected slots run in groups: a first
+// two 256-column accumulators, group by group (a token of one group per
+// accumulator, a longer token spread over both), so the epilogue of one group
+// overlaps the MMAs of the next; both epilogue warpgroups work on each group
+// (half the heads each at H >= 32). Tokens with more selected slots run in groups: a first
 // pass over the groups merges per-head (max, sum-exp) statistics, a second
 // forms u. With a spill buffer (H >= 64, its own instantiation) the first
 // pass also stores each group's raw scores there and the second reads them
@@ -573,8 +574,8 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
             bool ok = true, issued = false;
             int it = 0;
             int jobs0 = 0, jobs1 = 0;
+            int gseq = 0;                        // accumulator groups so far: they alternate buffers
             for (int gt = blockIdx.x; gt < a.n_tok && ok; gt += gridDim.x, ++it) {
-                const int mb = it & 1;
                 const int m3 = it % NM;
                 if (!mbar_wait(&sm->meta_full[m3], (it / NM) & 1, abort_flag, a.err)) {
                     ok = false;
@@ -584,11 +585,13 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
                 const int nt = (nsel + 127) / 128;
                 const int G = n_groups(nsel, TB);
                 const int passes = G > 1 && !kSpill ? 2 : 1;
-                const uint32_t dbase = tmem + mb * 256;
                 for (int pass = 0; pass < passes && ok; ++pass) {
                     for (int grp = 0; grp < G && ok; ++grp) {
                         const int i0 = grp * TB;
                         const int ntg = min(nt, i0 + TB) - i0;
+                        const int mb = gseq & 1;
+                        ++gseq;
+                        const uint32_t dbase = tmem + mb * 256;
                         const int jb = mb ? jobs1 : jobs0;
                         if (!mbar_wait(&sm->acc_empty[mb], (jb & 1) ^ 1u, abort_flag, a.err)) {
                             ok = false;
@@ -689,6 +692,7 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
         const float s2 = a.scale * kLog2e;    // scale > 0 (checked on the host)
         const float sink_h = (a.sink && et < HH) ? a.sink[et] : -INFINITY;
         int jobs0 = 0, jobs1 = 0;
+        int gseq = 0;                         // accumulator groups so far (as the MMA threads count)
         // fused KL: the global count N of rows with a valid slot, and this
         // CTA's running KL sum (thread et == 0, fixed token order)
         const bool kl = FUSE_KL;
@@ -715,7 +719,6 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
             const int gt = blockIdx.x + it * gridDim.x;
             const int g = a.n_tok - 1 - gt;
             const int m3 = it % NM;
-            const int mb = it & 1;
             // window log-mass of this token's heads, fetched early
             const float wl_h = (et < HH && a.wl) ? a.wl[(size_t)g * HH + et] : 0.f;
             // the first warp waits; the barrier hands the outcome to everyone
@@ -735,7 +738,7 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
             float *prow = a.p + (size_t)g * K;
             const int32_t *sl = slot + m3 * Kp;
             const bool ident = sm->ident[m3] != 0;    // slot jj of the compacted order is slot jj
-            const uint32_t tbase = tmem + mb * 256 + ((uint32_t)(q * 32) << 16);
+            const uint32_t tlane = tmem + ((uint32_t)(q * 32) << 16);
             // fused KL: this thread's scores and valid flags (slots et, et+256),
             // loaded now so the latency is hidden behind the token's MMAs
             constexpr int kKlReg = 2;
@@ -762,6 +765,12 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
                     const int t0 = hf * TBH;
                     const int t1 = min(ntg, t0 + TBH);
                     const bool from_spill = spill && pass == 1;   // this group's scores are in scr
+                    // groups alternate between the two accumulators (a spilled
+                    // group's second pass reads no accumulator)
+                    const int mb = gseq & 1;
+                    if (!from_spill)
+                        ++gseq;
+                    const uint32_t tbase = tlane + mb * 256;
                     if (!from_spill) {
                         bool fa = true;
                         if (ew == 0) {
