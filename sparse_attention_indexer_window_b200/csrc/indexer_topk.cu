@@ -16,7 +16,8 @@
 // (about half the row on average, since later blocks are in the future; only
 // the candidate range is read and walked), kept in shared memory as
 // order-preserving 32-bit keys, and selected with an 8-bit radix select
-// (four histogram passes) for the K-th largest key.
+// (up to four histogram passes; it stops early once the crossing bin holds
+// exactly the keys still needed) for the K-th largest key.
 // A block-wide scan then compacts the selected blocks in block order, which
 // gives the ascending slot order without a sort.
 #include <cuda_runtime.h>
@@ -75,10 +76,11 @@ __global__ void __launch_bounds__(kTkThreads)
                         uint8_t *__restrict__ valid)
 {
     extern __shared__ uint32_t keys[];   // [jhi - jlo] (at most P)
-    __shared__ int hist[256];
+    __shared__ int hist[2][256];         // one per radix pass, in turn
     __shared__ int warp_buf[kTkWarps];
     __shared__ uint32_t s_prefix;
     __shared__ int s_rem;
+    __shared__ int s_done;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g = blockIdx.x;
     const int t = g % S;
@@ -99,6 +101,7 @@ __global__ void __launch_bounds__(kTkThreads)
         keys[i] = k;
         cnt += k != 0u;
     }
+    hist[0][tid] = 0;                                // the first pass's bins (256 threads, 256 bins)
     int n_cand = 0;
     block_excl_scan(cnt, warp_buf, n_cand);   // also orders the key writes before the reads below
 
@@ -109,14 +112,16 @@ __global__ void __launch_bounds__(kTkThreads)
     if (n_cand > K) {
         uint32_t prefix = 0u, mask = 0u;
         rem = K;
-        for (int shift = 24; shift >= 0; shift -= 8) {
-            for (int i = tid; i < 256; i += kTkThreads)
-                hist[i] = 0;
-            __syncthreads();
+        int pass = 0;
+        for (int shift = 24; shift >= 0; shift -= 8, ++pass) {
+            int *h = hist[pass & 1];
+            // the next pass's bins, cleared now: nothing reads them until the
+            // barrier after this pass's scan
+            hist[(pass + 1) & 1][tid] = 0;
             for (int i = tid; i < L; i += kTkThreads) {
                 const uint32_t k = keys[i];
                 if (k != 0u && (k & mask) == prefix)
-                    atomicAdd(&hist[(k >> shift) & 255u], 1);
+                    atomicAdd(&h[(k >> shift) & 255u], 1);
             }
             __syncthreads();
             if (warp == 0) {
@@ -124,7 +129,7 @@ __global__ void __launch_bounds__(kTkThreads)
                 int c[8], sum = 0;
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
-                    c[e] = hist[255 - 8 * lane - e];
+                    c[e] = h[255 - 8 * lane - e];
                     sum += c[e];
                 }
                 int incl = sum;
@@ -144,12 +149,22 @@ __global__ void __launch_bounds__(kTkThreads)
                         acc += c[e++];
                     s_prefix = prefix | ((uint32_t)(255 - 8 * lane - e) << shift);
                     s_rem = rem - acc;
+                    // every key of the crossing bin is needed: the keys above the
+                    // bin's lowest value are exactly the selection
+                    s_done = (rem - acc == c[e]) ? 1 : 0;
                 }
             }
             __syncthreads();
             prefix = s_prefix;
             rem = s_rem;
             mask |= 255u << shift;
+            if (s_done && shift > 0 && prefix != 0u) {
+                // take every key with this prefix: k > prefix - 1 (the keys
+                // below the bin are smaller)
+                prefix -= 1u;
+                rem = 0;
+                break;
+            }
         }
         T = prefix;
     }
