@@ -44,30 +44,48 @@ __device__ __forceinline__ uint32_t order_key(float x)
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// Exclusive prefix sum of v over the block (thread order), and the total.
-__device__ __forceinline__ int block_excl_scan(int v, int *warp_buf, int &total)
+// Exclusive prefix sum of v over the block (thread order), and the total
+// (unsigned: callers pack two counts of at most 16 bits each into one word).
+__device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t *warp_buf, uint32_t &total)
 {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    int incl = v;
+    uint32_t incl = v;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
         if (lane >= o)
             incl += y;
     }
     if (lane == 31)
         warp_buf[warp] = incl;
     __syncthreads();
-    int before = 0, tot = 0;
+    uint32_t before = 0, tot = 0;
 #pragma unroll
     for (int w = 0; w < kTkWarps; ++w) {
-        const int x = warp_buf[w];
-        before += (w < warp) ? x : 0;
+        const uint32_t x = warp_buf[w];
+        before += (w < warp) ? x : 0u;
         tot += x;
     }
-    __syncthreads();   // warp_buf is free again for the next scan
     total = tot;
     return before + incl - v;
+}
+
+// Sum of v over the block, in every thread, with one barrier. The caller
+// must pass another barrier before warp_buf is written again.
+__device__ __forceinline__ int block_total(int v, uint32_t *warp_buf)
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1)
+        v += __shfl_xor_sync(0xffffffffu, v, o);
+    if (lane == 0)
+        warp_buf[warp] = (uint32_t)v;
+    __syncthreads();
+    int tot = 0;
+#pragma unroll
+    for (int w = 0; w < kTkWarps; ++w)
+        tot += (int)warp_buf[w];
+    return tot;
 }
 
 __global__ void __launch_bounds__(kTkThreads)
@@ -77,7 +95,7 @@ __global__ void __launch_bounds__(kTkThreads)
 {
     extern __shared__ uint32_t keys[];   // [jhi - jlo] (at most P)
     __shared__ int hist[2][256];         // one per radix pass, in turn
-    __shared__ int warp_buf[kTkWarps];
+    __shared__ uint32_t warp_buf[kTkWarps];
     __shared__ uint32_t s_prefix;
     __shared__ int s_rem;
     __shared__ int s_done;
@@ -102,8 +120,9 @@ __global__ void __launch_bounds__(kTkThreads)
         cnt += k != 0u;
     }
     hist[0][tid] = 0;                                // the first pass's bins (256 threads, 256 bins)
-    int n_cand = 0;
-    block_excl_scan(cnt, warp_buf, n_cand);   // also orders the key writes before the reads below
+    // one barrier: the candidate count, and the key writes ordered before the
+    // reads below (warp_buf is next written after the radix passes' barriers)
+    const int n_cand = block_total(cnt, warp_buf);
 
     // Threshold key T and the number `rem` of entries equal to T to take.
     // With no more candidates than K, every candidate is taken (T = 0).
@@ -169,6 +188,11 @@ __global__ void __launch_bounds__(kTkThreads)
         T = prefix;
     }
 
+    // warp_buf is written again below: with no radix pass since block_total's
+    // reads, a barrier first (n_cand is the same in every thread)
+    if (n_cand <= K)
+        __syncthreads();
+
     // Compaction in block order: thread n owns candidates [n*E, (n+1)*E).
     const int E = (L + kTkThreads - 1) / kTkThreads;
     const int i0 = min(L, tid * E), i1 = min(L, i0 + E);
@@ -178,11 +202,15 @@ __global__ void __launch_bounds__(kTkThreads)
         cgt += k > T;
         ceq += (k != 0u && k == T);
     }
-    int n_eq = 0;
-    const int eq_before = block_excl_scan(ceq, warp_buf, n_eq);
-    const int take_eq = max(0, min(ceq, rem - eq_before));
-    int n_out = 0;
-    int slot = block_excl_scan(cgt + take_eq, warp_buf, n_out);
+    // one scan of both counts, packed (each below 2^16: L <= P, and P keys
+    // fit the shared memory only below that)
+    uint32_t packed_total = 0;
+    const uint32_t packed_before =
+        block_excl_scan(((uint32_t)cgt << 16) | (uint32_t)ceq, warp_buf, packed_total);
+    const int eq_before = (int)(packed_before & 0xffffu);
+    // keys before this thread's: every key above T, and the first `rem` equal to T
+    int slot = (int)(packed_before >> 16) + min(eq_before, rem);
+    const int n_out = (int)(packed_total >> 16) + min((int)(packed_total & 0xffffu), rem);
     int32_t *irow = idx + (size_t)g * K;
     float *srow = sel ? sel + (size_t)g * K : nullptr;
     uint8_t *vrow = valid ? valid + (size_t)g * K : nullptr;
