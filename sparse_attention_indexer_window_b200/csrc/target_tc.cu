@@ -18,9 +18,10 @@
 // 64-element (128-byte, swizzled) chunks.
 //
 // Gather. A dedicated warp compacts each token's idx row (selected slots
-// first, masked slots last), up to two tokens ahead; the idx rows arrive by
-// its own cp.async copies, and the compaction turns pool rows into byte
-// offsets. A pipeline stage is 128 selected rows x CPS 128-byte chunks of D
+// first, masked slots last), up to three tokens ahead (one at large K, where
+// shared memory holds a ring of two); the idx rows arrive by its own cp.async
+// copies two tokens ahead, or at large K are read from global memory, and the
+// compaction turns pool rows into byte offsets. A pipeline stage is 128 selected rows x CPS 128-byte chunks of D
 // (CPS = 2 where D allows: 32 KB); the A ring holds NA stages (4 at the
 // V4-Flash shape) and 8 / NA gather warps fill each stage, each its share of
 // the rows, copied into the swizzled K-major operand layout with 16-byte
@@ -229,9 +230,10 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
     if (warp == kMetaWarp) {
         // ====================================================== idx compaction
         // idx rows are staged into shared memory with this warp's own
-        // 16-byte cp.async copies, two tokens ahead (three buffers). (A TMA
-        // bulk copy here queued behind the Q and pool TMA traffic of the same
-        // SM and arrived late.)
+        // 16-byte cp.async copies, two tokens ahead (three buffers), when the
+        // layout has room for them (else they are read from global memory in
+        // 16-byte loads). (A TMA bulk copy here queued behind the Q and pool
+        // TMA traffic of the same SM and arrived late.)
         const int n_vec = K / 4;                 // 16-byte pieces of an idx row (idx_bulk: K % 4 == 0)
         auto stage_idx = [&](int gts, int buf) {
             if (idx_stage && gts < a.n_tok) {
