@@ -322,8 +322,12 @@ size_t sai_distill_kl_workspace_bytes(int B, int S, int K);
  *              16-byte aligned; no initialisation needed; must not be shared
  *              by calls that overlap on the device.
  *
- * The loss is reduced in a fixed order (deterministic). Errors: SAI_ERR_NULL,
- * SAI_ERR_SHAPE, SAI_ERR_ALIGN, SAI_ERR_WORKSPACE, SAI_ERR_CUDA.
+ * The loss is reduced in a fixed order (deterministic). The work is one
+ * cooperative launch (all blocks resident; N is formed across them behind a
+ * bounded grid barrier) after a 16-byte cudaMemsetAsync of the workspace on
+ * the stream. Should that barrier ever time out, *loss is NaN and dscores is
+ * left unwritten. Errors: SAI_ERR_NULL, SAI_ERR_SHAPE, SAI_ERR_ALIGN,
+ * SAI_ERR_WORKSPACE, SAI_ERR_CUDA.
  */
 sai_status sai_distill_kl(const float *p, const float *scores, const uint8_t *valid,
                           int B, int S, int K, float coeff,
