@@ -50,6 +50,8 @@ def parse():
                     help="timed steps of the long-context side line (0: skip it)")
     ap.add_argument("--packed-steps", type=int, default=50,
                     help="timed steps of the packed-documents side line (0: skip it)")
+    ap.add_argument("--fused-steps", type=int, default=200,
+                    help="timed steps of the window-fused route on the main workload (0: skip it)")
     return ap.parse_args()
 
 
@@ -330,6 +332,41 @@ def side_line(name, steps, dev, stream, rank, err, flush_l2):
     torch.cuda.empty_cache()
     return line
 
+def fused_window_line(w, t, steps, stream, err, flush_l2, p, ds, loss, ws):
+    """The same step as two calls, distill_target_window -> distill_kl (the
+    window band inside the target kernel, Q read once), on the main
+    workload's inputs, timed like the main line."""
+    import torch
+    import sparse_attention_indexer_window_b200 as sai
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    for i in range(3 + steps):
+        flush_l2(i)
+        if i >= 3:
+            ev[i - 3][0].record(stream)
+        sai.distill_target_window(t["Q"], t["Kw"], t["pool"], t["idx"], w.W, w.cr, w.scale, sink=t["sink"],
+                                  doc_start=t["doc_start"], err=err, out=p)
+        if i >= 3:
+            ev[i - 3][1].record(stream)
+        sai.distill_kl(p, t["scores"], t["valid"], w.coeff, workspace=ws, loss=loss, dscores=ds)
+        if i >= 3:
+            ev[i - 3][2].record(stream)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    sel, win = algorithmic_counts(w)
+    ms = statistics.mean(e[0].elapsed_time(e[2]) for e in ev)
+    tgt = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
+    fl = 2.0 * w.H * w.D * (sel + win)
+    return {
+        "route": "sai_distill_target_window -> sai_distill_kl (two calls, Q read once)",
+        "steps": steps, "ms_per_step": ms, "tokens_per_s": w.B * w.S / (ms / 1e3),
+        "kernels_ms": {"distill_target_window": tgt,
+                       "distill_kl": statistics.mean(e[1].elapsed_time(e[2]) for e in ev)},
+        "distill_target_window_tflops": fl / (tgt / 1e3) / 1e12,
+        "algorithmic": f"2*H*D flops per selected slot and window key x ({sel} + {win}) = {fl:.4g} flops/launch",
+        "gpu_launches": 2 * steps,
+    }
+
+
 def main():
     args = parse()
     if args.impl == "reference":
@@ -485,6 +522,10 @@ def main():
     sel_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in sel_ev)
     del isc
 
+    # ------------------------------------- the window-fused route (side line)
+    fused = fused_window_line(w, t, args.fused_steps, stream, err, flush_l2, p, ds, loss, ws) \
+        if args.fused_steps > 0 else None
+
     # ------------------------------------------- side lines: long, packed
     # The same three calls on the long-context workload (S=16384, K=2048: up
     # to 2048 selected blocks per token) and the packed one (B=4, two
@@ -560,12 +601,15 @@ def main():
             },
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "steps": args.e2e_steps},
+            "fused_window": fused,
             "long": long_line,
             "packed": packed_line,
             "gpu_launches": 3 * nsteps * world,   # window, target, KL (one cooperative launch); every rank
             "clocks": clk,
             "loss": loss_all,
         }
+        if fused is not None:
+            fused["distill_target_window_frac"] = fused["distill_target_window_tflops"] / peak_tf
         for sl in (long_line, packed_line):
             if sl is not None:
                 sl["distill_target_frac"] = sl["distill_target_tflops"] / peak_tf

@@ -13,6 +13,7 @@
  * Around them: sai_distill_target_ex (the per-branch target, or the target
  * from the attention forward's own LSE), sai_distill_target_ws (the target
  * with a spill workspace, so long selections are gathered and multiplied
+ * once), sai_distill_target_window (window and target in one kernel, Q read
  * once), sai_distill_target_kl (target and
  * KL in one call), sai_distill_kl_noalloc (no workspace argument),
  * sai_indexer_topk, the block selection that produces idx, scores and valid
@@ -263,6 +264,45 @@ sai_status sai_distill_target_ws(const uint16_t *Q, const uint16_t *pool, const 
                                  int B, int S, int S_seq, int t_begin, int H, int D, int K, int cr, float scale,
                                  unsigned flags, float *p, int32_t *d_err, void *workspace, size_t ws_bytes,
                                  void *stream);
+
+/*
+ * sai_distill_target_window -- sai_window_lse and sai_distill_target in one
+ * kernel, so Q is read from device memory once.
+ *
+ * The pages' V4 CSA attention treats each token's keys as one list, the 128
+ * window entries followed by the pool's top-k entries (Primus page "Docker
+ * Build for DeepSeek-v4", gluon_v3 commit, "Optimization Notes" / Forward).
+ * Here the window band is one more 128-row operand tile of the target's
+ * tensor-core contraction: its rows are the Kw rows of positions t-127 .. t,
+ * its product with Q[b,t] gives the window logits, and each head's
+ * log-sum-exp over the rows in [lo, t] takes the place of the window_lse
+ * input. The result is what sai_window_lse followed by sai_distill_target
+ * computes (the joint target, Primus page "perf(deepseek-v4): fuse and
+ * enable the indexer distillation loss", second commit message):
+ *
+ *   window_lse[b,t,h] = log sum_{s=lo}^{t} exp(scale * <Q[b,t,h,:], Kw[b,s,:]>),
+ *   lo = max(d0, t - W + 1), d0 = clamp(doc_start[b,t], 0, t) or 0;
+ *   p[b,t,:] as sai_distill_target with that window_lse.
+ *
+ *   Q, pool, idx, sink, doc_start, scale, p, d_err: as sai_distill_target
+ *   Kw          [B,S,D] bf16, 16-byte aligned
+ *   W           window length, 1 <= W <= 128 (the band is one 128-row tile;
+ *               a longer window returns SAI_ERR_UNSUPPORTED)
+ *   window_lse  [B,S,H] fp32, 4-byte aligned: the window log-mass written
+ *               out, or NULL (not written)
+ *   workspace   as sai_distill_target_ws: the raw-score spill for tokens of
+ *               more than one TMEM group, or NULL (second sweep)
+ *
+ * Only the tensor-core target kernel does this (H in {16,32,64,128},
+ * D % 64 == 0): other shapes return SAI_ERR_UNSUPPORTED, with no fallback;
+ * the three-call route covers them. Errors otherwise as sai_distill_target_ws
+ * and sai_window_lse.
+ */
+sai_status sai_distill_target_window(const uint16_t *Q, const uint16_t *Kw, const uint16_t *pool,
+                                     const int32_t *idx, const float *sink, const int32_t *doc_start,
+                                     int B, int S, int H, int D, int K, int cr, int W, float scale,
+                                     float *p, float *window_lse, int32_t *d_err,
+                                     void *workspace, size_t ws_bytes, void *stream);
 
 /* Bytes of device workspace sai_distill_target_kl needs for these sizes. */
 size_t sai_distill_target_kl_workspace_bytes(int B, int S, int K);

@@ -73,6 +73,9 @@ _lib.sai_distill_target_workspace_bytes.restype = ctypes.c_size_t
 _lib.sai_distill_target_ws.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F,
                                        ctypes.c_uint, _P, _P, _P, ctypes.c_size_t, _P]
 _lib.sai_distill_target_ws.restype = _I
+_lib.sai_distill_target_window.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P,
+                                           _P, ctypes.c_size_t, _P]
+_lib.sai_distill_target_window.restype = _I
 _lib.sai_count_valid_rows.argtypes = [_P, _I, _I, _I, _P, _P]
 _lib.sai_count_valid_rows.restype = _I
 _lib.sai_distill_kl_ex.argtypes = [_P, _P, _P, _I, _I, _I, _F, _P, _P, _P, _P, ctypes.c_size_t, _P]
@@ -187,9 +190,11 @@ def window_lse_range(Q: torch.Tensor, Kw: torch.Tensor, W: int, scale: float, t_
     return out
 
 
-def _target_inputs(Q, pool, idx, wl, cr, sink, doc_start, err, per_branch, full_lse, S_seq=None):
+def _target_inputs(Q, pool, idx, wl, cr, sink, doc_start, err, per_branch, full_lse, S_seq=None,
+                   wl_from_kw=False):
     """Checked arguments shared by the target entry points:
-    (Q bits, pool bits, K, wl, sink, flags)."""
+    (Q bits, pool bits, K, wl, sink, flags). wl_from_kw: the window log-mass
+    is formed from Kw inside the kernel (wl is not an input)."""
     B, S, H, D = Q.shape
     S_seq = S if S_seq is None else S_seq
     K = idx.shape[-1] if idx is not None else S_seq // cr
@@ -202,7 +207,7 @@ def _target_inputs(Q, pool, idx, wl, cr, sink, doc_start, err, per_branch, full_
         raise ValueError("per_branch and full_lse exclude each other")
     if per_branch:
         wl, sink = None, None
-    elif wl is None:
+    elif wl is None and not wl_from_kw:
         raise ValueError("window_lse (the full LSE with full_lse=True) is required unless per_branch")
     if full_lse:
         sink = None   # already inside the given LSE
@@ -285,6 +290,32 @@ def distill_target_range(Q: torch.Tensor, pool: torch.Tensor, idx: Optional[torc
                _ptr(doc_start), B, S, int(S_seq), int(t_begin), H, D, K, int(cr), float(scale), flags,
                _ptr(out), _ptr(err), _ptr(ws), nb)
     _check(st, "sai_distill_target_ws")
+    return out
+
+
+def distill_target_window(Q: torch.Tensor, Kw: torch.Tensor, pool: torch.Tensor, idx: Optional[torch.Tensor],
+                          W: int, cr: int, scale: float, sink: Optional[torch.Tensor] = None,
+                          doc_start: Optional[torch.Tensor] = None, err: Optional[torch.Tensor] = None,
+                          out: Optional[torch.Tensor] = None, wl_out: Optional[torch.Tensor] = None,
+                          workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """p[B,S,K] through sai_distill_target_window: the window log-mass is
+    formed from Kw [B,S,D] inside the target kernel (W <= 128), so Q is read
+    once. wl_out [B,S,H] fp32, if given, receives the window log-mass."""
+    B, S, H, D = Q.shape
+    Kw = _bf16_bits(Kw, "Kw")
+    if tuple(Kw.shape) != (B, S, D):
+        raise ValueError("Kw must be [B,S,D]")
+    Q, pool, K, _, sink, _ = _target_inputs(Q, pool, idx, None, cr, sink, doc_start, err, False, False,
+                                            wl_from_kw=True)
+    if out is None:
+        out = torch.empty((B, S, K), dtype=torch.float32, device=Q.device)
+    _want(out, "out", torch.float32, (B, S, K))
+    _want(wl_out, "wl_out", torch.float32, (B, S, H))
+    ws, nb = _target_workspace(Q.device, B, S, H, D, K, workspace)
+    st = _call(_lib.sai_distill_target_window, Q.device, _ptr(Q), _ptr(Kw), _ptr(pool), _ptr(idx), _ptr(sink),
+               _ptr(doc_start), B, S, H, D, K, int(cr), int(W), float(scale), _ptr(out), _ptr(wl_out), _ptr(err),
+               _ptr(ws), nb)
+    _check(st, "sai_distill_target_window")
     return out
 
 

@@ -212,6 +212,15 @@ size_t spill_floats_per_cta(int H, int K)
     return groups > 1 ? (size_t)groups * tb * H * 128 : 0;
 }
 
+// The window band computed inside the target kernel
+// (sai_distill_target_window); NULL: window_lse is an input.
+struct WinFuse {
+    const uint16_t *Kw;   // [B, S + kw_lead, D]
+    int W;
+    int kw_lead;          // Kw rows before local token 0
+    float *wl_out;        // [B, S, H] the window log-mass written out, or NULL
+};
+
 // CTAs of the target kernel for n_tok tokens.
 int target_grid(int64_t n_tok)
 {
@@ -230,7 +239,8 @@ int target_grid(int64_t n_tok)
 sai_status target_impl(const uint16_t *Q, const uint16_t *pool, const int32_t *idx, const float *window_lse,
                        const float *sink, const int32_t *doc_start, int B, int S, int S_seq, int t_begin, int H,
                        int D, int K, int cr, float scale, unsigned flags, float *p, int32_t *d_err,
-                       cudaStream_t st, const KlFuse *kf, void *ws = nullptr, size_t ws_bytes = 0)
+                       cudaStream_t st, const KlFuse *kf, void *ws = nullptr, size_t ws_bytes = 0,
+                       const WinFuse *wf = nullptr)
 {
     if ((flags & ~(SAI_TARGET_PER_BRANCH | SAI_TARGET_FULL_LSE)) ||
         (flags & (SAI_TARGET_PER_BRANCH | SAI_TARGET_FULL_LSE)) == (SAI_TARGET_PER_BRANCH | SAI_TARGET_FULL_LSE))
@@ -242,8 +252,16 @@ sai_status target_impl(const uint16_t *Q, const uint16_t *pool, const int32_t *i
         window_lse = nullptr;   // not read in this mode
     if (lse_mode != sai::kLseJoint)
         sink = nullptr;         // per-branch: no sink; given LSE: the sink is inside it
+    if (wf) {
+        // the window from Kw: the joint target only, never with the KL fused
+        if (lse_mode != sai::kLseJoint || kf)
+            return SAI_ERR_UNSUPPORTED;
+        if (!wf->Kw)
+            return SAI_ERR_NULL;
+        window_lse = nullptr;
+    }
     // idx NULL: dense over all blocks; p may be NULL only when the KL is fused
-    if (!Q || !pool || (!window_lse && !per_branch) || (!p && !kf))
+    if (!Q || !pool || (!window_lse && !per_branch && !wf) || (!p && !kf))
         return SAI_ERR_NULL;
     if (B < 1 || S < 1 || H < 1 || D < 1 || K < 1 || cr < 1 || (D % 8) != 0 || S_seq < 1 || (S_seq % cr) != 0 ||
         !isfinite(scale) || scale <= 0.f)
@@ -255,6 +273,15 @@ sai_status target_impl(const uint16_t *Q, const uint16_t *pool, const int32_t *i
         return SAI_ERR_SHAPE;
     if ((int64_t)B * S * H * D > INT32_MAX || (int64_t)B * S * K > INT32_MAX)
         return SAI_ERR_SHAPE;
+    if (wf) {
+        if (wf->W < 1 || wf->kw_lead < 0 || wf->kw_lead > t_begin || wf->kw_lead < std::min(wf->W - 1, t_begin) ||
+            (int64_t)B * (S + wf->kw_lead) * D > INT32_MAX)
+            return SAI_ERR_SHAPE;
+        if (wf->W > 128)
+            return SAI_ERR_UNSUPPORTED;   // the window band is one 128-row tile
+        if (!al16(wf->Kw) || (wf->wl_out && !al4(wf->wl_out)))
+            return SAI_ERR_ALIGN;
+    }
     if (!al16(Q) || !al16(pool) || (idx && !al4(idx)) || (window_lse && !al4(window_lse)) || (p && !al4(p)) ||
         (sink && !al4(sink)) || (doc_start && !al4(doc_start)) || (d_err && !al4(d_err)))
         return SAI_ERR_ALIGN;
@@ -276,8 +303,10 @@ sai_status target_impl(const uint16_t *Q, const uint16_t *pool, const int32_t *i
             continue;
         n_meta = (c % 2 == 0) ? 4 : 2;
         idx_stage = (c % 2 == 0 && idx_vec) ? 1 : 0;
-        n_astages = sai::target_tc_stages(H, K, cps, n_meta, idx_stage, smem_cap);
+        n_astages = sai::target_tc_stages(H, K, cps, n_meta, idx_stage, wf ? 1 : 0, smem_cap);
     }
+    if (wf && n_astages == 0)
+        return SAI_ERR_UNSUPPORTED;   // the window band needs the tensor-core kernel
     // the epilogue computes the KL from two slots per thread (K <= 512)
     const bool fuse_here = kf && n_astages > 0 && K <= 512;
     if (kf && !fuse_here && !p)
@@ -320,10 +349,21 @@ sai_status target_impl(const uint16_t *Q, const uint16_t *pool, const int32_t *i
         a.kl_done = nullptr;
         a.spill = nullptr;
         a.spill_stride = 0;
-        CUtensorMap mq, mp;
+        a.win = wf ? wf->W : 0;
+        a.kw_lead = wf ? wf->kw_lead : 0;
+        a.kw_rows = S + a.kw_lead;
+        a.kw_box_rows = (int)std::min<int64_t>(128, (int64_t)B * a.kw_rows);
+        a.wl_out = wf ? wf->wl_out : nullptr;
+        CUtensorMap mq, mp, mk;
         if (!make_map_bf16(&mq, Q, (uint64_t)B * S * H, D, (uint32_t)H) ||
             !make_map_bf16(&mp, pool, (uint64_t)B * P, D, (uint32_t)a.pool_box_rows))
             return SAI_ERR_CUDA;
+        if (wf) {
+            if (!make_map_bf16(&mk, wf->Kw, (uint64_t)B * a.kw_rows, D, (uint32_t)a.kw_box_rows))
+                return SAI_ERR_CUDA;
+        } else {
+            mk = mp;   // not read
+        }
         const int grid = target_grid(a.n_tok);
         if (grid <= 0)
             return SAI_ERR_CUDA;
@@ -348,7 +388,7 @@ sai_status target_impl(const uint16_t *Q, const uint16_t *pool, const int32_t *i
             a.kl_count_blocks = kf->plan.count_blocks;
             a.kl_part = reinterpret_cast<double *>(w + 16 + (((size_t)kf->plan.count_blocks * 4 + 15) & ~size_t(15)));
         }
-        sai_status e = cuda_status(sai::launch_target_tc(mq, mp, a, grid, st));
+        sai_status e = cuda_status(sai::launch_target_tc(mq, mp, mk, a, grid, st));
         if (e != SAI_OK || fuse_here || !kf)
             return e;
     } else if ((int)sai::target_simt_smem_bytes(H, D, K) <= smem_cap) {
@@ -393,6 +433,18 @@ size_t sai_distill_target_workspace_bytes(int B, int S, int H, int D, int K)
         return 0;
     const int grid = target_grid((int64_t)B * S);
     return grid > 0 ? (size_t)grid * spf * sizeof(float) : 0;
+}
+
+sai_status sai_distill_target_window(const uint16_t *Q, const uint16_t *Kw, const uint16_t *pool,
+                                     const int32_t *idx, const float *sink, const int32_t *doc_start, int B, int S,
+                                     int H, int D, int K, int cr, int W, float scale, float *p, float *window_lse,
+                                     int32_t *d_err, void *workspace, size_t ws_bytes, void *stream)
+{
+    if (workspace && !al16(workspace))
+        return SAI_ERR_ALIGN;
+    const WinFuse wf = {Kw, W, 0, window_lse};
+    return target_impl(Q, pool, idx, nullptr, sink, doc_start, B, S, S, 0, H, D, K, cr, scale, 0u, p, d_err,
+                       reinterpret_cast<cudaStream_t>(stream), nullptr, workspace, ws_bytes, &wf);
 }
 
 sai_status sai_distill_target_ws(const uint16_t *Q, const uint16_t *pool, const int32_t *idx,

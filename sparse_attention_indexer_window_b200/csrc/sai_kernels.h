@@ -59,6 +59,14 @@ struct TgtTcArgs {
     // back. NULL: the groups are gathered and multiplied a second time.
     float *spill;
     int spill_stride;     // floats per CTA: groups x tiles per group x H x 128
+    // Window band in the same kernel (win > 0; sai_distill_target_window):
+    // the per-head log-sum-exp over each token's window keys is formed from
+    // Kw (the mapK tensor map, rows [B * kw_rows, D]) instead of read from wl.
+    int win;              // window length W (1..128); 0: wl is an input
+    int kw_rows;          // Kw rows per sequence (local tokens + kw_lead)
+    int kw_lead;          // Kw rows before local token 0 (token-range calls; else 0)
+    int kw_box_rows;      // rows of the Kw TMA box: min(128, B * kw_rows)
+    float *wl_out;        // [n_tok, H] the window log-mass written out, or NULL
     // KL fused into the epilogue (kl_scores NULL: not fused). N comes from the
     // per-block valid-row counts of kl_count_kernel, run before on the stream.
     const float *kl_scores;     // [n_tok, K]
@@ -73,10 +81,12 @@ struct TgtTcArgs {
 };
 // Deepest gathered-row stage ring of `cps`-chunk stages that fits
 // `smem_limit` bytes beside a compaction ring of n_meta tokens, with or
-// without the staged idx rows (0: none).
-int target_tc_stages(int H, int K, int cps, int n_meta, int idx_stage, int smem_limit);
-cudaError_t launch_target_tc(const CUtensorMap &mapQ, const CUtensorMap &mapP, const TgtTcArgs &a, int grid,
-                             cudaStream_t stream);
+// without the staged idx rows, with (win = 1) or without the window-fused
+// kernel's TMEM ring barriers (0: none).
+int target_tc_stages(int H, int K, int cps, int n_meta, int idx_stage, int win, int smem_limit);
+// mapK: the Kw tensor map when a.win > 0 (any valid map otherwise; unused)
+cudaError_t launch_target_tc(const CUtensorMap &mapQ, const CUtensorMap &mapP, const CUtensorMap &mapK,
+                             const TgtTcArgs &a, int grid, cudaStream_t stream);
 
 // ------------------------------------------- generic CUDA-core kernels
 // For shapes the tensor-core kernels do not take (small H or D).

@@ -132,9 +132,16 @@ struct TgtSmem {
     EpiState<HH> epi[1];
 };
 
-// Bytes of dynamic smem other than the A-stage ring.
-template <int HH, int CPS>
-__host__ __device__ inline size_t fixed_smem_bytes(int K);
+// The window-fused kernel's TMEM: a ring of 512 / H tile slots of H columns
+// each (at most 32). Tile n of the sequence of tiles the MMAs write lands in
+// slot n % (512 / H); the epilogue releases each slot when it is done with
+// it (the window tile right after its statistics, a group's tiles after its
+// u pass), and the MMA threads commit each group of tiles to one barrier of
+// a ring as deep as the slot count.
+struct TileRing {
+    uint64_t slot_empty[32];
+    uint64_t grp_full[32];
+};
 
 __device__ __forceinline__ int n_groups(int nsel, int TB)
 {
@@ -154,14 +161,20 @@ __device__ __forceinline__ bool selected(int j, int t, int d0, int P, int cr)
 // behind one barrier wait, one fence and one commit; on this part a commit
 // every 4 MMAs leaves the tensor pipe idle about half the time, so CPS = 2
 // whenever D allows it.
-template <int HH, bool FUSE_KL, int CPS, bool SPILL>
+// WIN: the window band is computed here too (sai_distill_target_window):
+// every token first runs one more tile, A = the 128 Kw rows ending at the
+// token (one TMA box per chunk), whose per-head log-sum-exp over the window
+// keys replaces the window_lse input; the TMEM is then a ring of tile slots
+// (TileRing) instead of two fixed accumulators.
+template <int HH, bool FUSE_KL, int CPS, bool SPILL, bool WIN>
 __global__ void __launch_bounds__(kTgtThreads, 1)
     target_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapP,
-                     const TgtTcArgs a)
+                     const __grid_constant__ CUtensorMap mapK, const TgtTcArgs a)
 {
     constexpr int TB = 256 / HH;                 // tiles per accumulator
     // the raw-score spill exists only in its own instantiation (H >= 64)
     constexpr bool kSpill = SPILL && TB <= 4;
+    constexpr int kSlots = 512 / HH;             // TMEM tile slots (WIN)
     constexpr uint32_t kQTile = HH * 128;        // one chunk of Q[t]: H rows x 128 bytes
     constexpr uint32_t kQEntry = CPS * kQTile;   // one Q ring entry
     constexpr uint32_t kAStage = CPS * kATile;   // one A ring stage: 128 rows x CPS chunks
@@ -184,6 +197,7 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
     float *ubuf = reinterpret_cast<float *>(idxs + (idx_stage ? 3 * Kp : 0)); // [Kp] u' of a token
     // then [2][TB*128] partial u of the two epilogue warpgroups (H >= 32)
     TgtSmem<HH> *sm = reinterpret_cast<TgtSmem<HH> *>(ubuf + Kp + (HH >= 32 ? 2 * TB * 128 : 0));
+    TileRing *ring = reinterpret_cast<TileRing *>(sm + 1);   // WIN only (no room reserved otherwise)
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -208,6 +222,12 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
         for (int b = 0; b < NM; ++b) {
             mbar_init(&sm->meta_full[b], 1);
             mbar_init(&sm->meta_empty[b], 1);
+        }
+        if constexpr (WIN) {
+            for (int k = 0; k < kSlots; ++k) {
+                mbar_init(&ring->slot_empty[k], 8);   // lane 0 of each epilogue warp
+                mbar_init(&ring->grp_full[k], 2);     // both MMA threads commit a group
+            }
         }
         mbar_init(&sm->drain[0], 1);
         mbar_init(&sm->drain[1], 1);
@@ -423,7 +443,8 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
                 break;
             const int nsel = sm->nsel[m3];
             const int G = n_groups(nsel, TB);
-            const int nq = (G > 1 && !kSpill ? 2 : 1) * G * n_cp;
+            // (WIN: the window tile's group first, one more set of chunks)
+            const int nq = (G > 1 && !kSpill ? 2 : 1) * G * n_cp + (WIN ? n_cp : 0);
             for (int qi = 0; qi < nq && ok; ++qi) {
                 const int c0 = (qi % n_cp) * CPS;
                 ok = warp_mbar_wait(&sm->q_empty[qs], qph ^ 1u, abort_flag, a.err);
@@ -470,8 +491,11 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
             const int r_in = lane >> 3;          // row within a 4-row group
             const uint32_t dst0 = smem_u32(a_buf + aslot * kAStage);
             const uint32_t row_bytes = (uint32_t)a.D * 2u;
-            if (lane == 0)
+            if (lane == 0) {
                 tma_prefetch_desc(&mapP);
+                if (WIN)
+                    tma_prefetch_desc(&mapK);
+            }
             uint32_t ph = 0;
             int s = 0;                           // stage index modulo NA
             bool ok = true;
@@ -487,10 +511,20 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
                 const int nt = (nsel + 127) / 128;
                 const int G = n_groups(nsel, TB);
                 const int passes = G > 1 && !kSpill ? 2 : 1;
-                for (int pass = 0; pass < passes && ok; ++pass) {
-                    for (int grp = 0; grp < G && ok; ++grp) {
+                // WIN: Kw row of the window tile's first row (the box's last
+                // row is the token's own key; negative rows read as zeros)
+                int wrow0 = 0;
+                if constexpr (WIN) {
+                    const int g = a.n_tok - 1 - gt;
+                    const int b = g / a.S;
+                    wrow0 = b * a.kw_rows + a.kw_lead + (g - b * a.S) - (a.kw_box_rows - 1);
+                }
+                for (int pass = WIN ? -1 : 0; pass < passes && ok; ++pass) {
+                    const bool wpass = WIN && pass < 0;   // the window tile
+                    const int GP = wpass ? 1 : G;
+                    for (int grp = 0; grp < GP && ok; ++grp) {
                         const int i0 = grp * TB;
-                        const int ntg = min(nt, i0 + TB) - i0;
+                        const int ntg = wpass ? 1 : min(nt, i0 + TB) - i0;
                         for (int cp = 0; cp < n_cp && ok; ++cp) {
                             for (int i = 0; i < ntg; ++i) {
                                 const bool mine = (s == aslot);
@@ -504,9 +538,23 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
                                 const int tile_row0 = (i0 + i) * 128;
                                 const int rows = min(128, nsel - tile_row0);
                                 const uint32_t *ro = rw + tile_row0;
-                                // a tile whose rows are consecutive pool rows (the compaction
-                                // warp marks it) is one TMA box per chunk
-                                if ((tcontig >> (i0 + i)) & 1u) {
+                                if (wpass) {
+                                    if (lane == 0) {
+                                        if (part == 0) {
+                                            mbar_arrive_expect_tx(&sm->a_full[aslot],
+                                                                  (uint32_t)(CPS * a.kw_box_rows) * 128u);
+#pragma unroll
+                                            for (int cc = 0; cc < CPS; ++cc)
+                                                tma_load_2d(a_buf + aslot * kAStage + cc * kATile, &mapK,
+                                                            &sm->a_full[aslot], (cp * CPS + cc) * 64, wrow0);
+                                        } else {
+                                            mbar_arrive(&sm->a_full[aslot]);
+                                        }
+                                    }
+                                    __syncwarp();
+                                } else if ((tcontig >> (i0 + i)) & 1u) {
+                                    // a tile whose rows are consecutive pool rows (the compaction
+                                    // warp marks it) is one TMA box per chunk
                                     const uint32_t ro0 = ro[0];
                                     if (lane == 0) {
                                         if (part == 0) {
@@ -577,6 +625,7 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
             int it = 0;
             int jobs0 = 0, jobs1 = 0;
             int gseq = 0;                        // accumulator groups so far: they alternate buffers
+            int tn = 0, gq = 0;                  // WIN: tiles and groups so far (the TMEM ring)
             for (int gt = blockIdx.x; gt < a.n_tok && ok; gt += gridDim.x, ++it) {
                 const int m3 = it % NM;
                 if (!mbar_wait(&sm->meta_full[m3], (it / NM) & 1, abort_flag, a.err)) {
@@ -587,22 +636,40 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
                 const int nt = (nsel + 127) / 128;
                 const int G = n_groups(nsel, TB);
                 const int passes = G > 1 && !kSpill ? 2 : 1;
-                for (int pass = 0; pass < passes && ok; ++pass) {
-                    for (int grp = 0; grp < G && ok; ++grp) {
+                for (int pass = WIN ? -1 : 0; pass < passes && ok; ++pass) {
+                    const bool wpass = WIN && pass < 0;   // the window tile
+                    const int GP = wpass ? 1 : G;
+                    for (int grp = 0; grp < GP && ok; ++grp) {
                         const int i0 = grp * TB;
-                        const int ntg = min(nt, i0 + TB) - i0;
+                        const int ntg = wpass ? 1 : min(nt, i0 + TB) - i0;
                         const int mb = gseq & 1;
                         ++gseq;
                         const uint32_t dbase = tmem + mb * 256;
-                        const int jb = mb ? jobs1 : jobs0;
-                        if (!mbar_wait(&sm->acc_empty[mb], (jb & 1) ^ 1u, abort_flag, a.err)) {
-                            ok = false;
-                            break;
+                        int n0 = 0;
+                        if constexpr (WIN) {
+                            // both threads wait for every slot of the group, so neither
+                            // commits a group before the epilogue has taken the group
+                            // that used its commit barrier kSlots groups earlier
+                            n0 = tn;
+                            tn += ntg;
+                            for (int i = 0; i < ntg && ok; ++i) {
+                                const int n = n0 + i;
+                                ok = mbar_wait(&ring->slot_empty[n & (kSlots - 1)], ((n / kSlots) & 1) ^ 1u,
+                                               abort_flag, a.err);
+                            }
+                            if (!ok)
+                                break;
+                        } else {
+                            const int jb = mb ? jobs1 : jobs0;
+                            if (!mbar_wait(&sm->acc_empty[mb], (jb & 1) ^ 1u, abort_flag, a.err)) {
+                                ok = false;
+                                break;
+                            }
+                            if (mb)
+                                ++jobs1;
+                            else
+                                ++jobs0;
                         }
-                        if (mb)
-                            ++jobs1;
-                        else
-                            ++jobs0;
                         for (int cp = 0; cp < n_cp && ok; ++cp) {
                             if (!mbar_wait(&sm->q_full[qs], qph, abort_flag, a.err)) {
                                 ok = false;
@@ -624,7 +691,8 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
                                 }
                                 tc_fence_after();
                                 const uint64_t da = sdesc_k_sw128(smem_u32(a_buf + as * kAStage));
-                                const uint32_t d_tmem = dbase + i * HH;
+                                const uint32_t d_tmem =
+                                    WIN ? tmem + (uint32_t)(((n0 + i) & (kSlots - 1)) * HH) : dbase + i * HH;
                                 // CPS chunks x 4 K-steps; chunks are kATile bytes apart in A and
                                 // kQTile in Q (descriptor start addresses are in 16-byte units)
 #pragma unroll
@@ -651,7 +719,12 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
                         }
                         if (!ok)
                             break;
-                        umma_commit(&sm->acc_full[mb]);
+                        if constexpr (WIN) {
+                            umma_commit(&ring->grp_full[gq & (kSlots - 1)]);
+                            ++gq;
+                        } else {
+                            umma_commit(&sm->acc_full[mb]);
+                        }
                     }
                 }
             }
@@ -695,6 +768,7 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
         const float sink_h = (a.sink && et < HH) ? a.sink[et] : -INFINITY;
         int jobs0 = 0, jobs1 = 0;
         int gseq = 0;                         // accumulator groups so far (as the MMA threads count)
+        int tn = 0, gq = 0;                   // WIN: tiles and groups so far (the TMEM ring)
         // fused KL: the global count N of rows with a valid slot, and this
         // CTA's running KL sum (thread et == 0, fixed token order)
         const bool kl = FUSE_KL;
@@ -721,8 +795,23 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
             const int gt = blockIdx.x + it * gridDim.x;
             const int g = a.n_tok - 1 - gt;
             const int m3 = it % NM;
-            // window log-mass of this token's heads, fetched early
-            const float wl_h = (et < HH && a.wl) ? a.wl[(size_t)g * HH + et] : 0.f;
+            // window log-mass of this token's heads, fetched early (WIN: taken
+            // from the window tile below)
+            float wl_h = (!WIN && et < HH && a.wl) ? a.wl[(size_t)g * HH + et] : 0.f;
+            // WIN: window tile row r holds the key kw_box_rows - 1 - r positions
+            // before the token; rows [wr_lo, kw_box_rows) are the window
+            // [max(d0, t - W + 1), t]
+            int wr_lo = 0;
+            if constexpr (WIN) {
+                const int b = g / a.S;
+                const int t = g - b * a.S + a.t_begin;
+                int d0 = 0;
+                if (a.doc_start) {
+                    d0 = a.doc_start[g];
+                    d0 = d0 < 0 ? 0 : (d0 > t ? t : d0);
+                }
+                wr_lo = a.kw_box_rows - 1 - (t - max(d0, t - a.win + 1));
+            }
             // the first warp waits; the barrier hands the outcome to everyone
             bool fm = true;
             if (ew == 0)
@@ -759,10 +848,12 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
             float m_part = 0.f;
             float At = 0.f;
             bool ok = true;
-            for (int pass = 0; pass < passes && ok; ++pass) {
-                for (int grp = 0; grp < G; ++grp) {
+            for (int pass = WIN ? -1 : 0; pass < passes && ok; ++pass) {
+                const bool wpass = WIN && pass < 0;   // the window tile
+                const int GP = wpass ? 1 : G;
+                for (int grp = 0; grp < GP; ++grp) {
                     const int i0 = grp * TB;
-                    const int ntg = min(nt, i0 + TB) - i0;
+                    const int ntg = wpass ? 1 : min(nt, i0 + TB) - i0;
                     // this warpgroup's tiles of the group: [t0, t1) (possibly empty)
                     const int t0 = hf * TBH;
                     const int t1 = min(ntg, t0 + TBH);
@@ -773,22 +864,95 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
                     if (!from_spill)
                         ++gseq;
                     const uint32_t tbase = tlane + mb * 256;
+                    int n0 = 0;
+                    if constexpr (WIN) {
+                        if (!from_spill) {
+                            n0 = tn;
+                            tn += ntg;
+                        }
+                    }
+                    // TMEM address of tile i of the group (this thread's lane quarter)
+                    auto tcol = [&](int i) -> uint32_t {
+                        if constexpr (WIN)
+                            return tlane + (uint32_t)(((n0 + i) & (kSlots - 1)) * HH);
+                        else
+                            return tbase + (uint32_t)(i * HH);
+                    };
                     if (!from_spill) {
                         bool fa = true;
                         if (ew == 0) {
-                            const int jb = mb ? jobs1 : jobs0;
-                            fa = warp_mbar_wait(&sm->acc_full[mb], jb & 1, abort_flag, a.err);
+                            if constexpr (WIN) {
+                                fa = warp_mbar_wait(&ring->grp_full[gq & (kSlots - 1)], (gq / kSlots) & 1,
+                                                    abort_flag, a.err);
+                            } else {
+                                const int jb = mb ? jobs1 : jobs0;
+                                fa = warp_mbar_wait(&sm->acc_full[mb], jb & 1, abort_flag, a.err);
+                            }
                         }
                         fa = named_bar_and(bar_id, kEpiThreads, fa);
-                        if (mb)
-                            ++jobs1;
-                        else
-                            ++jobs0;
+                        if constexpr (WIN) {
+                            ++gq;
+                        } else {
+                            if (mb)
+                                ++jobs1;
+                            else
+                                ++jobs0;
+                        }
                         if (!fa) {
                             ok = false;
                             break;
                         }
                         tc_fence_after();
+                    }
+                    if constexpr (WIN) {
+                    if (wpass) {
+                        // ---- the window tile: each head's log-sum-exp over the
+                        // window keys (rows [wr_lo, kw_box_rows)). Per 8-column
+                        // block the stabiliser of a column is the warp's maximum
+                        // (one redux), then the warp's column sums; the four lane
+                        // quarters' (max, sum) pairs are merged per head.
+                        const bool rv = r >= wr_lo && r < a.kw_box_rows;
+#pragma unroll 1
+                        for (int cb = 0; cb < HC / 8; ++cb) {
+                            const int col0 = c_lo + cb * 8;
+                            uint32_t v[8];
+                            tmem_ld8(tcol(0) + col0, v);
+                            tmem_ld_wait();
+                            float m8[8];
+                            float mine = -INFINITY;
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) {
+                                m8[e] = warp_max_f32(rv ? __uint_as_float(v[e]) : -INFINITY) * s2;
+                                mine = lane == e ? m8[e] : mine;
+                            }
+                            float s8[8];
+#pragma unroll
+                            for (int e = 0; e < 8; ++e)
+                                s8[e] = rv ? ex2_approx(fmaf(__uint_as_float(v[e]), s2, -m8[e])) : 0.f;
+                            const float red = warp_colreduce8(s8, OpAdd());
+                            if (lane < 8) {
+                                st.red_max[q][col0 + lane] = mine;
+                                st.red_sum[q][col0 + lane] = red;
+                            }
+                        }
+                        named_bar_sync(bar_id, kEpiThreads);
+                        if (et < HH) {
+                            float gm = st.red_max[0][et];
+#pragma unroll
+                            for (int w = 1; w < 4; ++w)
+                                gm = fmaxf(gm, st.red_max[w][et]);
+                            float gs = 0.f;
+#pragma unroll
+                            for (int w = 0; w < 4; ++w)
+                                gs += st.red_sum[w][et] * exp2f(st.red_max[w][et] - gm);
+                            // the token's own key is always in its window: gm is finite
+                            wl_h = (gm + log2f(gs)) * 0.69314718055994531f;
+                            if (a.wl_out)
+                                a.wl_out[(size_t)g * HH + et] = wl_h;
+                        }
+                        // red_max / red_sum are written again only after the next
+                        // group's wait, a barrier every thread passes first
+                    }
                     }
                     const bool single = (G == 1);
                     if constexpr (HH >= 32) {
@@ -809,7 +973,7 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
 #pragma unroll
                             for (int i = 0; i < TB; ++i)
                                 if (i < ntg)
-                                    tmem_ld8(tbase + i * HH + col0, v[i]);
+                                    tmem_ld8(tcol(i) + col0, v[i]);
                             tmem_ld_wait();
                             if (spill) {
                                 // raw scores, lane-contiguous per (tile, head)
@@ -865,7 +1029,7 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
 #pragma unroll
                                 for (int i = 0; i < TB; ++i)
                                     if (i < ntg)
-                                        tmem_st8(tbase + i * HH + col0, v[i]);
+                                        tmem_st8(tcol(i) + col0, v[i]);
                             }
                             const float red = warp_colreduce8(s8, OpAdd());
                             if (lane < 8) {
@@ -917,7 +1081,7 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
 #pragma unroll
                                     for (int i = 0; i < IB; ++i)
                                         if (ib + i < ntg)
-                                            tmem_ld16(tbase + (ib + i) * HH + col0, v[i]);
+                                            tmem_ld16(tcol(ib + i) + col0, v[i]);
                                     tmem_ld_wait();
 #pragma unroll
                                     for (int i = 0; i < IB; ++i) {
@@ -964,7 +1128,7 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
 #pragma unroll
                                     for (int i = 0; i < IB; ++i)
                                         if (ib + i < ntg)
-                                            tmem_ld16(tbase + (ib + i) * HH + col0, v[i]);
+                                            tmem_ld16(tcol(ib + i) + col0, v[i]);
                                     tmem_ld_wait();
 #pragma unroll
                                     for (int i = 0; i < IB; ++i) {
@@ -988,7 +1152,7 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
 #pragma unroll
                                         for (int i = 0; i < IB; ++i)
                                             if (ib + i < ntg)
-                                                tmem_st16(tbase + (ib + i) * HH + col0, v[i]);
+                                                tmem_st16(tcol(ib + i) + col0, v[i]);
                                     }
                                 }
                                 const float red = warp_colreduce16(s16, OpAdd());
@@ -1031,7 +1195,7 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
 #pragma unroll
                                 for (int i = 0; i < IBH; ++i)
                                     if (ib + i < t1)
-                                        tmem_ld16(tbase + (ib + i) * HH + cc * 16, v[i]);
+                                        tmem_ld16(tcol(ib + i) + cc * 16, v[i]);
                                 tmem_ld_wait();
 #pragma unroll
                                 for (int i = 0; i < IBH; ++i) {
@@ -1068,7 +1232,7 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
 #pragma unroll
                                 for (int i = 0; i < IBH; ++i)
                                     if (ib + i < t1)
-                                        tmem_ld16(tbase + (ib + i) * HH + cc * 16, v[i]);
+                                        tmem_ld16(tcol(ib + i) + cc * 16, v[i]);
                                 tmem_ld_wait();
 #pragma unroll
                                 for (int i = 0; i < IBH; ++i) {
@@ -1092,7 +1256,7 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
 #pragma unroll
                                     for (int i = 0; i < IBH; ++i)
                                         if (ib + i < t1)
-                                            tmem_st16(tbase + (ib + i) * HH + cc * 16, v[i]);
+                                            tmem_st16(tcol(ib + i) + cc * 16, v[i]);
                                 }
                             }
                             const float red = warp_colreduce16(s16, OpAdd());
@@ -1201,7 +1365,7 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
 #pragma unroll
                                     for (int i = 0; i < IB; ++i)
                                         if (ib + i < ntg)
-                                            tmem_ld16(tbase + (ib + i) * HH + col0, v[i]);
+                                            tmem_ld16(tcol(ib + i) + col0, v[i]);
                                     tmem_ld_wait();
                                 }
 #pragma unroll
@@ -1255,7 +1419,7 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
 #pragma unroll
                                 for (int i = 0; i < IBH; ++i)
                                     if (t0 + ib + i < t1)
-                                        tmem_ld16(tbase + (t0 + ib + i) * HH + cc * 16, v[i]);
+                                        tmem_ld16(tcol(t0 + ib + i) + cc * 16, v[i]);
                                 tmem_ld_wait();
 #pragma unroll
                                 for (int i = 0; i < IBH; ++i) {
@@ -1290,8 +1454,14 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
                     if (!from_spill) {
                         tc_fence_before();
                         __syncwarp();
-                        if (lane == 0)
-                            mbar_arrive(&sm->acc_empty[mb]);
+                        if (lane == 0) {
+                            if constexpr (WIN) {
+                                for (int i = 0; i < ntg; ++i)
+                                    mbar_arrive(&ring->slot_empty[(n0 + i) & (kSlots - 1)]);
+                            } else {
+                                mbar_arrive(&sm->acc_empty[mb]);
+                            }
+                        }
                         __syncwarp();
                     }
                 }
@@ -1437,21 +1607,22 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
 }
 
 template <int HH, int CPS>
-__host__ __device__ inline size_t fixed_smem_bytes(int K, int n_meta, int idx_stage)
+__host__ __device__ inline size_t fixed_smem_bytes(int K, int n_meta, int idx_stage, int win)
 {
     const size_t Kp = (size_t)((K + 3) & ~3);
     const size_t uh = HH >= 32 ? (size_t)2 * (256 / HH) * 128 * 4 : 0;   // partial u of the two warpgroups
     const size_t rows = 2 * (size_t)n_meta + (idx_stage ? 3 : 0) + 1;    // row offsets, slots, idx, u'
-    return 1024 + q_entries<HH, CPS>() * (size_t)(CPS * HH * 128) + Kp * 4 * rows + uh + sizeof(TgtSmem<HH>) + 64;
+    return 1024 + q_entries<HH, CPS>() * (size_t)(CPS * HH * 128) + Kp * 4 * rows + uh + sizeof(TgtSmem<HH>) +
+           (win ? sizeof(TileRing) : 0) + 64;
 }
 
 // Deepest A-stage ring that fits the per-block smem limit, as a divisor of
 // the eight gather warps (so every slot has the same number of producers),
 // with two slots at least for each of the two MMA threads; 0 if none fits.
 template <int HH, int CPS>
-int stages_for(int K, int n_meta, int idx_stage, int smem_limit)
+int stages_for(int K, int n_meta, int idx_stage, int win, int smem_limit)
 {
-    const long room = (long)smem_limit - (long)fixed_smem_bytes<HH, CPS>(K, n_meta, idx_stage);
+    const long room = (long)smem_limit - (long)fixed_smem_bytes<HH, CPS>(K, n_meta, idx_stage, win);
     long n = room / (long)(CPS * kATile);
     if (n > kMaxAStages)
         n = kMaxAStages;
@@ -1462,19 +1633,20 @@ int stages_for(int K, int n_meta, int idx_stage, int smem_limit)
 }
 
 template <int HH, int CPS>
-size_t smem_bytes_for(int K, int n_meta, int idx_stage, int stages)
+size_t smem_bytes_for(int K, int n_meta, int idx_stage, int win, int stages)
 {
-    return fixed_smem_bytes<HH, CPS>(K, n_meta, idx_stage) + (size_t)stages * CPS * kATile;
+    return fixed_smem_bytes<HH, CPS>(K, n_meta, idx_stage, win) + (size_t)stages * CPS * kATile;
 }
 
-template <int HH, bool FUSE_KL, int CPS, bool SPILL>
-cudaError_t launch_hkcs(const CUtensorMap &mapQ, const CUtensorMap &mapP, const TgtTcArgs &a, int grid,
-                       cudaStream_t stream)
+template <int HH, bool FUSE_KL, int CPS, bool SPILL, bool WIN>
+cudaError_t launch_hkcsw(const CUtensorMap &mapQ, const CUtensorMap &mapP, const CUtensorMap &mapK,
+                         const TgtTcArgs &a, int grid, cudaStream_t stream)
 {
+    auto kern = target_tc_kernel<HH, FUSE_KL, CPS, SPILL, WIN>;
     // The register split above is only safe if every thread was launched with
     // exactly kLaunchRegs registers; refuse to launch otherwise.
     cudaFuncAttributes fa;
-    cudaError_t e = cudaFuncGetAttributes(&fa, target_tc_kernel<HH, FUSE_KL, CPS, SPILL>);
+    cudaError_t e = cudaFuncGetAttributes(&fa, kern);
     if (e != cudaSuccess)
         return e;
     if (fa.numRegs != kLaunchRegs)
@@ -1482,73 +1654,90 @@ cudaError_t launch_hkcs(const CUtensorMap &mapQ, const CUtensorMap &mapP, const 
     if (a.n_astages < 1 || kGatherWarps % a.n_astages != 0 || (a.D / 64) % CPS != 0 ||
         (a.n_meta != 2 && a.n_meta != 4) || (a.idx_stage && !a.idx_bulk))
         return cudaErrorInvalidValue;
-    const size_t smem = smem_bytes_for<HH, CPS>(a.K, a.n_meta, a.idx_stage, a.n_astages);
-    e = cudaFuncSetAttribute(target_tc_kernel<HH, FUSE_KL, CPS, SPILL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem);
+    // the window tile: one box of at most 128 rows, a window that fits in it
+    if (WIN && (a.kw_box_rows < 1 || a.kw_box_rows > 128 || a.win < 1 || a.win > 128 || a.kw_rows < 1 ||
+                a.lse_mode != kLseJoint))
+        return cudaErrorInvalidValue;
+    const size_t smem = smem_bytes_for<HH, CPS>(a.K, a.n_meta, a.idx_stage, WIN ? 1 : 0, a.n_astages);
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess)
         return e;
-    target_tc_kernel<HH, FUSE_KL, CPS, SPILL><<<grid, kTgtThreads, smem, stream>>>(mapQ, mapP, a);
+    kern<<<grid, kTgtThreads, smem, stream>>>(mapQ, mapP, mapK, a);
     return cudaGetLastError();
+}
+
+// The window-fused instantiation only for the plain target (no fused KL).
+template <int HH, bool FUSE_KL, int CPS, bool SPILL>
+cudaError_t launch_hkcs(const CUtensorMap &mapQ, const CUtensorMap &mapP, const CUtensorMap &mapK,
+                        const TgtTcArgs &a, int grid, cudaStream_t stream)
+{
+    if constexpr (!FUSE_KL) {
+        if (a.win)
+            return launch_hkcsw<HH, FUSE_KL, CPS, SPILL, true>(mapQ, mapP, mapK, a, grid, stream);
+    }
+    if (a.win)
+        return cudaErrorInvalidValue;
+    return launch_hkcsw<HH, FUSE_KL, CPS, SPILL, false>(mapQ, mapP, mapK, a, grid, stream);
 }
 
 // The spill instantiation only where it can be used (H >= 64, no fused KL).
 template <int HH, bool FUSE_KL, int CPS>
-cudaError_t launch_hkc(const CUtensorMap &mapQ, const CUtensorMap &mapP, const TgtTcArgs &a, int grid,
-                       cudaStream_t stream)
+cudaError_t launch_hkc(const CUtensorMap &mapQ, const CUtensorMap &mapP, const CUtensorMap &mapK,
+                       const TgtTcArgs &a, int grid, cudaStream_t stream)
 {
     if constexpr (HH >= 64 && !FUSE_KL) {
         if (a.spill)
-            return launch_hkcs<HH, FUSE_KL, CPS, true>(mapQ, mapP, a, grid, stream);
+            return launch_hkcs<HH, FUSE_KL, CPS, true>(mapQ, mapP, mapK, a, grid, stream);
     }
     if (a.spill)
         return cudaErrorInvalidValue;
-    return launch_hkcs<HH, FUSE_KL, CPS, false>(mapQ, mapP, a, grid, stream);
+    return launch_hkcs<HH, FUSE_KL, CPS, false>(mapQ, mapP, mapK, a, grid, stream);
 }
 
 template <int HH, bool FUSE_KL>
-cudaError_t launch_hk(const CUtensorMap &mapQ, const CUtensorMap &mapP, const TgtTcArgs &a, int grid,
-                      cudaStream_t stream)
+cudaError_t launch_hk(const CUtensorMap &mapQ, const CUtensorMap &mapP, const CUtensorMap &mapK,
+                      const TgtTcArgs &a, int grid, cudaStream_t stream)
 {
-    return a.cps == 2 ? launch_hkc<HH, FUSE_KL, 2>(mapQ, mapP, a, grid, stream)
-                      : launch_hkc<HH, FUSE_KL, 1>(mapQ, mapP, a, grid, stream);
+    return a.cps == 2 ? launch_hkc<HH, FUSE_KL, 2>(mapQ, mapP, mapK, a, grid, stream)
+                      : launch_hkc<HH, FUSE_KL, 1>(mapQ, mapP, mapK, a, grid, stream);
 }
 
 template <int HH>
-cudaError_t launch_h(const CUtensorMap &mapQ, const CUtensorMap &mapP, const TgtTcArgs &a, int grid,
-                     cudaStream_t stream)
+cudaError_t launch_h(const CUtensorMap &mapQ, const CUtensorMap &mapP, const CUtensorMap &mapK,
+                     const TgtTcArgs &a, int grid, cudaStream_t stream)
 {
-    return a.kl_scores ? launch_hk<HH, true>(mapQ, mapP, a, grid, stream)
-                       : launch_hk<HH, false>(mapQ, mapP, a, grid, stream);
+    return a.kl_scores ? launch_hk<HH, true>(mapQ, mapP, mapK, a, grid, stream)
+                       : launch_hk<HH, false>(mapQ, mapP, mapK, a, grid, stream);
 }
 
 template <int HH>
-int stages_h(int K, int cps, int n_meta, int idx_stage, int smem_limit)
+int stages_h(int K, int cps, int n_meta, int idx_stage, int win, int smem_limit)
 {
-    return cps == 2 ? stages_for<HH, 2>(K, n_meta, idx_stage, smem_limit)
-                    : stages_for<HH, 1>(K, n_meta, idx_stage, smem_limit);
+    return cps == 2 ? stages_for<HH, 2>(K, n_meta, idx_stage, win, smem_limit)
+                    : stages_for<HH, 1>(K, n_meta, idx_stage, win, smem_limit);
 }
 
 }  // namespace
 
-int target_tc_stages(int H, int K, int cps, int n_meta, int idx_stage, int smem_limit)
+int target_tc_stages(int H, int K, int cps, int n_meta, int idx_stage, int win, int smem_limit)
 {
     switch (H) {
-    case 16: return stages_h<16>(K, cps, n_meta, idx_stage, smem_limit);
-    case 32: return stages_h<32>(K, cps, n_meta, idx_stage, smem_limit);
-    case 64: return stages_h<64>(K, cps, n_meta, idx_stage, smem_limit);
-    case 128: return stages_h<128>(K, cps, n_meta, idx_stage, smem_limit);
+    case 16: return stages_h<16>(K, cps, n_meta, idx_stage, win, smem_limit);
+    case 32: return stages_h<32>(K, cps, n_meta, idx_stage, win, smem_limit);
+    case 64: return stages_h<64>(K, cps, n_meta, idx_stage, win, smem_limit);
+    case 128: return stages_h<128>(K, cps, n_meta, idx_stage, win, smem_limit);
     default: return 0;
     }
 }
 
-cudaError_t launch_target_tc(const CUtensorMap &mapQ, const CUtensorMap &mapP, const TgtTcArgs &a, int grid,
-                             cudaStream_t stream)
+cudaError_t launch_target_tc(const CUtensorMap &mapQ, const CUtensorMap &mapP, const CUtensorMap &mapK,
+                             const TgtTcArgs &a, int grid, cudaStream_t stream)
 {
     switch (a.H) {
-    case 16: return launch_h<16>(mapQ, mapP, a, grid, stream);
-    case 32: return launch_h<32>(mapQ, mapP, a, grid, stream);
-    case 64: return launch_h<64>(mapQ, mapP, a, grid, stream);
-    case 128: return launch_h<128>(mapQ, mapP, a, grid, stream);
+    case 16: return launch_h<16>(mapQ, mapP, mapK, a, grid, stream);
+    case 32: return launch_h<32>(mapQ, mapP, mapK, a, grid, stream);
+    case 64: return launch_h<64>(mapQ, mapP, mapK, a, grid, stream);
+    case 128: return launch_h<128>(mapQ, mapP, mapK, a, grid, stream);
     default: return cudaErrorInvalidValue;
     }
 }

@@ -111,6 +111,24 @@ def test_distill_target_ws_host_errors_and_size(sai):
     assert sz(0, 4096, 64, 512, 2048) == 0
 
 
+def test_distill_target_window_host_errors(sai):
+    """The window-fused target: a misaligned workspace is refused first; Kw
+    is required; 1 <= W <= 128 (a longer window is unsupported, not a shape
+    error); the target's own shape checks; Kw and the window_lse output
+    aligned. Only paths that return before any launch."""
+    f = sai.lib().sai_distill_target_window
+    args = lambda Kw=FAKE, W=16, ws=None, K=8, cr=4, wlo=FAKE: (FAKE, Kw, FAKE, FAKE, None, None, 1, 64, 4, 32, K,
+                                                                 cr, W, 0.1, FAKE, wlo, None, ws, 0, None)
+    assert f(*args(ws=FAKE_MIS)) == 7                # SAI_ERR_ALIGN: workspace
+    assert f(*args(Kw=None)) == 1                    # SAI_ERR_NULL: Kw
+    assert f(*args(W=0)) == 2
+    assert f(*args(W=129)) == 3                      # the window band is one 128-row tile
+    assert f(*args(cr=3)) == 2                       # S % cr
+    assert f(*args(K=17)) == 2                       # K > S/cr
+    assert f(*args(Kw=FAKE_MIS)) == 7
+    assert f(*args(wlo=FAKE + 2)) == 7               # window_lse out not 4-byte aligned
+
+
 def test_distill_target_kl_host_errors(sai):
     """The fused target + KL call refuses missing KL buffers and a short or
     misaligned workspace before launching anything."""

@@ -92,6 +92,11 @@ def test_h64_d128(sai):
     check_full(sai, workload("h64_d128", name="flash", S=512, K=100, D=128))
 
 
+def test_h64_d64(sai):
+    # D = 64: stages of one 64-column chunk (the one-chunk shared-memory layout)
+    check_full(sai, workload("h64_d64", name="flash", S=512, K=100, D=64))
+
+
 def test_flash_recipe_odd_k(sai):
     """K not a multiple of 4: idx rows are read directly, not staged."""
     check_full(sai, synth.make("flash", S=512, K=101, seed=4242))
