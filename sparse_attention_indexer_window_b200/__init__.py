@@ -7,6 +7,7 @@ fallback here: if ``libsai.so`` is missing the import fails.
     window_lse(Q, Kw, W, scale, doc_start=None)                -> [B,S,H] fp32
     distill_target(Q, pool, idx, wl, cr, scale, sink=None, doc_start=None, err=None) -> [B,S,K] fp32
     distill_kl(p, scores, valid, coeff, want_grad=True, workspace=None, n_rows=None) -> (loss[1], dscores)
+    distill_target_window(Q, Kw, pool, idx, W, cr, scale, ...) -> [B,S,K] fp32 (window band inside, Q read once)
 
 The token-range calls (window_lse_range, distill_target_range,
 count_valid_rows) serve a batch split across GPUs by sequence position; see
@@ -428,11 +429,19 @@ def distill_kl_noalloc(p: torch.Tensor, scores: torch.Tensor, valid: torch.Tenso
 
 
 def distill_loss(Q, Kw, pool, idx, scores, valid, *, W: int, cr: int, scale: float, coeff: float,
-                 sink=None, doc_start=None, err=None, workspace=None):
-    """The whole path, three calls on the current stream:
-    window_lse -> distill_target -> distill_kl. Returns (loss, dscores, p, wl)."""
-    wl = window_lse(Q, Kw, W, scale, doc_start)
-    p = distill_target(Q, pool, idx, wl, cr, scale, sink=sink, doc_start=doc_start, err=err)
+                 sink=None, doc_start=None, err=None, workspace=None, fused_window: bool = False):
+    """The whole path on the current stream: window_lse -> distill_target ->
+    distill_kl, or with fused_window=True distill_target_window ->
+    distill_kl (the window band inside the target kernel, Q read once; the
+    window log-mass is still returned). Returns (loss, dscores, p, wl)."""
+    if fused_window:
+        B, S, H, _ = Q.shape
+        wl = torch.empty((B, S, H), dtype=torch.float32, device=Q.device)
+        p = distill_target_window(Q, Kw, pool, idx, W, cr, scale, sink=sink, doc_start=doc_start, err=err,
+                                  wl_out=wl)
+    else:
+        wl = window_lse(Q, Kw, W, scale, doc_start)
+        p = distill_target(Q, pool, idx, wl, cr, scale, sink=sink, doc_start=doc_start, err=err)
     loss, ds = distill_kl(p, scores, valid, coeff, workspace=workspace)
     return loss, ds, p, wl
 

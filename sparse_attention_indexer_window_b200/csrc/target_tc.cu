@@ -141,6 +141,8 @@ struct TgtSmem {
 struct TileRing {
     uint64_t slot_empty[32];
     uint64_t grp_full[32];
+    float wred_max[4][128];   // the window tile's per-quarter (max, sum) per head
+    float wred_sum[4][128];
 };
 
 __device__ __forceinline__ int n_groups(int nsel, int TB)
@@ -639,6 +641,9 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
                 for (int pass = WIN ? -1 : 0; pass < passes && ok; ++pass) {
                     const bool wpass = WIN && pass < 0;   // the window tile
                     const int GP = wpass ? 1 : G;
+                    // the window tile's owner alternates token by token, so both
+                    // threads issue window MMAs
+                    const int wown = wpass ? (it & 1) : 0;
                     for (int grp = 0; grp < GP && ok; ++grp) {
                         const int i0 = grp * TB;
                         const int ntg = wpass ? 1 : min(nt, i0 + TB) - i0;
@@ -681,7 +686,7 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
                                     ok = false;
                                     break;
                                 }
-                                if ((i & 1) != mt) {
+                                if (((i + wown) & 1) != mt) {
                                     mbar_arrive(&sm->a_empty[as]);
                                     if (++as == NA) {
                                         as = 0;
@@ -796,22 +801,8 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
             const int g = a.n_tok - 1 - gt;
             const int m3 = it % NM;
             // window log-mass of this token's heads, fetched early (WIN: taken
-            // from the window tile below)
+            // from the window tile)
             float wl_h = (!WIN && et < HH && a.wl) ? a.wl[(size_t)g * HH + et] : 0.f;
-            // WIN: window tile row r holds the key kw_box_rows - 1 - r positions
-            // before the token; rows [wr_lo, kw_box_rows) are the window
-            // [max(d0, t - W + 1), t]
-            int wr_lo = 0;
-            if constexpr (WIN) {
-                const int b = g / a.S;
-                const int t = g - b * a.S + a.t_begin;
-                int d0 = 0;
-                if (a.doc_start) {
-                    d0 = a.doc_start[g];
-                    d0 = d0 < 0 ? 0 : (d0 > t ? t : d0);
-                }
-                wr_lo = a.kw_box_rows - 1 - (t - max(d0, t - a.win + 1));
-            }
             // the first warp waits; the barrier hands the outcome to everyone
             bool fm = true;
             if (ew == 0)
@@ -845,15 +836,97 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
                     kl_v[i] = in ? a.kl_valid[gi] : 0;
                 }
             }
+            // WIN: the token's window tile, its first TMEM group: wait for it,
+            // take each head's log-sum-exp over the window keys into wl_h and
+            // release its slot at once. Tile row r holds the key kw_box_rows - 1 - r positions
+            // before the token; rows [wr_lo, kw_box_rows) are the window
+            // [max(d0, t - W + 1), t]. Per 8-column block the stabiliser of a
+            // column is the warp's maximum (one redux), then the warp's column
+            // sums; the four lane quarters' (max, sum) pairs are merged per
+            // head. False: a wait gave up.
+            auto window_tile = [&](int gw, float *wl_dst) -> bool {
+                if constexpr (WIN) {
+                const int bw = gw / a.S;
+                const int tw_pos = gw - bw * a.S + a.t_begin;
+                int d0 = 0;
+                if (a.doc_start) {
+                    d0 = a.doc_start[gw];
+                    d0 = d0 < 0 ? 0 : (d0 > tw_pos ? tw_pos : d0);
+                }
+                const int wr_lo = a.kw_box_rows - 1 - (tw_pos - max(d0, tw_pos - a.win + 1));
+                const int nw = tn++;
+                bool fw = true;
+                if (ew == 0)
+                    fw = warp_mbar_wait(&ring->grp_full[gq & (kSlots - 1)], (gq / kSlots) & 1, abort_flag, a.err);
+                fw = named_bar_and(bar_id, kEpiThreads, fw);
+                ++gq;
+                if (!fw)
+                    return false;
+                tc_fence_after();
+                const uint32_t tw = tlane + (uint32_t)((nw & (kSlots - 1)) * HH);
+                const bool rv = r >= wr_lo && r < a.kw_box_rows;
+#pragma unroll 1
+                for (int cb = 0; cb < HC / 8; ++cb) {
+                    const int col0 = c_lo + cb * 8;
+                    uint32_t v[8];
+                    tmem_ld8(tw + col0, v);
+                    tmem_ld_wait();
+                    float m8[8];
+                    float mine = -INFINITY;
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        m8[e] = warp_max_f32(rv ? __uint_as_float(v[e]) : -INFINITY) * s2;
+                        mine = lane == e ? m8[e] : mine;
+                    }
+                    float s8[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        s8[e] = rv ? ex2_approx(fmaf(__uint_as_float(v[e]), s2, -m8[e])) : 0.f;
+                    const float red = warp_colreduce8(s8, OpAdd());
+                    if (lane < 8) {
+                        ring->wred_max[q][col0 + lane] = mine;
+                        ring->wred_sum[q][col0 + lane] = red;
+                    }
+                }
+                tc_fence_before();
+                named_bar_sync(bar_id, kEpiThreads);
+                if (lane == 0)
+                    mbar_arrive(&ring->slot_empty[nw & (kSlots - 1)]);
+                __syncwarp();
+                if (et < HH) {
+                    float gm = ring->wred_max[0][et];
+#pragma unroll
+                    for (int w = 1; w < 4; ++w)
+                        gm = fmaxf(gm, ring->wred_max[w][et]);
+                    float gs = 0.f;
+#pragma unroll
+                    for (int w = 0; w < 4; ++w)
+                        gs += ring->wred_sum[w][et] * exp2f(ring->wred_max[w][et] - gm);
+                    // the token's own key is always in its window: gm is finite
+                    const float wl = (gm + log2f(gs)) * 0.69314718055994531f;
+                    *wl_dst = wl;
+                    if (a.wl_out)
+                        a.wl_out[(size_t)gw * HH + et] = wl;
+                }
+                // wred_* are written again only after the next window tile's
+                // wait, a barrier every thread passes first
+                }
+                return true;
+            };
             float m_part = 0.f;
             float At = 0.f;
             bool ok = true;
             for (int pass = WIN ? -1 : 0; pass < passes && ok; ++pass) {
-                const bool wpass = WIN && pass < 0;   // the window tile
-                const int GP = wpass ? 1 : G;
-                for (int grp = 0; grp < GP; ++grp) {
+                if constexpr (WIN) {
+                    if (pass < 0) {
+                        if (!window_tile(g, &wl_h))
+                            ok = false;
+                        continue;
+                    }
+                }
+                for (int grp = 0; grp < G; ++grp) {
                     const int i0 = grp * TB;
-                    const int ntg = wpass ? 1 : min(nt, i0 + TB) - i0;
+                    const int ntg = min(nt, i0 + TB) - i0;
                     // this warpgroup's tiles of the group: [t0, t1) (possibly empty)
                     const int t0 = hf * TBH;
                     const int t1 = min(ntg, t0 + TBH);
@@ -903,56 +976,6 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
                             break;
                         }
                         tc_fence_after();
-                    }
-                    if constexpr (WIN) {
-                    if (wpass) {
-                        // ---- the window tile: each head's log-sum-exp over the
-                        // window keys (rows [wr_lo, kw_box_rows)). Per 8-column
-                        // block the stabiliser of a column is the warp's maximum
-                        // (one redux), then the warp's column sums; the four lane
-                        // quarters' (max, sum) pairs are merged per head.
-                        const bool rv = r >= wr_lo && r < a.kw_box_rows;
-#pragma unroll 1
-                        for (int cb = 0; cb < HC / 8; ++cb) {
-                            const int col0 = c_lo + cb * 8;
-                            uint32_t v[8];
-                            tmem_ld8(tcol(0) + col0, v);
-                            tmem_ld_wait();
-                            float m8[8];
-                            float mine = -INFINITY;
-#pragma unroll
-                            for (int e = 0; e < 8; ++e) {
-                                m8[e] = warp_max_f32(rv ? __uint_as_float(v[e]) : -INFINITY) * s2;
-                                mine = lane == e ? m8[e] : mine;
-                            }
-                            float s8[8];
-#pragma unroll
-                            for (int e = 0; e < 8; ++e)
-                                s8[e] = rv ? ex2_approx(fmaf(__uint_as_float(v[e]), s2, -m8[e])) : 0.f;
-                            const float red = warp_colreduce8(s8, OpAdd());
-                            if (lane < 8) {
-                                st.red_max[q][col0 + lane] = mine;
-                                st.red_sum[q][col0 + lane] = red;
-                            }
-                        }
-                        named_bar_sync(bar_id, kEpiThreads);
-                        if (et < HH) {
-                            float gm = st.red_max[0][et];
-#pragma unroll
-                            for (int w = 1; w < 4; ++w)
-                                gm = fmaxf(gm, st.red_max[w][et]);
-                            float gs = 0.f;
-#pragma unroll
-                            for (int w = 0; w < 4; ++w)
-                                gs += st.red_sum[w][et] * exp2f(st.red_max[w][et] - gm);
-                            // the token's own key is always in its window: gm is finite
-                            wl_h = (gm + log2f(gs)) * 0.69314718055994531f;
-                            if (a.wl_out)
-                                a.wl_out[(size_t)g * HH + et] = wl_h;
-                        }
-                        // red_max / red_sum are written again only after the next
-                        // group's wait, a barrier every thread passes first
-                    }
                     }
                     const bool single = (G == 1);
                     if constexpr (HH >= 32) {
