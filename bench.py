@@ -362,6 +362,10 @@ def fused_window_line(w, t, steps, stream, err, flush_l2, p, ds, loss, ws):
         "kernels_ms": {"distill_target_window": tgt,
                        "distill_kl": statistics.mean(e[1].elapsed_time(e[2]) for e in ev)},
         "distill_target_window_tflops": fl / (tgt / 1e3) / 1e12,
+        # DRAM bytes of one launch (ncu), against the algorithmic Q + Kw + idx
+        # + pool + p: Q is read once for both the window band and the scores
+        "traffic": traffic_record("target_tc.cu#window"),
+        "algorithmic_bytes": w.B * w.S * (w.H * w.D * 2 + w.D * 2 + w.K * 4 + w.K * 4) + w.B * (w.S // w.cr) * w.D * 2,
         "algorithmic": f"2*H*D flops per selected slot and window key x ({sel} + {win}) = {fl:.4g} flops/launch",
         "gpu_launches": 2 * steps,
     }
