@@ -304,6 +304,29 @@ sai_status sai_distill_target_window(const uint16_t *Q, const uint16_t *Kw, cons
                                      float *p, float *window_lse, int32_t *d_err,
                                      void *workspace, size_t ws_bytes, void *stream);
 
+/*
+ * sai_distill_target_window_range -- sai_distill_target_window over a token
+ * range of longer sequences (a sequence split across GPUs by position, as
+ * sai_window_lse_range and sai_distill_target_range).
+ *
+ *   Q, idx, doc_start, p, window_lse: the range's own rows [B,S,...]
+ *   Kw          [B,S+kw_lead,D] bf16: the keys of positions
+ *               t_begin-kw_lead .. t_begin+S-1 (the range and its halo)
+ *   pool        [B,S_seq/cr,D]: every compressed entry of the sequence
+ *   t_begin     >= 0, t_begin + S <= S_seq; kw_lead in
+ *               [min(W-1, t_begin), t_begin]
+ *
+ * Positions, not row numbers, decide the window, causal and document rules.
+ * sai_distill_target_window is this call with S_seq = S and t_begin =
+ * kw_lead = 0. Errors as for sai_distill_target_window (SAI_ERR_SHAPE for a
+ * short halo or a range outside the sequence).
+ */
+sai_status sai_distill_target_window_range(const uint16_t *Q, const uint16_t *Kw, const uint16_t *pool,
+                                           const int32_t *idx, const float *sink, const int32_t *doc_start,
+                                           int B, int S, int S_seq, int t_begin, int kw_lead, int H, int D,
+                                           int K, int cr, int W, float scale, float *p, float *window_lse,
+                                           int32_t *d_err, void *workspace, size_t ws_bytes, void *stream);
+
 /* Bytes of device workspace sai_distill_target_kl needs for these sizes. */
 size_t sai_distill_target_kl_workspace_bytes(int B, int S, int K);
 

@@ -77,6 +77,9 @@ _lib.sai_distill_target_ws.restype = _I
 _lib.sai_distill_target_window.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P,
                                            _P, ctypes.c_size_t, _P]
 _lib.sai_distill_target_window.restype = _I
+_lib.sai_distill_target_window_range.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _I, _I,
+                                                 _F, _P, _P, _P, _P, ctypes.c_size_t, _P]
+_lib.sai_distill_target_window_range.restype = _I
 _lib.sai_count_valid_rows.argtypes = [_P, _I, _I, _I, _P, _P]
 _lib.sai_count_valid_rows.restype = _I
 _lib.sai_distill_kl_ex.argtypes = [_P, _P, _P, _I, _I, _I, _F, _P, _P, _P, _P, ctypes.c_size_t, _P]
@@ -317,6 +320,34 @@ def distill_target_window(Q: torch.Tensor, Kw: torch.Tensor, pool: torch.Tensor,
                _ptr(doc_start), B, S, H, D, K, int(cr), int(W), float(scale), _ptr(out), _ptr(wl_out), _ptr(err),
                _ptr(ws), nb)
     _check(st, "sai_distill_target_window")
+    return out
+
+
+def distill_target_window_range(Q: torch.Tensor, Kw: torch.Tensor, pool: torch.Tensor,
+                                idx: Optional[torch.Tensor], W: int, cr: int, scale: float, S_seq: int,
+                                t_begin: int, kw_lead: int, sink: Optional[torch.Tensor] = None,
+                                doc_start: Optional[torch.Tensor] = None, err: Optional[torch.Tensor] = None,
+                                out: Optional[torch.Tensor] = None, wl_out: Optional[torch.Tensor] = None,
+                                workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """p for sequence positions t_begin .. t_begin+S-1 of sequences of S_seq
+    tokens through sai_distill_target_window_range: Q, idx and doc_start are
+    the range's rows, Kw [B,S+kw_lead,D] the range's keys and its halo, pool
+    the whole sequence's [B,S_seq/cr,D]."""
+    B, S, H, D = Q.shape
+    Kw = _bf16_bits(Kw, "Kw")
+    if tuple(Kw.shape) != (B, S + kw_lead, D):
+        raise ValueError(f"Kw must be [B,S+kw_lead,D] = {(B, S + kw_lead, D)}, got {tuple(Kw.shape)}")
+    Q, pool, K, _, sink, _ = _target_inputs(Q, pool, idx, None, cr, sink, doc_start, err, False, False,
+                                            S_seq=S_seq, wl_from_kw=True)
+    if out is None:
+        out = torch.empty((B, S, K), dtype=torch.float32, device=Q.device)
+    _want(out, "out", torch.float32, (B, S, K))
+    _want(wl_out, "wl_out", torch.float32, (B, S, H))
+    ws, nb = _target_workspace(Q.device, B, S, H, D, K, workspace)
+    st = _call(_lib.sai_distill_target_window_range, Q.device, _ptr(Q), _ptr(Kw), _ptr(pool), _ptr(idx),
+               _ptr(sink), _ptr(doc_start), B, S, int(S_seq), int(t_begin), int(kw_lead), H, D, K, int(cr), int(W),
+               float(scale), _ptr(out), _ptr(wl_out), _ptr(err), _ptr(ws), nb)
+    _check(st, "sai_distill_target_window_range")
     return out
 
 

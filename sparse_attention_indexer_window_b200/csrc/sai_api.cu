@@ -435,16 +435,26 @@ size_t sai_distill_target_workspace_bytes(int B, int S, int H, int D, int K)
     return grid > 0 ? (size_t)grid * spf * sizeof(float) : 0;
 }
 
+sai_status sai_distill_target_window_range(const uint16_t *Q, const uint16_t *Kw, const uint16_t *pool,
+                                           const int32_t *idx, const float *sink, const int32_t *doc_start, int B,
+                                           int S, int S_seq, int t_begin, int kw_lead, int H, int D, int K, int cr,
+                                           int W, float scale, float *p, float *window_lse, int32_t *d_err,
+                                           void *workspace, size_t ws_bytes, void *stream)
+{
+    if (workspace && !al16(workspace))
+        return SAI_ERR_ALIGN;
+    const WinFuse wf = {Kw, W, kw_lead, window_lse};
+    return target_impl(Q, pool, idx, nullptr, sink, doc_start, B, S, S_seq, t_begin, H, D, K, cr, scale, 0u, p,
+                       d_err, reinterpret_cast<cudaStream_t>(stream), nullptr, workspace, ws_bytes, &wf);
+}
+
 sai_status sai_distill_target_window(const uint16_t *Q, const uint16_t *Kw, const uint16_t *pool,
                                      const int32_t *idx, const float *sink, const int32_t *doc_start, int B, int S,
                                      int H, int D, int K, int cr, int W, float scale, float *p, float *window_lse,
                                      int32_t *d_err, void *workspace, size_t ws_bytes, void *stream)
 {
-    if (workspace && !al16(workspace))
-        return SAI_ERR_ALIGN;
-    const WinFuse wf = {Kw, W, 0, window_lse};
-    return target_impl(Q, pool, idx, nullptr, sink, doc_start, B, S, S, 0, H, D, K, cr, scale, 0u, p, d_err,
-                       reinterpret_cast<cudaStream_t>(stream), nullptr, workspace, ws_bytes, &wf);
+    return sai_distill_target_window_range(Q, Kw, pool, idx, sink, doc_start, B, S, S, 0, 0, H, D, K, cr, W, scale,
+                                           p, window_lse, d_err, workspace, ws_bytes, stream);
 }
 
 sai_status sai_distill_target_ws(const uint16_t *Q, const uint16_t *pool, const int32_t *idx,

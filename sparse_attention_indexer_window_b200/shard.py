@@ -149,7 +149,7 @@ def range_views(t_begin: int, t_end: int, W: int, Q, Kw, idx, scores, valid, doc
 
 
 def sharded_distill_loss(calls, view, pool, *, S_seq: int, W: int, cr: int, scale: float, coeff: float,
-                         sink=None, err=None):
+                         sink=None, err=None, fused_window: bool = False):
     """One rank's share of the loss over a batch split by token range.
 
     ``calls`` provides window_lse_range, distill_target_range,
@@ -161,13 +161,22 @@ def sharded_distill_loss(calls, view, pool, *, S_seq: int, W: int, cr: int, scal
       distill_kl(n_rows=N)                       (dscores with the batch-wide 1/N)
       all-reduce(sum) of the loss shares         (the batch loss on every rank)
 
+    With fused_window=True the first two calls are one,
+    distill_target_window_range (the window band inside the target kernel,
+    Q read once), which also returns the window log-mass.
+
     Returns (loss [1], dscores, p, window_lse) with dscores, p and window_lse
     for this rank's positions. Every rank must call it (two collectives)."""
     t_begin = view["t_begin"]
-    wl = calls.window_lse_range(view["Q"], view["Kw"], W, scale, t_begin, view["kw_lead"],
-                                doc_start=view["doc_start"])
-    p = calls.distill_target_range(view["Q"], pool, view["idx"], wl, cr, scale, S_seq, t_begin, sink=sink,
-                                   doc_start=view["doc_start"], err=err)
+    if fused_window:
+        p, wl = calls.distill_target_window_range(view["Q"], view["Kw"], pool, view["idx"], W, cr, scale, S_seq,
+                                                  t_begin, view["kw_lead"], sink=sink, doc_start=view["doc_start"],
+                                                  err=err)
+    else:
+        wl = calls.window_lse_range(view["Q"], view["Kw"], W, scale, t_begin, view["kw_lead"],
+                                    doc_start=view["doc_start"])
+        p = calls.distill_target_range(view["Q"], pool, view["idx"], wl, cr, scale, S_seq, t_begin, sink=sink,
+                                       doc_start=view["doc_start"], err=err)
     n = calls.count_valid_rows(view["valid"])
     dist = _dist()
     if dist is not None and dist.get_world_size() > 1:

@@ -129,6 +129,18 @@ def test_distill_target_window_host_errors(sai):
     assert f(*args(wlo=FAKE + 2)) == 7               # window_lse out not 4-byte aligned
 
 
+def test_distill_target_window_range_host_errors(sai):
+    """The range form of the window-fused target: a halo shorter than the
+    window needs, or a range outside the sequence, is a shape error."""
+    f = sai.lib().sai_distill_target_window_range
+    args = lambda S=32, S_seq=64, t0=32, lead=15, W=16: (FAKE, FAKE, FAKE, FAKE, None, None, 1, S, S_seq, t0, lead,
+                                                         4, 32, 8, 4, W, 0.1, FAKE, None, None, None, 0, None)
+    assert f(*args(lead=10)) == 2                    # 10 halo keys, W - 1 = 15 needed
+    assert f(*args(lead=33)) == 2                    # more halo than positions before the range
+    assert f(*args(t0=40)) == 2                      # t_begin + S > S_seq
+    assert f(*args(W=129, lead=32)) == 3
+
+
 def test_distill_target_kl_host_errors(sai):
     """The fused target + KL call refuses missing KL buffers and a short or
     misaligned workspace before launching anything."""

@@ -73,6 +73,14 @@ class OracleRangeCalls:
         assert bad == 0
         return p.reshape(B, S, K)
 
+    def distill_target_window_range(self, Q, Kw, pool, idx, W, cr, scale, S_seq, t_begin, kw_lead, sink=None,
+                                    doc_start=None, err=None):
+        # the fused call's contract: (p, window log-mass) from the same inputs
+        wl = self.window_lse_range(Q, Kw, W, scale, t_begin, kw_lead, doc_start=doc_start)
+        p = self.distill_target_range(Q, pool, idx, wl, cr, scale, S_seq, t_begin, sink=sink, doc_start=doc_start,
+                                      err=err)
+        return p, wl
+
     def count_valid_rows(self, valid):
         import oracle
         return torch.tensor([oracle.count_valid_rows(valid)], dtype=torch.int64)
@@ -92,7 +100,7 @@ def _workload(name):
     return synth.make("packed", B=2, S=512, K=64, H=16, D=64, seed=32)
 
 
-def _rank_main(rank, world, port, out_dir, name, balanced):
+def _rank_main(rank, world, port, out_dir, name, balanced, fused=False):
     os.environ["MASTER_ADDR"] = "127.0.0.1"
     os.environ["MASTER_PORT"] = str(port)
     from datetime import timedelta
@@ -103,17 +111,21 @@ def _rank_main(rank, world, port, out_dir, name, balanced):
         t0, t1 = shard.token_ranges(w.S, world, cost)[rank]
         v = shard.range_views(t0, t1, w.W, w.Q, w.Kw, w.idx, w.scores, w.valid, w.doc_start)
         loss, ds, p, wl = shard.sharded_distill_loss(OracleRangeCalls(w.S), v, w.pool, S_seq=w.S, W=w.W, cr=w.cr,
-                                                     scale=w.scale, coeff=w.coeff, sink=w.sink)
+                                                     scale=w.scale, coeff=w.coeff, sink=w.sink,
+                                                     fused_window=fused)
         np.savez(os.path.join(out_dir, f"{name}_rank{rank}.npz"), loss=float(loss.item()), ds=ds, p=p, wl=wl,
                  t0=t0, t1=t1, kw_lead=v["kw_lead"], kw_rows=v["Kw"].shape[1])
     finally:
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("name,balanced", [("flash", True), ("packed", False)])
-def test_two_rank_token_range_split(tmp_path, name, balanced):
+@pytest.mark.parametrize("name,balanced,fused", [("flash", True, False), ("packed", False, False),
+                                                ("packed", True, True)])
+def test_two_rank_token_range_split(tmp_path, name, balanced, fused):
+    """fused: the rank's window and target come from the one window-fused
+    range call (shard.sharded_distill_loss(fused_window=True))."""
     world = 2
-    mp.start_processes(_rank_main, args=(world, _free_port(), str(tmp_path), name, balanced), nprocs=world,
+    mp.start_processes(_rank_main, args=(world, _free_port(), str(tmp_path), name, balanced, fused), nprocs=world,
                        join=True, start_method="spawn")
     import oracle
     w = _workload(name)
