@@ -19,7 +19,8 @@
  * sai_indexer_topk, the block selection that produces idx, scores and valid
  * from the indexer's scores, and the calls for splitting sequences across
  * GPUs by token range: sai_window_lse_range, sai_distill_target_range,
- * sai_count_valid_rows and sai_distill_kl_ex (a batch-wide N).
+ * sai_distill_target_window_range, sai_count_valid_rows and
+ * sai_distill_kl_ex (a batch-wide N).
  *
  * Conventions for every call
  *   - Tensor arguments are DEVICE pointers to dense row-major (C-contiguous)
