@@ -48,6 +48,14 @@
 // (sai_distill_target_kl), the epilogue then computes each row's KL and
 // dscores from the target in shared memory.
 //
+// Window-fused instantiation (WIN, sai_distill_target_window): each token
+// first runs one more tile, A = the 128 Kw rows ending at the token (one TMA
+// box per chunk, rows outside the window masked), against the same Q[t]
+// chunks; its per-head log-sum-exp is the window log-mass the joint merge
+// needs, so window_lse is not an input and Q is read once. TMEM is then a
+// ring of 512/H tile slots released one by one (TileRing), so the window
+// tile's slot is free again as soon as its statistics are taken.
+//
 // Epilogue arithmetic (one exponential per score):
 //   M[h] = max_k z[k,h]  (per 8 columns: each warp's maximum by one redux,
 //          then the four lane quarters merged per head through smem)
@@ -163,11 +171,7 @@ __device__ __forceinline__ bool selected(int j, int t, int d0, int P, int cr)
 // behind one barrier wait, one fence and one commit; on this part a commit
 // every 4 MMAs leaves the tensor pipe idle about half the time, so CPS = 2
 // whenever D allows it.
-// WIN: the window band is computed here too (sai_distill_target_window):
-// every token first runs one more tile, A = the 128 Kw rows ending at the
-// token (one TMA box per chunk), whose per-head log-sum-exp over the window
-// keys replaces the window_lse input; the TMEM is then a ring of tile slots
-// (TileRing) instead of two fixed accumulators.
+// WIN: the window-fused instantiation (window tile first, TMEM as TileRing).
 template <int HH, bool FUSE_KL, int CPS, bool SPILL, bool WIN>
 __global__ void __launch_bounds__(kTgtThreads, 1)
     target_tc_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapP,
