@@ -190,6 +190,26 @@ def test_multi_group_spill_matches_second_sweep(sai, K, S):
     assert_close("p", p1.cpu().numpy().reshape(-1, K)[tok], op, TOL_P)
 
 
+@pytest.mark.parametrize("fused", [False, True])
+def test_pro_shape_sampled(sai, fused):
+    """The V4-Pro head count with its 1024 pool entries (H=128, K=1024,
+    S=4096): two score tiles per TMEM group, so late tokens take four groups
+    through the raw-score spill. Both routes, against the oracle on the last
+    tokens and a sample of the rest."""
+    w = synth.make("flash", S=4096, K=1024, H=128, seed=2024)
+    t = to_dev(w)
+    if fused:
+        wl, p = run_fused(sai, w, t)
+    else:
+        wl = sai.window_lse(t["Q"], t["Kw"], w.W, w.scale)
+        p = sai.distill_target(t["Q"], t["pool"], t["idx"], wl, w.cr, w.scale, sink=t["sink"])
+        torch.cuda.synchronize()
+    tok = np.unique(np.concatenate([np.arange(w.S - 16, w.S), synth.sample_tokens(w.B, w.S, 32)]))
+    owl, op, _, _, _ = oracle.run_all(w, tok)
+    assert_close("window_lse", wl.cpu().numpy().reshape(-1, w.H)[tok] - owl, 0 * owl, tol_wl(owl))
+    assert_close("p", p.cpu().numpy().reshape(-1, w.K)[tok], op, TOL_P)
+
+
 def test_matches_three_call_route(sai):
     """The fused call and window_lse -> distill_target agree to within both
     routes' tolerance of the oracle, and the fused call is deterministic."""
