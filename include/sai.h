@@ -254,9 +254,11 @@ sai_status sai_distill_target_range(const uint16_t *Q, const uint16_t *pool, con
  *   sai_distill_target_ws(...): sai_distill_target_range plus the workspace.
  *     workspace: device memory, 16-byte aligned, owned by the caller, read
  *     and written by the kernel, no contents required or kept between calls;
- *     calls that overlap on the GPU must not share it. NULL, or ws_bytes
- *     below the size above: the second sweep is used, with identical
- *     results. Errors as for sai_distill_target_range, and SAI_ERR_ALIGN for
+ *     calls that overlap on the GPU must not share it. With it the last
+ *     group's scores also stay in tensor memory for their u pass. NULL, or
+ *     ws_bytes below the size above: the second sweep is used; the results
+ *     agree up to float32 rounding (the order and form of the exponentials
+ *     differ). Errors as for sai_distill_target_range, and SAI_ERR_ALIGN for
  *     a misaligned workspace.
  */
 size_t sai_distill_target_workspace_bytes(int B, int S, int H, int D, int K);

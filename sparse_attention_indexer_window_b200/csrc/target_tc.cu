@@ -43,7 +43,9 @@
 // pass over the groups merges per-head (max, sum-exp) statistics, a second
 // forms u. With a spill buffer (H >= 64, its own instantiation) the first
 // pass also stores each group's raw scores there and the second reads them
-// back, so every row is gathered and multiplied once; without one the second
+// back, so every row is gathered and multiplied once; the last group's
+// scores are not spilled but stay in TMEM, with their exponentials, for its
+// u pass, the first of the second pass. Without a spill buffer the second
 // pass gathers and multiplies each group again. When the KL stage is fused
 // (sai_distill_target_kl), the epilogue then computes each row's KL and
 // dscores from the target in shared memory.
@@ -820,6 +822,12 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
             // more than one group and a spill buffer: the second pass reads the
             // groups' raw scores back instead of waiting for them again
             const bool spill = kSpill && G > 1;
+            // with the spill: the last group's scores stay in TMEM (their
+            // exponentials stored there, as for a single group) until its u
+            // pass, the first of the second pass; only the earlier groups
+            // are spilled and read back
+            const bool keep = spill;
+            int mb_keep = 0, n0_keep = 0;
             float *scr = kSpill ? a.spill + (size_t)blockIdx.x * a.spill_stride : nullptr;
             float *prow = a.p + (size_t)g * K;
             const int32_t *sl = slot + m3 * Kp;
@@ -928,25 +936,34 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
                         continue;
                     }
                 }
-                for (int grp = 0; grp < G; ++grp) {
+                for (int gi = 0; gi < G; ++gi) {
+                    const int grp = (keep && pass == 1) ? (gi == 0 ? G - 1 : gi - 1) : gi;
                     const int i0 = grp * TB;
                     const int ntg = min(nt, i0 + TB) - i0;
                     // this warpgroup's tiles of the group: [t0, t1) (possibly empty)
                     const int t0 = hf * TBH;
                     const int t1 = min(ntg, t0 + TBH);
-                    const bool from_spill = spill && pass == 1;   // this group's scores are in scr
+                    const bool kept = keep && grp == G - 1;       // scores stay in TMEM across the passes
+                    const bool held = kept && pass == 1;          // waited for in the first pass
+                    const bool from_spill = spill && pass == 1 && !kept;   // this group's scores are in scr
                     // groups alternate between the two accumulators (a spilled
                     // group's second pass reads no accumulator)
-                    const int mb = gseq & 1;
-                    if (!from_spill)
+                    const int mb = held ? mb_keep : (gseq & 1);
+                    if (!from_spill && !held)
                         ++gseq;
                     const uint32_t tbase = tlane + mb * 256;
                     int n0 = 0;
                     if constexpr (WIN) {
-                        if (!from_spill) {
+                        if (held) {
+                            n0 = n0_keep;
+                        } else if (!from_spill) {
                             n0 = tn;
                             tn += ntg;
                         }
+                    }
+                    if (kept && pass == 0) {
+                        mb_keep = mb;
+                        n0_keep = n0;
                     }
                     // TMEM address of tile i of the group (this thread's lane quarter)
                     auto tcol = [&](int i) -> uint32_t {
@@ -955,7 +972,7 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
                         else
                             return tbase + (uint32_t)(i * HH);
                     };
-                    if (!from_spill) {
+                    if (!from_spill && !held) {
                         bool fa = true;
                         if (ew == 0) {
                             if constexpr (WIN) {
@@ -982,6 +999,7 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
                         tc_fence_after();
                     }
                     const bool single = (G == 1);
+                    const bool e_tmem = single || kept;   // exponentials kept in TMEM (H >= 64)
                     if constexpr (HH >= 32) {
                     if (pass == 0) {
                     if constexpr (TB <= 4) {
@@ -1002,7 +1020,7 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
                                 if (i < ntg)
                                     tmem_ld8(tcol(i) + col0, v[i]);
                             tmem_ld_wait();
-                            if (spill) {
+                            if (spill && !kept) {
                                 // raw scores, lane-contiguous per (tile, head)
 #pragma unroll
                                 for (int i = 0; i < TB; ++i)
@@ -1052,7 +1070,7 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
                                     }
                                 }
                             }
-                            if (single) {
+                            if (e_tmem) {
 #pragma unroll
                                 for (int i = 0; i < TB; ++i)
                                     if (i < ntg)
@@ -1064,7 +1082,7 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
                                 st.red_sum[q][col0 + lane] = red;
                             }
                         }
-                        if (single)
+                        if (e_tmem)
                             tmem_st_wait();
                         named_bar_sync(bar_id, kEpiThreads);
                         if (et < HH) {
@@ -1314,7 +1332,7 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
                     }
                     }
                     if (pass == passes - 1) {
-                        if (grp == 0) {
+                        if (gi == 0) {
                             // ---- per-head merge with the window and the sink
                             if (et < HH) {
                                 const float M = st.colM[et] * 0.69314718055994531f;  // natural log units
@@ -1345,10 +1363,10 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
                                 const float wp = expf(st.head_a[et] - At);
                                 st.wprime[et] = wp;
                                 if constexpr (HH >= 32 && TB <= 4) {
-                                    // a single group's e are relative to their lane
-                                    // quarter's maximum: fold the rescale to the head's
-                                    // maximum into the weight, per quarter
-                                    if (single) {
+                                    // a single (or the kept last) group's e are relative
+                                    // to their lane quarter's maximum: fold the rescale
+                                    // to the head's maximum into the weight, per quarter
+                                    if (single || keep) {
 #pragma unroll
                                         for (int w = 0; w < 4; ++w)
                                             st.red_max[w][et] = wp * exp2f(st.red_max[w][et] - st.colM[et]);
@@ -1371,8 +1389,8 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
                             float w16[16], cm16[16];
 #pragma unroll
                             for (int e = 0; e < 16; ++e) {
-                                w16[e] = (TB <= 4 && single) ? st.red_max[q][col0 + e] : st.wprime[col0 + e];
-                                cm16[e] = single ? 0.f : st.colM[col0 + e];
+                                w16[e] = (TB <= 4 && e_tmem) ? st.red_max[q][col0 + e] : st.wprime[col0 + e];
+                                cm16[e] = e_tmem ? 0.f : st.colM[col0 + e];
                             }
 #pragma unroll
                             for (int ib = 0; ib < TB; ib += IB) {
@@ -1399,7 +1417,7 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
                                 for (int i = 0; i < IB; ++i) {
                                     if (ib + i < ntg) {
                                         float acc = u[ib + i];
-                                        if (single) {
+                                        if (e_tmem) {
 #pragma unroll
                                             for (int e = 0; e < 16; ++e)
                                                 acc = fmaf(__uint_as_float(v[i][e]), w16[e], acc);
@@ -1478,7 +1496,7 @@ __global__ void __launch_bounds__(kTgtThreads, 1)
                         }
                         }
                     }
-                    if (!from_spill) {
+                    if (!from_spill && !(kept && pass == 0)) {   // the kept group is released after its u pass
                         tc_fence_before();
                         __syncwarp();
                         if (lane == 0) {

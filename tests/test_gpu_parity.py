@@ -190,10 +190,10 @@ def test_multi_group_tokens(sai):
 @pytest.mark.parametrize("K,S", [(576, 2304), (1000, 4096), (2048, 8192)])
 def test_spill_matches_second_sweep(sai, K, S):
     """Tokens of two to four TMEM groups (K > 512 at H=64): the target with its
-    raw-score spill (one sweep of gathers and MMAs) is bit-identical to the
-    two-sweep target without a workspace, and both match the oracle on late
-    tokens (the most groups) and a sample of the rest. K=1000 leaves a
-    ragged last group."""
+    raw-score spill (one sweep of gathers and MMAs, the last group kept in
+    TMEM) and the two-sweep target without a workspace agree within the
+    target's tolerance, and both match the oracle on late tokens (the most
+    groups) and a sample of the rest. K=1000 leaves a ragged last group."""
     w = workload(f"long_s{S}_k{K}", name="long", S=S, K=K)
     t = to_dev(w)
     B, H, D = w.B, w.H, w.D
@@ -210,10 +210,13 @@ def test_spill_matches_second_sweep(sai, K, S):
         ctypes.c_void_p(p_two.data_ptr()), None, None, 0, ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
     assert st == 0
     torch.cuda.synchronize()
-    assert torch.equal(p_ws, p_two)
+    pw, pt = p_ws.cpu().numpy(), p_two.cpu().numpy()
+    assert_close("p spill vs second sweep", pw, pt, TOL_P)
+    assert np.array_equal(pw == 0, pt == 0)   # the same masked slots
     tok = np.unique(np.concatenate([np.arange(w.S - 24, w.S), synth.sample_tokens(w.B, w.S, 24)]))
     _, op, _, _, _ = oracle.run_all(w, tok)
-    assert_close("p", p_ws.cpu().numpy().reshape(-1, w.K)[tok], op, TOL_P)
+    assert_close("p", pw.reshape(-1, w.K)[tok], op, TOL_P)
+    assert_close("p (second sweep)", pt.reshape(-1, w.K)[tok], op, TOL_P)
 
 
 def test_deterministic(sai):

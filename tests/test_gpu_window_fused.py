@@ -164,9 +164,10 @@ def test_dense_warm_up(sai):
 @pytest.mark.parametrize("K,S", [(576, 2304), (2048, 8192)])
 def test_multi_group_spill_matches_second_sweep(sai, K, S):
     """Two and four TMEM groups per late token (K > 512 at H=64): with the
-    spill workspace and without it (second sweep) the fused kernel's p and
-    window log-mass are bit-identical, and both match the oracle on late
-    tokens and a sample of the rest."""
+    spill workspace and without it (second sweep) the fused kernel's window
+    log-mass is bit-identical and its p agrees within the target's
+    tolerance; both match the oracle on late tokens and a sample of the
+    rest."""
     w = synth.make("long", S=S, K=K)
     t = to_dev(w)
     ws_bytes = sai.target_workspace_bytes(w.B, S, w.H, w.D, K)
@@ -183,11 +184,13 @@ def test_multi_group_spill_matches_second_sweep(sai, K, S):
         ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
     assert st == 0
     torch.cuda.synchronize()
-    assert torch.equal(p1, p2) and torch.equal(wl1, wl2)
+    assert torch.equal(wl1, wl2)
+    assert_close("p spill vs second sweep", p1.cpu().numpy(), p2.cpu().numpy(), TOL_P)
     tok = np.unique(np.concatenate([np.arange(S - 24, S), synth.sample_tokens(w.B, S, 24)]))
     owl, op, _, _, _ = oracle.run_all(w, tok)
     assert_close("window_lse", wl1.cpu().numpy().reshape(-1, w.H)[tok] - owl, 0 * owl, tol_wl(owl))
     assert_close("p", p1.cpu().numpy().reshape(-1, K)[tok], op, TOL_P)
+    assert_close("p (second sweep)", p2.cpu().numpy().reshape(-1, K)[tok], op, TOL_P)
 
 
 @pytest.mark.parametrize("fused", [False, True])
